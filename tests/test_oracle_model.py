@@ -1,0 +1,316 @@
+"""Pins of the model oracle: a pure-Python brute-force forward on micro shapes
+(explicit index loops, complex-number RoPE, Python sorting), plus invariants
+the pages fix -- 256-wide canvas, bidirectional canvas attention, causal
+prompt, top-k weights summing to 1, stop on low entropy (CPU only)."""
+import cmath
+import math
+
+import numpy as np
+import pytest
+
+from block_text_diffusion_b200 import inputs as I
+from oracle import model as om, sampler as sp
+
+F32 = np.float32
+
+MICRO = I.Workload("micro", n_layers=2, d_model=8, n_heads=2, n_kv_heads=1, head_dim=4,
+                   n_experts=4, top_k=2, d_ff=6, vocab=16, dtype=I.DTYPE_FP32, logit_scale=2.0,
+                   max_steps=4, weight_seed=21, sample_seed=5, prompt_len=5)
+
+
+class BruteWeights:
+    """Every weight fetched one by one by (tensor, row-major index)."""
+
+    def __init__(self, cfg):
+        self.cfg, self.cache = cfg, {}
+
+    def __call__(self, tid, idx, shape):
+        flat = 0
+        for i, n in zip(idx, shape):
+            assert 0 <= i < n
+            flat = flat * n + i
+        key = (tid, flat)
+        if key not in self.cache:
+            self.cache[key] = om.weight_element(self.cfg.weight_seed, tid, flat, bf16=False)
+        return self.cache[key]
+
+
+def r32(x):
+    return float(np.float32(x))
+
+
+def bf_block(cfg, W, l, h, positions, kpre, vpre, causal):
+    d, H, G, hd, E, ff = cfg.d_model, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.n_experts, cfg.d_ff
+    tid = lambda w: om.layer_tensor_id(l, w)
+    n = len(h)
+
+    def norm(v):
+        ms = sum(a * a for a in v) / len(v)
+        return [r32(a / math.sqrt(ms + cfg.rms_eps)) for a in v]
+
+    def rot(vec, pos):
+        out = list(vec)
+        for c in range(hd // 2):
+            z = complex(vec[c], vec[c + hd // 2]) * cmath.exp(1j * pos * cfg.rope_theta ** (-2 * c / hd))
+            out[c], out[c + hd // 2] = z.real, z.imag
+        return out
+
+    x = [norm(v) for v in h]
+    q = [[[r32(a) for a in rot([sum(W(tid("wq"), (hh * hd + c, i), (H * hd, d)) * x[t][i] for i in range(d))
+                                 for c in range(hd)], positions[t])] for hh in range(H)] for t in range(n)]
+    k = [[[r32(a) for a in rot([sum(W(tid("wk"), (g * hd + c, i), (G * hd, d)) * x[t][i] for i in range(d))
+                                 for c in range(hd)], positions[t])] for g in range(G)] for t in range(n)]
+    v = [[[r32(sum(W(tid("wv"), (g * hd + c, i), (G * hd, d)) * x[t][i] for i in range(d)))
+           for c in range(hd)] for g in range(G)] for t in range(n)]
+    keys = kpre + k
+    vals = vpre + v
+    o = []
+    for t in range(n):
+        row = []
+        for hh in range(H):
+            g = hh // (H // G)
+            vis = [j for j in range(len(keys)) if not causal or j <= len(kpre) + t]
+            sc = [sum(q[t][hh][c] * keys[j][g][c] for c in range(hd)) / math.sqrt(hd) for j in vis]
+            mx = max(sc)
+            ex = [math.exp(s - mx) for s in sc]
+            z = sum(ex)
+            row += [r32(sum(ex[a] / z * vals[j][g][c] for a, j in enumerate(vis))) for c in range(hd)]
+        o.append(row)
+    h = [[r32(h[t][i] + sum(W(tid("wo"), (i, c), (d, H * hd)) * o[t][c] for c in range(H * hd)))
+          for i in range(d)] for t in range(n)]
+    x2 = [norm(vv) for vv in h]
+    out = []
+    for t in range(n):
+        logit = [sum(W(tid("wr"), (e, i), (E, d)) * x2[t][i] for i in range(d)) for e in range(E)]
+        if cfg.zipf_s:
+            logit = [a - cfg.zipf_s * math.log(e + 1) for e, a in enumerate(logit)]
+        chosen = sorted(range(E), key=lambda e: (-logit[e], e))[:cfg.top_k]
+        mx = max(logit[e] for e in chosen)
+        gate = [math.exp(logit[e] - mx) for e in chosen]
+        gate = [a / sum(gate) for a in gate]
+        y = [0.0] * d
+        for e, w in zip(chosen, gate):
+            act = []
+            for f in range(ff):
+                gg = sum(W(tid("wg"), (e, f, i), (E, ff, d)) * x2[t][i] for i in range(d))
+                uu = sum(W(tid("wu"), (e, f, i), (E, ff, d)) * x2[t][i] for i in range(d))
+                act.append(r32(gg / (1 + math.exp(-gg)) * uu))
+            for i in range(d):
+                y[i] += w * sum(W(tid("wd"), (e, i, f), (E, d, ff)) * act[f] for f in range(ff))
+        out.append([r32(h[t][i] + y[i]) for i in range(d)])
+    return out, k, v
+
+
+def bf_embed(cfg, W, ids):
+    return [[W(om.T_EMBED, (int(t), i), (cfg.vocab, cfg.d_model)) for i in range(cfg.d_model)] for t in ids]
+
+
+def bf_encode(cfg, W, prompt):
+    h = bf_embed(cfg, W, prompt)
+    K, V = [], []
+    for l in range(cfg.n_layers):
+        h, k, v = bf_block(cfg, W, l, h, list(range(len(prompt))), [], [], causal=True)
+        K.append(k)
+        V.append(v)
+    return K, V
+
+
+def bf_logits(cfg, W, K, V, canvas, selfcond=None):
+    h = bf_embed(cfg, W, canvas)
+    if selfcond is not None:
+        h = [[r32(a + b) for a, b in zip(hr, sr)] for hr, sr in zip(h, selfcond)]
+    P = len(K[0])
+    for l in range(cfg.n_layers):
+        h, _, _ = bf_block(cfg, W, l, h, [P + t for t in range(len(canvas))], K[l], V[l], causal=False)
+    out = []
+    for vec in h:
+        ms = sum(a * a for a in vec) / len(vec)
+        x = [r32(a / math.sqrt(ms + cfg.rms_eps)) for a in vec]
+        out.append([cfg.logit_scale * sum(W(om.T_EMBED, (tok, i), (cfg.vocab, cfg.d_model)) * x[i]
+                                          for i in range(cfg.d_model)) for tok in range(cfg.vocab)])
+    return np.array(out)
+
+
+@pytest.fixture(scope="module")
+def micro():
+    cfg = MICRO
+    return cfg, om.Model(cfg), BruteWeights(cfg)
+
+
+def _cache_to_lists(K):
+    # oracle cache [L, Hkv, P, hd] -> brute [L][P][Hkv][hd]
+    return [[[list(map(float, K[l, g, p])) for g in range(K.shape[1])] for p in range(K.shape[2])]
+            for l in range(K.shape[0])]
+
+
+@pytest.mark.parametrize("zipf", [0.0, 1.1])
+def test_encode_and_canvas_forward_match_brute_force(micro, zipf):
+    cfg, model, W = micro
+    cfg = cfg.replace(zipf_s=zipf)
+    model.cfg = cfg
+    prompt = I.prompt_ids(1, 1, cfg.prompt_len, cfg.vocab)[0]
+    K, V = om.encode_prompt(model, prompt)
+    bK, bV = bf_encode(cfg, W, prompt)
+    assert np.allclose(K, np.array(bK).transpose(0, 2, 1, 3), rtol=1e-6, atol=1e-7)
+    assert np.allclose(V, np.array(bV).transpose(0, 2, 1, 3), rtol=1e-6, atol=1e-7)
+    canvas = I.canvas_ids(2, 1, cfg.vocab)[0]
+    sc = I.normal(3, 7, (256, cfg.d_model), std=0.05)
+    logits, _ = om.forward_canvas(model, K, V, canvas, sc)
+    ref = bf_logits(cfg, W, _cache_to_lists(K), _cache_to_lists(V), canvas, sc.tolist())
+    assert logits.shape == (256, cfg.vocab)
+    assert np.allclose(logits, ref, rtol=1e-5, atol=1e-6)
+    model.cfg = MICRO
+
+
+def test_self_conditioning_matches_brute_force(micro):
+    cfg, model, W = micro
+    p = np.abs(I.normal(4, 8, (256, cfg.vocab)))
+    p = (p / p.sum(axis=1, keepdims=True)).astype(F32)
+    s = om.self_condition(model, p)
+    d = cfg.d_model
+    for t in (0, 100, 255):
+        u = [r32(sum(float(p[t, v]) * W(om.T_EMBED, (v, i), (cfg.vocab, d)) for v in range(cfg.vocab)))
+             for i in range(d)]
+        ref = [r32(sum(W(om.T_WSC, (o, i), (d, d)) * u[i] for i in range(d))) for o in range(d)]
+        assert np.allclose(s[t], ref, rtol=1e-6, atol=1e-9)
+
+
+def test_canvas_is_256_wide_and_bidirectional(micro):
+    cfg, model, _ = micro
+    K, V = I.prompt_kv(1, cfg.n_layers, 1, cfg.n_kv_heads, 7, cfg.head_dim, bf16=False)
+    c = I.canvas_ids(3, 1, cfg.vocab)[0]
+    a, _ = om.forward_canvas(model, K[:, 0], V[:, 0], c, None)
+    c2 = c.copy()
+    c2[255] = (c2[255] + 1) % cfg.vocab
+    b, _ = om.forward_canvas(model, K[:, 0], V[:, 0], c2, None)
+    assert a.shape[0] == 256
+    # the first position sees the last one: bidirectional canvas attention
+    assert np.abs(a[0] - b[0]).max() > 1e-6
+
+
+def test_prompt_encode_is_causal(micro):
+    cfg, model, _ = micro
+    p = I.prompt_ids(5, 1, 9, cfg.vocab)[0]
+    K1, V1 = om.encode_prompt(model, p)
+    p2 = p.copy()
+    p2[-1] = (p2[-1] + 3) % cfg.vocab
+    K2, V2 = om.encode_prompt(model, p2)
+    assert np.array_equal(K1[:, :, :-1], K2[:, :, :-1]) and np.array_equal(V1[:, :, :-1], V2[:, :, :-1])
+    assert not np.array_equal(K1[:, :, -1], K2[:, :, -1])
+
+
+def test_attention_special_cases():
+    g = np.random.default_rng(0)
+    q = g.standard_normal((3, 4, 8))
+    k = g.standard_normal((1, 2, 8))
+    v = g.standard_normal((1, 2, 8))
+    o = om.attention(q, k, v)
+    # one key: the output is that value, for every query and head
+    assert np.allclose(o, np.repeat(v[:, [0, 0, 1, 1], :], 3, axis=0))
+    k = g.standard_normal((6, 2, 8))
+    v = g.standard_normal((6, 2, 8))
+    # causal: query 0 with no prefix sees key 0 only
+    oc = om.attention(q[:1], k, v, causal_offset=0)
+    assert np.allclose(oc[0], v[0, [0, 0, 1, 1]])
+    # bidirectional attention is invariant to permuting the keys with their values
+    perm = g.permutation(6)
+    assert np.allclose(om.attention(q, k, v), om.attention(q, k[perm], v[perm]))
+    # identical keys: uniform weights -> mean of the values
+    kk = np.repeat(k[:1], 6, axis=0)
+    assert np.allclose(om.attention(q, kk, v), np.repeat(v.mean(axis=0)[[0, 0, 1, 1]][None], 3, axis=0))
+
+
+def test_rope_rotation_properties():
+    g = np.random.default_rng(1)
+    x = g.standard_normal((5, 2, 16))
+    pos = np.array([0, 1, 7, 100, 33000])
+    r = om.rope(x, pos, 10000.0)
+    assert np.allclose(r[0], x[0])
+    assert np.allclose(np.linalg.norm(r, axis=-1), np.linalg.norm(x, axis=-1))
+    # relative position: <R_m q, R_n k> depends on m - n only
+    q, k = x[:1], x[1:2]
+    a = (om.rope(q, [10], 1e4) * om.rope(k, [3], 1e4)).sum()
+    b = (om.rope(q, [1010], 1e4) * om.rope(k, [1003], 1e4)).sum()
+    assert abs(a - b) < 1e-9
+
+
+def test_rmsnorm_unit_rms():
+    x = np.random.default_rng(2).standard_normal((4, 64)) * 7
+    y = om.rmsnorm(x, 0.0)
+    assert np.allclose(np.sqrt((y * y).mean(axis=1)), 1.0)
+
+
+def test_router_topk_weights_sum_to_one_and_ties():
+    g = np.random.default_rng(3)
+    x = g.standard_normal((50, 16))
+    wr = g.standard_normal((12, 16))
+    ids, w = om.router(x, wr, 8)
+    assert np.allclose(w.sum(axis=1), 1.0)
+    r = x @ wr.T
+    for t in range(50):
+        assert list(ids[t]) == list(np.argsort(-r[t], kind="stable")[:8])
+        assert np.all(np.diff(w[t]) <= 1e-15)
+    # all-equal logits: ties go to the lower ids, equal weights
+    ids, w = om.router(np.zeros((2, 16)), wr, 3)
+    assert ids.tolist() == [[0, 1, 2]] * 2 and np.allclose(w, 1 / 3)
+    # Zipf bias alone: experts 0..k-1, weights proportional to (e+1)^-s
+    ids, w = om.router(np.zeros((1, 16)), wr, 4, zipf_s=1.1)
+    ref = np.arange(1, 5) ** -1.1
+    assert ids.tolist() == [[0, 1, 2, 3]] and np.allclose(w[0], ref / ref.sum())
+
+
+def test_moe_all_experts_equal_gates_is_mean(micro):
+    cfg, model, _ = micro
+    layer = model.layers[0]
+    x = np.random.default_rng(4).standard_normal((5, cfg.d_model))
+    zero = om.Layer(**{**layer.__dict__, "wr": np.zeros_like(layer.wr)})
+    model.cfg = cfg.replace(top_k=cfg.n_experts)
+    y, ids, w = om.moe(model, zero, x)
+    model.cfg = cfg
+    ref = np.zeros_like(x)
+    for e in range(cfg.n_experts):
+        a = model.store(om.silu(x @ layer.wg[e].T.astype(np.float64)) * (x @ layer.wu[e].T.astype(np.float64)))
+        ref += a @ layer.wd[e].T.astype(np.float64)
+    assert np.allclose(y, ref / cfg.n_experts)
+
+
+def test_low_entropy_canvas_stops_at_first_round(micro):
+    # a huge logit scale makes every row one-hot: entropy ~0 -> all commit -> stop
+    cfg, model, _ = micro
+    model.cfg = cfg.replace(logit_scale=1e5)
+    K, V = I.prompt_kv(2, cfg.n_layers, 1, cfg.n_kv_heads, 4, cfg.head_dim, bf16=False)
+    r = om.generate_block(model, K[:, 0], V[:, 0])
+    model.cfg = cfg
+    assert r["steps_used"] == 1 and r["n_committed"] == 256
+    assert np.array_equal(r["canvas"], r["trace"][0]["amax"])
+
+
+def test_generate_runs_to_budget_when_uncertain(micro):
+    cfg, model, _ = micro
+    K, V = I.prompt_kv(2, cfg.n_layers, 1, cfg.n_kv_heads, 4, cfg.head_dim, bf16=False)
+    r = om.generate_block(model, K[:, 0], V[:, 0])
+    assert r["steps_used"] == cfg.max_steps
+    assert np.array_equal(r["canvas"], r["trace"][-1]["tokens"])
+    # round 0 used the uniform-noise canvas; later rounds the re-noised one
+    t0 = r["trace"][0]
+    assert np.array_equal(r["trace"][1]["canvas_next"].shape, (256,))
+    assert np.array_equal(t0["canvas_next"][t0["commit"] == 1], t0["tokens"][t0["commit"] == 1])
+
+
+def test_zero_selfcond_equals_none(micro):
+    cfg, model, _ = micro
+    K, V = I.prompt_kv(2, cfg.n_layers, 1, cfg.n_kv_heads, 4, cfg.head_dim, bf16=False)
+    c = I.canvas_ids(9, 1, cfg.vocab)[0]
+    a, _ = om.forward_canvas(model, K[:, 0], V[:, 0], c, None)
+    b, _ = om.forward_canvas(model, K[:, 0], V[:, 0], c, np.zeros((256, cfg.d_model)))
+    assert np.array_equal(a, b)
+
+
+def test_bf16_storage_rounds_values(micro):
+    cfg, _, _ = micro
+    m = om.Model(cfg.replace(dtype=I.DTYPE_BF16), layers=1)
+    w = m.layers[0].wg
+    assert np.array_equal(w.view(np.uint32) & np.uint32(0xFFFF), np.zeros_like(w.view(np.uint32)))
+    # bf16 spacing at 1 is 2^-7; exact ties go to the even mantissa
+    x = np.array([1.0 + 2 ** -9, 1.0 + 3 * 2 ** -9, -3.14159, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8])
+    assert np.array_equal(m.store(x), [1.0, 1.0 + 2 ** -7, -3.140625, 1.0, 1.0 + 2 ** -6])
