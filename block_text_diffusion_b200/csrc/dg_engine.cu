@@ -1,0 +1,932 @@
+// Host engine of the denoising step: model allocation and weight init,
+// TMA tensor maps, the per-layer launch sequence, the device block loop as a
+// CUDA graph with a while-condition node, and the C ABI (include/dg.h,
+// include/dg_test.h).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "../../include/dg_test.h"
+#include "dg_attn.cuh"
+#include "dg_device.cuh"
+#include "dg_gemm.cuh"
+#include "dg_kernels.cuh"
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Tensor maps through the driver entry point (no link-time libcuda need).
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encode)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                               CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                               CUtensorMapFloatOOBfill);
+
+PFN_encode encode_fn() {
+  static PFN_encode fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_encode)p;
+  }
+  return fn;
+}
+
+// 2D bf16 [rows][cols] row-major; box = 64 columns (128 B, swizzled) x box_rows.
+bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  PFN_encode enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D bf16 map; strides in bytes of dims 1 and 2.
+bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+           uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  PFN_encode enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+constexpr int kSMs = 148;
+constexpr int kCanvas = 256;
+constexpr int kEncodeChunk = 4096;
+
+// Launch bookkeeping: optional per-phase event timing and a launch counter.
+enum Phase {
+  PH_EMBED, PH_NORM, PH_QKV_GEMM, PH_QKV_POST, PH_ATTN, PH_ATTN_COMBINE, PH_O_GEMM, PH_RESIDUAL,
+  PH_ROUTER, PH_PERMUTE, PH_GATHER, PH_GU_GEMM, PH_SWIGLU, PH_DOWN_GEMM, PH_COMBINE, PH_LM_HEAD,
+  PH_SAMPLER, PH_COMMIT, PH_SC_GEMM, PH_SC_ROUND, PH_CONTROL, PH_COUNT
+};
+
+struct Prof {
+  bool on = false;
+  std::vector<int> phase;
+  std::vector<cudaEvent_t> ev;   // pairs
+};
+
+}  // namespace
+
+struct LayerW {
+  void *qkv = nullptr, *wo = nullptr, *wr = nullptr, *gu = nullptr, *wd = nullptr;
+  CUtensorMap tm_qkv, tm_wo, tm_gu, tm_wd;
+};
+
+struct dg_model {
+  dg_config c;
+  bool bf;
+  int esz;
+  int L, d, hq, hkv, hd, G, E, k, ff, V, nqkv;
+  int T_cap;         // canvas tokens (max_canvases * 256)
+  int Tw;            // token capacity of the layer workspace
+  size_t ws_elems, part_rows_cap;
+  std::vector<void*> allocs;
+  cudaStream_t cap_stream = nullptr;
+
+  void *emb = nullptr, *embT = nullptr, *Wsc = nullptr;
+  std::vector<LayerW> layers;
+  float2* rope = nullptr;
+  double* rbias = nullptr;
+  CUtensorMap tm_E, tm_ET, tm_Wsc;
+
+  void *h = nullptr, *x = nullptr, *q = nullptr, *o = nullptr, *xp = nullptr, *act = nullptr;
+  void *probs = nullptr, *u = nullptr, *sc = nullptr;
+  CUtensorMap tm_x, tm_o, tm_xp, tm_act, tm_probs, tm_u;
+  float* ws = nullptr;
+  float *o_part = nullptr, *lse_part = nullptr;
+  int *ids = nullptr, *perm = nullptr, *inv = nullptr, *work_count = nullptr, *counts = nullptr;
+  float* gate = nullptr;
+  int4* work = nullptr;
+  float *logits = nullptr, *H = nullptr;
+  int *tok = nullptr, *amax = nullptr, *prev_amax = nullptr;
+  int *canvas_cur = nullptr, *done = nullptr, *steps_used = nullptr, *ncom_out = nullptr,
+      *canvas_out = nullptr;
+  DevState* st = nullptr;
+
+  // cached block-loop graph
+  cudaGraphExec_t gexec = nullptr;
+  cudaGraph_t graph = nullptr;
+  void* g_kv = nullptr;
+  int g_B = -1, g_P = -1;
+  int launches_per_round = 0;
+
+  Prof prof;
+  int launch_count = 0;
+  int cur_phase = PH_CONTROL;
+};
+
+namespace {
+
+dg_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DG_OK;
+  if (e == cudaErrorMemoryAllocation) return DG_ERR_OOM;
+  return DG_ERR_CUDA;
+}
+
+#define DG_TRY(x)                              \
+  do {                                         \
+    dg_status _s = (x);                        \
+    if (_s != DG_OK) return _s;                \
+  } while (0)
+#define CU_TRY(x)                              \
+  do {                                         \
+    cudaError_t _e = (x);                      \
+    if (_e != cudaSuccess) return cuda_status(_e); \
+  } while (0)
+
+dg_status dalloc(dg_model* m, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return e == cudaErrorMemoryAllocation ? DG_ERR_OOM : DG_ERR_CUDA;
+  }
+  m->allocs.push_back(*p);
+  return DG_OK;
+}
+template <typename P>
+dg_status dalloc_t(dg_model* m, P** p, size_t count) {
+  return dalloc(m, (void**)p, count * sizeof(P));
+}
+
+// Per-launch hooks: count launches; in profiling mode bracket each launch
+// with events on its stream.
+struct LaunchScope {
+  dg_model* m;
+  cudaStream_t s;
+  int idx = -1;
+  LaunchScope(dg_model* mm, cudaStream_t ss, int phase) : m(mm), s(ss) {
+    m->launch_count++;
+    if (m->prof.on) {
+      cudaEvent_t a, b;
+      cudaEventCreate(&a);
+      cudaEventCreate(&b);
+      m->prof.ev.push_back(a);
+      m->prof.ev.push_back(b);
+      m->prof.phase.push_back(phase);
+      idx = (int)m->prof.phase.size() - 1;
+      cudaEventRecord(a, s);
+    }
+  }
+  ~LaunchScope() {
+    if (idx >= 0) cudaEventRecord(m->prof.ev[2 * idx + 1], s);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// GEMM launcher.
+// ---------------------------------------------------------------------------
+struct GemmCall {
+  const CUtensorMap* tA = nullptr;   // bf16 path
+  const CUtensorMap* tB = nullptr;
+  const float* A32 = nullptr;        // fp32 path
+  const float* B32 = nullptr;
+  long long lda = 0, ldb = 0;
+  int M = 0, K = 0, N = 0;
+  int splits = 1;
+  float alpha = 1.0f;
+  float* out = nullptr;
+  long long ldo = 0, split_stride = 0;
+  const int4* work = nullptr;        // grouped
+  const int* work_count = nullptr;
+  int a_group_rows = 0;
+  int max_items = 0;
+  int bn = 256;
+};
+
+template <int BN, int ST>
+dg_status launch_tc(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
+  using C = GemmTcCfg<BN, ST>;
+  static bool attr = false;
+  if (!attr) {
+    CU_TRY(cudaFuncSetAttribute(k_gemm_tc<BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
+    attr = true;
+  }
+  const int items = g.work ? g.max_items : cdiv(g.N, a.n_tile);
+  const long long grid = (long long)a.m_tiles * a.k_splits * items;
+  if (grid <= 0) return DG_OK;
+  if (grid > 0x7FFFFFFFLL) return DG_ERR_UNSUPPORTED;
+  k_gemm_tc<BN, ST><<<(unsigned)grid, 128, C::kSmem, s>>>(*g.tA, *g.tB, a);
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
+  LaunchScope ls(m, s, phase);
+  GemmArgs a{};
+  a.M = g.M;
+  a.kb_total = cdiv(g.K, 64);
+  a.k_splits = std::max(1, std::min(g.splits, a.kb_total));
+  a.N = g.N;
+  a.alpha = g.alpha;
+  a.out = g.out;
+  a.ldo = g.ldo;
+  a.split_stride = g.split_stride;
+  a.work = g.work;
+  a.work_count = g.work_count;
+  a.a_group_rows = g.a_group_rows;
+  a.err = &m->st->err;
+  if (!m->bf) {
+    a.m_tiles = cdiv(g.M, 64);
+    a.n_tile = 64;
+    const int items = g.work ? g.max_items : cdiv(g.N, 64);
+    const long long grid = (long long)a.m_tiles * a.k_splits * items;
+    if (grid <= 0) return DG_OK;
+    k_gemm_f32<<<(unsigned)grid, 256, 0, s>>>(g.A32, g.lda, g.B32, g.ldb, g.K, a);
+    CU_TRY(cudaGetLastError());
+    return DG_OK;
+  }
+  a.m_tiles = cdiv(g.M, 128);
+  a.n_tile = g.bn;
+  switch (g.bn) {
+    case 256: return launch_tc<256, 4>(g, a, s);
+    case 128: return launch_tc<128, 5>(g, a, s);
+    case 64: return launch_tc<64, 4>(g, a, s);
+    case 32: return launch_tc<32, 6>(g, a, s);
+    default: return DG_ERR_UNSUPPORTED;
+  }
+}
+
+// Split-K factor so that a dense GEMM fills about two waves of CTAs.
+int pick_splits(int m_tiles, int n_items, int kb_total, int cap) {
+  const int base = m_tiles * n_items;
+  int s = std::max(1, (2 * kSMs) / std::max(1, base));
+  s = std::min(s, std::max(1, kb_total / 4));
+  return std::min(s, cap);
+}
+
+int dense_bn(int N) {
+  if (N <= 32) return 32;
+  if (N <= 64) return 64;
+  if (N <= 128) return 128;
+  return 256;
+}
+
+// ---------------------------------------------------------------------------
+// Validation.
+// ---------------------------------------------------------------------------
+bool config_ok(const dg_config& c) {
+  if (c.canvas_len != kCanvas) return false;
+  if (c.n_layers < 1 || c.d_model < 64 || c.d_model % 64) return false;
+  if (c.n_heads < 1 || c.n_kv_heads < 1 || c.n_heads % c.n_kv_heads) return false;
+  const int G = c.n_heads / c.n_kv_heads;
+  if (128 % G) return false;
+  if (c.head_dim != 64 && c.head_dim != 128) return false;
+  if (c.dtype == DG_BF16 && c.head_dim != 128) return false;
+  if (c.dtype != DG_BF16 && c.dtype != DG_FP32) return false;
+  if (c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 || c.top_k > c.n_experts || c.top_k > 64)
+    return false;
+  if (c.d_ff < 64 || c.d_ff % 64) return false;
+  if (c.vocab < 64 || c.vocab % 64) return false;
+  if (c.max_canvases < 1 || c.max_canvases > 4096 || c.max_prompt < 1 || c.max_prompt > (1 << 20)) return false;
+  if (c.max_steps < 1) return false;
+  if (c.commit_mode != DG_COMMIT_THRESH && c.commit_mode != DG_COMMIT_EB) return false;
+  if (c.stop_mode != DG_STOP_MEAN && c.stop_mode != DG_STOP_EB) return false;
+  if (!(c.logit_scale == c.logit_scale) || !(c.rope_theta > 0.0f) || !(c.rms_eps >= 0.0f)) return false;
+  return true;
+}
+
+// Tensor ids of the weight generator (shared numbering with the published
+// recipe): 0 = embedding E [V, d], 1 = W_sc [d, d]; layer l uses 16 + 16 l
+// + {0 Wq, 1 Wk, 2 Wv, 3 Wo, 4 Wr, 5 Wg, 6 Wu, 7 Wd}.
+uint32_t tid_layer(int l, int which) { return 16u + 16u * (uint32_t)l + (uint32_t)which; }
+
+template <typename T>
+void init_tensor(T* out, uint64_t n, uint64_t inner, uint64_t outer, uint64_t offset, uint64_t seed,
+                 uint32_t tid, cudaStream_t s) {
+  const int grid = (int)std::min<uint64_t>((n + 255) / 256, 148ull * 64);
+  k_init_weights<T><<<grid, 256, 0, s>>>(out, n, inner, outer, offset, seed, tid);
+}
+
+template <typename T>
+dg_status init_all_weights(dg_model* m, uint64_t seed, cudaStream_t s) {
+  const uint64_t d = m->d, V = m->V, hd = m->hd;
+  const uint64_t nq = (uint64_t)m->hq * hd, nk = (uint64_t)m->hkv * hd;
+  init_tensor<T>((T*)m->emb, V * d, V * d, V * d, 0, seed, 0, s);
+  {
+    const int grid = (int)std::min<uint64_t>((V * d + 255) / 256, 148ull * 64);
+    k_init_weights_t<T><<<grid, 256, 0, s>>>((T*)m->embT, V, d, seed, 0);
+  }
+  init_tensor<T>((T*)m->Wsc, d * d, d * d, d * d, 0, seed, 1, s);
+  const uint64_t E = m->E, ff = m->ff;
+  for (int l = 0; l < m->L; ++l) {
+    LayerW& w = m->layers[l];
+    init_tensor<T>((T*)w.qkv, nq * d, nq * d, nq * d, 0, seed, tid_layer(l, 0), s);
+    init_tensor<T>((T*)w.qkv, nk * d, nk * d, nk * d, nq * d, seed, tid_layer(l, 1), s);
+    init_tensor<T>((T*)w.qkv, nk * d, nk * d, nk * d, (nq + nk) * d, seed, tid_layer(l, 2), s);
+    init_tensor<T>((T*)w.wo, d * nq, d * nq, d * nq, 0, seed, tid_layer(l, 3), s);
+    init_tensor<T>((T*)w.wr, E * d, E * d, E * d, 0, seed, tid_layer(l, 4), s);
+    init_tensor<T>((T*)w.gu, E * ff * d, ff * d, 2 * ff * d, 0, seed, tid_layer(l, 5), s);
+    init_tensor<T>((T*)w.gu, E * ff * d, ff * d, 2 * ff * d, ff * d, seed, tid_layer(l, 6), s);
+    init_tensor<T>((T*)w.wd, E * d * ff, E * d * ff, E * d * ff, 0, seed, tid_layer(l, 7), s);
+  }
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+dg_status build_maps(dg_model* m) {
+  if (!m->bf) return DG_OK;
+  const uint64_t d = m->d, V = m->V;
+  bool ok = true;
+  ok &= map2d(&m->tm_E, m->emb, V, d, 128);
+  ok &= map2d(&m->tm_ET, m->embT, d, V, 128);
+  ok &= map2d(&m->tm_Wsc, m->Wsc, d, d, 128);
+  for (int l = 0; l < m->L; ++l) {
+    LayerW& w = m->layers[l];
+    ok &= map2d(&w.tm_qkv, w.qkv, m->nqkv, d, 128);
+    ok &= map2d(&w.tm_wo, w.wo, d, (uint64_t)m->hq * m->hd, 128);
+    ok &= map2d(&w.tm_gu, w.gu, (uint64_t)m->E * 2 * m->ff, d, 128);
+    ok &= map2d(&w.tm_wd, w.wd, (uint64_t)m->E * d, m->ff, 128);
+  }
+  const uint64_t Tw = m->Tw, Tk = (uint64_t)m->Tw * m->k;
+  ok &= map2d(&m->tm_x, m->x, Tw, d, kBoxRowsB);
+  ok &= map2d(&m->tm_o, m->o, Tw, (uint64_t)m->hq * m->hd, kBoxRowsB);
+  ok &= map2d(&m->tm_xp, m->xp, Tk, d, kBoxRowsB);
+  ok &= map2d(&m->tm_act, m->act, Tk, m->ff, kBoxRowsB);
+  ok &= map2d(&m->tm_probs, m->probs, m->T_cap, V, kBoxRowsB);
+  ok &= map2d(&m->tm_u, m->u, m->T_cap, d, kBoxRowsB);
+  return ok ? DG_OK : DG_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// KV cache geometry and attention maps.
+// ---------------------------------------------------------------------------
+struct KvGeom {
+  int B, P, S;
+  void* K;
+  void* Vt;
+};
+
+KvGeom kv_geom(const dg_model* m, void* kv, int B, int P) {
+  KvGeom g;
+  g.B = B;
+  g.P = P;
+  g.S = ((P + kCanvas + 63) / 64) * 64;
+  g.K = kv;
+  g.Vt = (uint8_t*)kv + (size_t)m->L * B * m->hkv * g.S * m->hd * m->esz;
+  return g;
+}
+
+struct AttnMaps {
+  CUtensorMap q, k, v;
+};
+
+bool attn_maps(const dg_model* m, const KvGeom& g, int n_keys, int T_q, AttnMaps& am) {
+  const uint64_t hd = m->hd, lbh = (uint64_t)m->L * g.B * m->hkv;
+  bool ok = map3d(&am.q, m->q, hd, m->hq, T_q, hd * 2, (uint64_t)m->hq * hd * 2, 64, m->G, 128 / m->G);
+  ok &= map3d(&am.k, g.K, hd, n_keys, lbh, hd * 2, (uint64_t)g.S * hd * 2, 64, 128, 1);
+  ok &= map3d(&am.v, g.Vt, n_keys, hd, lbh, (uint64_t)g.S * 2, (uint64_t)hd * g.S * 2, 64, 128, 1);
+  return ok;
+}
+
+// ---------------------------------------------------------------------------
+// One transformer layer stack over `T` tokens of `n_canvas` canvases
+// (n_per tokens each, positions pos0..), writing keys/values into the cache.
+// ---------------------------------------------------------------------------
+template <typename T>
+dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_per, int pos0, int n_keys,
+                     bool causal, cudaStream_t s) {
+  const int Tn = n_canvas * n_per;
+  const int d = m->d, nq = m->hq * m->hd;
+  AttnMaps am;
+  if (m->bf && !attn_maps(m, g, n_keys, Tn, am)) return DG_ERR_CUDA;
+  const int n_pairs = Tn * m->k;
+  const int bn_g = m->bf ? (n_pairs / m->E <= 48 ? 64 : (n_pairs / m->E <= 100 ? 128 : 256)) : 64;
+  const int max_items = m->E + cdiv(n_pairs, bn_g);
+
+  for (int l = 0; l < m->L; ++l) {
+    const LayerW& w = m->layers[l];
+    { LaunchScope ls(m, s, PH_NORM);
+      k_rmsnorm<T><<<Tn, 256, 0, s>>>((const T*)m->h, (T*)m->x, d, m->c.rms_eps); }
+    // QKV projection
+    GemmCall qc;
+    qc.tA = &w.tm_qkv; qc.tB = &m->tm_x; qc.A32 = (const float*)w.qkv; qc.B32 = (const float*)m->x;
+    qc.lda = d; qc.ldb = d; qc.M = m->nqkv; qc.K = d; qc.N = Tn; qc.out = m->ws; qc.ldo = m->nqkv;
+    qc.bn = dense_bn(Tn);
+    {
+      const int mt = m->bf ? cdiv(qc.M, 128) : cdiv(qc.M, 64);
+      const int items = m->bf ? cdiv(Tn, qc.bn) : cdiv(Tn, 64);
+      qc.splits = pick_splits(mt, items, cdiv(d, 64), 8);
+      while (qc.splits > 1 && (size_t)qc.splits * Tn * m->nqkv > m->ws_elems) --qc.splits;
+      qc.split_stride = (long long)Tn * m->nqkv;
+    }
+    DG_TRY(gemm(m, qc, PH_QKV_GEMM, s));
+    {
+      LaunchScope ls(m, s, PH_QKV_POST);
+      QkvPostArgs qa;
+      qa.ws = m->ws; qa.split_stride = qc.split_stride; qa.splits = std::min(qc.splits, cdiv(d, 64));
+      qa.Hq = m->hq; qa.Hkv = m->hkv; qa.hd = m->hd; qa.n_per = n_per; qa.pos0 = pos0; qa.b0 = b0;
+      qa.B = g.B; qa.layer = l; qa.S = g.S; qa.rope = m->rope;
+      k_qkv_post<T><<<Tn, 256, 0, s>>>(qa, (T*)m->q, (T*)g.K, (T*)g.Vt);
+    }
+    // attention
+    AttnArgs aa{};
+    aa.n_q = n_per; aa.q_pos0 = pos0; aa.n_keys = n_keys; aa.causal = causal ? 1 : 0;
+    aa.G = m->G; aa.Hq = m->hq; aa.Hkv = m->hkv; aa.lbh0 = (l * g.B + b0) * m->hkv;
+    aa.n_canvas = n_canvas; aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->hd));
+    aa.o_part = m->o_part; aa.lse_part = m->lse_part; aa.err = &m->st->err;
+    const long long rows = (long long)Tn * m->hq;
+    {
+      LaunchScope ls(m, s, PH_ATTN);
+      if (m->bf) {
+        aa.q_tiles = cdiv((long long)n_per * m->G, 128);
+        const int nblocks = cdiv(n_keys, 128);
+        const int base = aa.q_tiles * m->hkv * n_canvas;
+        int splits = std::max(1, std::min(nblocks, cdiv(2 * kSMs, base)));
+        while (splits > 1 && (size_t)splits * rows > m->part_rows_cap) --splits;
+        aa.blocks_per_split = cdiv(nblocks, splits);
+        aa.n_splits = cdiv(nblocks, aa.blocks_per_split);
+        static bool attr = false;
+        if (!attr) {
+          CU_TRY(cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem));
+          attr = true;
+        }
+        k_attn_tc<<<base * aa.n_splits, kAttnThreads, kAttnSmem, s>>>(am.q, am.k, am.v, aa);
+      } else {
+        aa.q_tiles = 1; aa.n_splits = 1; aa.blocks_per_split = 1;
+        const long long threads = rows * 32;
+        k_attn_f32<<<cdiv(threads, 256), 256, 0, s>>>((const float*)m->q, (const float*)g.K,
+                                                      (const float*)g.Vt, g.S, m->hd, aa);
+      }
+      CU_TRY(cudaGetLastError());
+    }
+    { LaunchScope ls(m, s, PH_ATTN_COMBINE);
+      k_attn_combine<T><<<(unsigned)rows, 128, 0, s>>>(m->o_part, m->lse_part, aa.n_splits, rows, m->hd,
+                                                        (T*)m->o); }
+    // output projection + residual
+    GemmCall oc;
+    oc.tA = &w.tm_wo; oc.tB = &m->tm_o; oc.A32 = (const float*)w.wo; oc.B32 = (const float*)m->o;
+    oc.lda = nq; oc.ldb = nq; oc.M = d; oc.K = nq; oc.N = Tn; oc.out = m->ws; oc.ldo = d;
+    oc.bn = dense_bn(Tn);
+    {
+      const int mt = m->bf ? cdiv(d, 128) : cdiv(d, 64);
+      const int items = m->bf ? cdiv(Tn, oc.bn) : cdiv(Tn, 64);
+      oc.splits = pick_splits(mt, items, cdiv(nq, 64), 8);
+      while (oc.splits > 1 && (size_t)oc.splits * Tn * d > m->ws_elems) --oc.splits;
+      oc.split_stride = (long long)Tn * d;
+    }
+    DG_TRY(gemm(m, oc, PH_O_GEMM, s));
+    { LaunchScope ls(m, s, PH_RESIDUAL);
+      const long long n = (long long)Tn * d;
+      k_residual<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(
+          (T*)m->h, m->ws, oc.split_stride, std::min(oc.splits, cdiv(nq, 64)), n); }
+    // MoE
+    { LaunchScope ls(m, s, PH_NORM);
+      k_rmsnorm<T><<<Tn, 256, 0, s>>>((const T*)m->h, (T*)m->x, d, m->c.rms_eps); }
+    { LaunchScope ls(m, s, PH_ROUTER);
+      const size_t sm = (size_t)(d + m->E) * sizeof(double);
+      k_router<T><<<Tn, 256, sm, s>>>((const T*)m->x, (const T*)w.wr, m->rbias, d, m->E, m->k, m->ids,
+                                       m->gate); }
+    { LaunchScope ls(m, s, PH_PERMUTE);
+      k_permute<<<1, 1024, (2 * m->E + 1) * sizeof(int), s>>>(m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
+                                                             m->work, m->work_count, m->counts, &m->st->err); }
+    { LaunchScope ls(m, s, PH_GATHER);
+      k_gather<T><<<n_pairs, 128, 0, s>>>((const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
+    GemmCall gu;
+    gu.tA = &w.tm_gu; gu.tB = &m->tm_xp; gu.A32 = (const float*)w.gu; gu.B32 = (const float*)m->xp;
+    gu.lda = d; gu.ldb = d; gu.M = 2 * m->ff; gu.K = d; gu.out = m->ws; gu.ldo = 2 * m->ff;
+    gu.work = m->work; gu.work_count = m->work_count; gu.a_group_rows = 2 * m->ff;
+    gu.max_items = max_items; gu.bn = bn_g;
+    DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
+    { LaunchScope ls(m, s, PH_SWIGLU);
+      const long long n = (long long)n_pairs * m->ff;
+      k_swiglu<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(m->ws, m->ff, n, (T*)m->act); }
+    GemmCall dn;
+    dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
+    dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;
+    dn.work = m->work; dn.work_count = m->work_count; dn.a_group_rows = d;
+    dn.max_items = max_items; dn.bn = bn_g;
+    DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
+    { LaunchScope ls(m, s, PH_COMBINE);
+      k_moe_combine<T><<<Tn, 256, 0, s>>>((T*)m->h, m->ws, m->inv, m->gate, m->k, d); }
+  }
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+// Output pointers of one round (single-step or block-loop mode).
+struct RoundIO {
+  const int* canvas;         // input tokens [B*256]
+  const void* selfcond;      // input self-conditioning or null
+  const int* use_sc;         // device flag gating selfcond (block loop) or null
+  float* logits;             // [B*256*V]
+  float* entropy;
+  int* tokens;
+  int* argmax;
+  uint8_t* commit;
+  int* canvas_next;
+  void* selfcond_next;       // null: skip the self-conditioning GEMMs
+  int* stop;
+  int* n_committed;
+  int step_override;         // >= 0 single step
+  float t_override;
+  bool loop;
+};
+
+template <typename T>
+dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_t s) {
+  const int B = g.B, Tn = B * kCanvas, d = m->d, V = m->V;
+  { LaunchScope ls(m, s, PH_EMBED);
+    k_embed<T><<<Tn, 256, 0, s>>>(io.canvas, (const T*)m->emb, (const T*)io.selfcond, io.use_sc, (T*)m->h, d,
+                                  V, &m->st->err); }
+  DG_TRY(run_layers<T>(m, g, 0, B, kCanvas, g.P, g.P + kCanvas, false, s));
+  { LaunchScope ls(m, s, PH_NORM);
+    k_rmsnorm<T><<<Tn, 256, 0, s>>>((const T*)m->h, (T*)m->x, d, m->c.rms_eps); }
+  // LM head (tied embedding) with the logit scale
+  GemmCall lc;
+  lc.tA = &m->tm_E; lc.tB = &m->tm_x; lc.A32 = (const float*)m->emb; lc.B32 = (const float*)m->x;
+  lc.lda = d; lc.ldb = d; lc.M = V; lc.K = d; lc.N = Tn; lc.alpha = m->c.logit_scale;
+  lc.out = io.logits; lc.ldo = V; lc.bn = dense_bn(Tn); lc.splits = 1;
+  DG_TRY(gemm(m, lc, PH_LM_HEAD, s));
+  // vocab sampler
+  {
+    LaunchScope ls(m, s, PH_SAMPLER);
+    SamplerArgs sa{};
+    sa.logits = io.logits; sa.vocab = V; sa.positions = kCanvas; sa.seed = m->c.sample_seed;
+    sa.temp_start = m->c.temp_start; sa.temp_end = m->c.temp_end; sa.state = m->st;
+    sa.step_override = io.step_override; sa.t_override = io.t_override;
+    sa.H = io.entropy; sa.tok = io.tokens; sa.amax = io.argmax;
+    k_sampler<T><<<Tn, 512, 0, s>>>(sa, io.selfcond_next ? (T*)m->probs : nullptr);
+  }
+  // commit / re-noise / stop
+  {
+    LaunchScope ls(m, s, PH_COMMIT);
+    CommitArgs ca{};
+    ca.H = io.entropy; ca.tok = io.tokens; ca.amax = io.argmax; ca.prev_amax = m->prev_amax; ca.vocab = V;
+    ca.seed = m->c.sample_seed; ca.commit_mode = m->c.commit_mode; ca.commit_bound = m->c.commit_bound;
+    ca.stop_mode = m->c.stop_mode; ca.stop_bound = m->c.stop_bound;
+    ca.max_steps = io.loop ? 0 : m->c.max_steps;
+    ca.state = m->st; ca.step_override = io.step_override;
+    ca.commit = io.commit; ca.canvas_next = io.canvas_next; ca.stop = io.stop; ca.n_committed = io.n_committed;
+    if (io.loop) {
+      ca.max_steps = -1;   // replaced below by the state's budget
+      ca.canvas_cur = m->canvas_cur; ca.done = m->done; ca.steps_used = m->steps_used;
+      ca.n_committed_out = m->ncom_out; ca.canvas_out = m->canvas_out;
+    }
+    ca.max_steps = io.loop ? m->c.max_steps : m->c.max_steps;
+    k_commit<<<B, 256, 0, s>>>(ca);
+  }
+  // self-conditioning for the next round: s' = round(round(p E) W_sc^T)
+  if (io.selfcond_next) {
+    GemmCall sc;
+    sc.tA = &m->tm_ET; sc.tB = &m->tm_probs; sc.A32 = (const float*)m->embT; sc.B32 = (const float*)m->probs;
+    sc.lda = V; sc.ldb = V; sc.M = d; sc.K = V; sc.N = Tn; sc.out = m->ws; sc.ldo = d; sc.bn = dense_bn(Tn);
+    {
+      const int mt = m->bf ? cdiv(d, 128) : cdiv(d, 64);
+      const int items = m->bf ? cdiv(Tn, sc.bn) : cdiv(Tn, 64);
+      sc.splits = pick_splits(mt, items, cdiv(V, 64), 16);
+      while (sc.splits > 1 && (size_t)sc.splits * Tn * d > m->ws_elems) --sc.splits;
+      sc.split_stride = (long long)Tn * d;
+    }
+    DG_TRY(gemm(m, sc, PH_SC_GEMM, s));
+    const long long n = (long long)Tn * d;
+    { LaunchScope ls(m, s, PH_SC_ROUND);
+      k_sum_round<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(
+          (T*)m->u, m->ws, sc.split_stride, std::min(sc.splits, cdiv(V, 64)), n); }
+    GemmCall s2;
+    s2.tA = &m->tm_Wsc; s2.tB = &m->tm_u; s2.A32 = (const float*)m->Wsc; s2.B32 = (const float*)m->u;
+    s2.lda = d; s2.ldb = d; s2.M = d; s2.K = d; s2.N = Tn; s2.out = m->ws; s2.ldo = d; s2.bn = dense_bn(Tn);
+    {
+      const int mt = m->bf ? cdiv(d, 128) : cdiv(d, 64);
+      const int items = m->bf ? cdiv(Tn, s2.bn) : cdiv(Tn, 64);
+      s2.splits = pick_splits(mt, items, cdiv(d, 64), 8);
+      while (s2.splits > 1 && (size_t)s2.splits * Tn * d > m->ws_elems) --s2.splits;
+      s2.split_stride = (long long)Tn * d;
+    }
+    DG_TRY(gemm(m, s2, PH_SC_GEMM, s));
+    { LaunchScope ls(m, s, PH_SC_ROUND);
+      k_sum_round<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(
+          (T*)io.selfcond_next, m->ws, s2.split_stride, std::min(s2.splits, cdiv(d, 64)), n); }
+  }
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+dg_status check_shape(const dg_model* m, int B, int P) {
+  if (B < 1 || B > m->c.max_canvases || P < 1 || P > m->c.max_prompt) return DG_ERR_INVALID_ARG;
+  return DG_OK;
+}
+
+void release_graph(dg_model* m) {
+  if (m->gexec) cudaGraphExecDestroy(m->gexec);
+  if (m->graph) cudaGraphDestroy(m->graph);
+  m->gexec = nullptr;
+  m->graph = nullptr;
+  m->g_kv = nullptr;
+  m->g_B = m->g_P = -1;
+}
+
+template <typename T>
+dg_status capture_block_graph(dg_model* m, const KvGeom& g) {
+  release_graph(m);
+  cudaStream_t cs = m->cap_stream;
+  cudaGraph_t graph;
+  CU_TRY(cudaGraphCreate(&graph, 0));
+  cudaGraphConditionalHandle handle;
+  cudaError_t e = cudaGraphConditionalHandleCreate(&handle, graph, 1, cudaGraphCondAssignDefault);
+  if (e != cudaSuccess) { cudaGraphDestroy(graph); return cuda_status(e); }
+  cudaGraphNodeParams np{};
+  np.type = cudaGraphNodeTypeConditional;
+  np.conditional.handle = handle;
+  np.conditional.type = cudaGraphCondTypeWhile;
+  np.conditional.size = 1;
+  cudaGraphNode_t node;
+  e = cudaGraphAddNode(&node, graph, nullptr, 0, &np);
+  if (e != cudaSuccess) { cudaGraphDestroy(graph); return cuda_status(e); }
+  cudaGraph_t body = np.conditional.phGraph_out[0];
+  e = cudaStreamBeginCaptureToGraph(cs, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) { cudaGraphDestroy(graph); return cuda_status(e); }
+  const int before = m->launch_count;
+  {
+    LaunchScope ls(m, cs, PH_CONTROL);
+    k_round_begin<<<1, 1, 0, cs>>>(m->st);
+  }
+  RoundIO io{};
+  io.canvas = m->canvas_cur;
+  io.selfcond = m->sc;
+  io.use_sc = &m->st->use_selfcond;
+  io.logits = m->logits; io.entropy = m->H; io.tokens = m->tok; io.argmax = m->amax;
+  io.selfcond_next = m->sc;
+  io.step_override = -1;
+  io.loop = true;
+  dg_status st = run_round<T>(m, g, io, cs);
+  {
+    LaunchScope ls(m, cs, PH_CONTROL);
+    k_round_end_cond<<<1, 1, 0, cs>>>(m->st, handle);
+  }
+  cudaGraph_t captured = nullptr;
+  e = cudaStreamEndCapture(cs, &captured);
+  if (st != DG_OK || e != cudaSuccess) {
+    cudaGraphDestroy(graph);
+    return st != DG_OK ? st : cuda_status(e);
+  }
+  m->launches_per_round = m->launch_count - before;
+  e = cudaGraphInstantiate(&m->gexec, graph, 0);
+  if (e != cudaSuccess) { cudaGraphDestroy(graph); m->gexec = nullptr; return cuda_status(e); }
+  m->graph = graph;
+  return DG_OK;
+}
+
+dg_status latched(dg_model* m, cudaStream_t s) {
+  int err = 0;
+  CU_TRY(cudaMemcpyAsync(&err, &m->st->err, sizeof(int), cudaMemcpyDeviceToHost, s));
+  CU_TRY(cudaStreamSynchronize(s));
+  if (err) {
+    CU_TRY(cudaMemsetAsync(&m->st->err, 0, sizeof(int), s));
+    CU_TRY(cudaStreamSynchronize(s));
+    return err == DGDEV_BAD_INDEX ? DG_ERR_STATE : DG_ERR_TIMEOUT;
+  }
+  return DG_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* dg_status_string(dg_status s) {
+  switch (s) {
+    case DG_OK: return "ok";
+    case DG_ERR_INVALID_ARG: return "invalid argument";
+    case DG_ERR_OOM: return "out of device memory";
+    case DG_ERR_CUDA: return "CUDA error";
+    case DG_ERR_TIMEOUT: return "device wait timed out";
+    case DG_ERR_STATE: return "invalid state or device-side index error";
+    case DG_ERR_UNSUPPORTED: return "unsupported shape or feature";
+  }
+  return "unknown status";
+}
+
+dg_status dg_free(dg_model* m) {
+  if (!m) return DG_OK;
+  cudaDeviceSynchronize();
+  release_graph(m);
+  for (void* p : m->allocs) cudaFree(p);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+  for (cudaEvent_t e : m->prof.ev) cudaEventDestroy(e);
+  delete m;
+  return DG_OK;
+}
+
+dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_model** out) {
+  if (!cfg || !out) return DG_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!config_ok(*cfg)) return DG_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  dg_model* m = new (std::nothrow) dg_model();
+  if (!m) return DG_ERR_OOM;
+  m->c = *cfg;
+  m->bf = cfg->dtype == DG_BF16;
+  m->esz = m->bf ? 2 : 4;
+  m->L = cfg->n_layers; m->d = cfg->d_model; m->hq = cfg->n_heads; m->hkv = cfg->n_kv_heads;
+  m->hd = cfg->head_dim; m->G = m->hq / m->hkv; m->E = cfg->n_experts; m->k = cfg->top_k;
+  m->ff = cfg->d_ff; m->V = cfg->vocab;
+  m->nqkv = (m->hq + 2 * m->hkv) * m->hd;
+  m->T_cap = cfg->max_canvases * kCanvas;
+  m->Tw = std::max(m->T_cap, std::min(cfg->max_prompt, kEncodeChunk));
+  m->Tw = ((m->Tw + 127) / 128) * 128;
+  const size_t es = m->esz;
+  const size_t d = m->d, V = m->V, Tw = m->Tw, Tk = (size_t)m->Tw * m->k;
+  {
+    size_t w = 8 * Tw * (size_t)m->nqkv;
+    w = std::max(w, 8 * Tw * d);
+    w = std::max(w, Tk * 2 * m->ff);
+    w = std::max(w, Tk * d);
+    w = std::max(w, 16 * (size_t)m->T_cap * d);
+    m->ws_elems = w;
+    m->part_rows_cap = 8 * Tw * (size_t)m->hq;
+  }
+  dg_status st = DG_OK;
+  auto A = [&](void** p, size_t bytes) { if (st == DG_OK) st = dalloc(m, p, bytes); };
+  A(&m->emb, V * d * es);
+  A(&m->embT, V * d * es);
+  A(&m->Wsc, d * d * es);
+  m->layers.resize(m->L);
+  const size_t nq = (size_t)m->hq * m->hd;
+  for (int l = 0; l < m->L; ++l) {
+    LayerW& w = m->layers[l];
+    A(&w.qkv, (size_t)m->nqkv * d * es);
+    A(&w.wo, d * nq * es);
+    A(&w.wr, (size_t)m->E * d * es);
+    A(&w.gu, (size_t)m->E * 2 * m->ff * d * es);
+    A(&w.wd, (size_t)m->E * d * m->ff * es);
+  }
+  const int max_pos = cfg->max_prompt + kCanvas;
+  A((void**)&m->rope, (size_t)max_pos * (m->hd / 2) * sizeof(float2));
+  A((void**)&m->rbias, (size_t)m->E * sizeof(double));
+  A(&m->h, Tw * d * es);
+  A(&m->x, Tw * d * es);
+  A(&m->q, Tw * nq * es);
+  A(&m->o, Tw * nq * es);
+  A(&m->xp, Tk * d * es);
+  A(&m->act, Tk * m->ff * es);
+  A(&m->probs, (size_t)m->T_cap * V * es);
+  A(&m->u, (size_t)m->T_cap * d * es);
+  A(&m->sc, (size_t)m->T_cap * d * es);
+  A((void**)&m->ws, m->ws_elems * sizeof(float));
+  A((void**)&m->o_part, m->part_rows_cap * m->hd * sizeof(float));
+  A((void**)&m->lse_part, m->part_rows_cap * sizeof(float));
+  A((void**)&m->ids, Tk * sizeof(int));
+  A((void**)&m->gate, Tk * sizeof(float));
+  A((void**)&m->perm, Tk * sizeof(int));
+  A((void**)&m->inv, Tk * sizeof(int));
+  A((void**)&m->work, ((size_t)m->E + Tk / 16 + 8) * sizeof(int4));
+  A((void**)&m->work_count, sizeof(int));
+  A((void**)&m->counts, (size_t)m->E * sizeof(int));
+  A((void**)&m->logits, (size_t)m->T_cap * V * sizeof(float));
+  A((void**)&m->H, (size_t)m->T_cap * sizeof(float));
+  A((void**)&m->tok, (size_t)m->T_cap * sizeof(int));
+  A((void**)&m->amax, (size_t)m->T_cap * sizeof(int));
+  A((void**)&m->prev_amax, (size_t)m->T_cap * sizeof(int));
+  A((void**)&m->canvas_cur, (size_t)m->T_cap * sizeof(int));
+  A((void**)&m->canvas_out, (size_t)m->T_cap * sizeof(int));
+  A((void**)&m->done, (size_t)cfg->max_canvases * sizeof(int));
+  A((void**)&m->steps_used, (size_t)cfg->max_canvases * sizeof(int));
+  A((void**)&m->ncom_out, (size_t)cfg->max_canvases * sizeof(int));
+  A((void**)&m->st, sizeof(DevState));
+  if (st != DG_OK) { dg_free(m); return st; }
+  if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    dg_free(m);
+    return DG_ERR_CUDA;
+  }
+  cudaMemsetAsync(m->st, 0, sizeof(DevState), s);
+  cudaMemsetAsync(m->prev_amax, 0xFF, (size_t)m->T_cap * sizeof(int), s);
+  cudaMemsetAsync(m->sc, 0, (size_t)m->T_cap * d * es, s);
+  st = m->bf ? init_all_weights<bf16>(m, seed, s) : init_all_weights<float>(m, seed, s);
+  if (st == DG_OK) {
+    const int n = max_pos * (m->hd / 2);
+    k_rope_table<<<cdiv(n, 256), 256, 0, s>>>(m->rope, max_pos, m->hd / 2, m->hd, (double)cfg->rope_theta);
+    k_router_bias<<<cdiv(m->E, 128), 128, 0, s>>>(m->rbias, m->E, (double)cfg->zipf_s);
+    if (cudaGetLastError() != cudaSuccess) st = DG_ERR_CUDA;
+  }
+  if (st == DG_OK) st = build_maps(m);
+  if (st == DG_OK && cudaStreamSynchronize(s) != cudaSuccess) st = DG_ERR_CUDA;
+  if (st != DG_OK) { dg_free(m); return st; }
+  *out = m;
+  return DG_OK;
+}
+
+size_t dg_kv_bytes(const dg_model* m, int32_t B, int32_t P) {
+  if (!m || check_shape(m, B, P) != DG_OK) return 0;
+  const size_t S = ((size_t)(P + kCanvas + 63) / 64) * 64;
+  return 2 * (size_t)m->L * B * m->hkv * S * m->hd * m->esz;
+}
+
+int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
+  if (!m) return 0;
+  (void)B; (void)P;
+  // per layer: norm, qkv gemm, qkv post, attention, combine, o gemm, residual,
+  // norm, router, permute, gather, gate/up gemm, swiglu, down gemm, combine
+  return 15 * m->L + 1 /*embed*/ + 1 /*norm*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
+         4 /*self-conditioning*/;
+}
+
+dg_status dg_encode_prompt(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, void* kv, void* stream) {
+  if (!m || !prompt || !kv) return DG_ERR_INVALID_ARG;
+  DG_TRY(check_shape(m, B, P));
+  cudaStream_t s = (cudaStream_t)stream;
+  const KvGeom g = kv_geom(m, kv, B, P);
+  CU_TRY(cudaMemsetAsync(kv, 0, dg_kv_bytes(m, B, P), s));
+  const int chunk = std::min(P, m->Tw);
+  for (int b = 0; b < B; ++b) {
+    for (int c0 = 0; c0 < P; c0 += chunk) {
+      const int n = std::min(chunk, P - c0);
+      {
+        LaunchScope ls(m, s, PH_EMBED);
+        if (m->bf)
+          k_embed<bf16><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const bf16*)m->emb, nullptr, nullptr,
+                                         (bf16*)m->h, m->d, m->V, &m->st->err);
+        else
+          k_embed<float><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const float*)m->emb, nullptr, nullptr,
+                                          (float*)m->h, m->d, m->V, &m->st->err);
+      }
+      dg_status st = m->bf ? run_layers<bf16>(m, g, b, 1, n, c0, c0 + n, true, s)
+                           : run_layers<float>(m, g, b, 1, n, c0, c0 + n, true, s);
+      if (st != DG_OK) return st;
+    }
+  }
+  return DG_OK;
+}
+
+dg_status dg_denoise_step(dg_model* m, void* kv, int32_t B, int32_t P, const int32_t* canvas,
+                          const void* selfcond, int32_t step, float t, const dg_step_out* out, void* stream) {
+  if (!m || !kv || !canvas || !out || !out->tokens) return DG_ERR_INVALID_ARG;
+  DG_TRY(check_shape(m, B, P));
+  if (step < 0 || !(t >= 0.0f && t <= 1.0f)) return DG_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const KvGeom g = kv_geom(m, kv, B, P);
+  RoundIO io{};
+  io.canvas = canvas;
+  io.selfcond = selfcond;
+  io.use_sc = nullptr;
+  io.logits = out->logits ? out->logits : m->logits;
+  io.entropy = out->entropy ? out->entropy : m->H;
+  io.tokens = out->tokens;
+  io.argmax = out->argmax ? out->argmax : m->amax;
+  io.commit = out->commit;
+  io.canvas_next = out->canvas_next;
+  io.selfcond_next = out->selfcond_next;
+  io.stop = out->stop;
+  io.n_committed = out->n_committed;
+  io.step_override = step;
+  io.t_override = t;
+  io.loop = false;
+  { LaunchScope ls(m, s, PH_CONTROL);
+    k_set_round<<<1, 1, 0, s>>>(m->st, step, t, selfcond ? 1 : 0); }
+  return m->bf ? run_round<bf16>(m, g, io, s) : run_round<float>(m, g, io, s);
+}
+
+dg_status dg_generate_block(dg_model* m, void* kv, int32_t B, int32_t P, int32_t* canvas_out, int32_t* steps_used,
+                            int32_t* n_committed, void* stream) {
+  if (!m || !kv || !canvas_out || !steps_used || !n_committed) return DG_ERR_INVALID_ARG;
+  DG_TRY(check_shape(m, B, P));
+  cudaStream_t s = (cudaStream_t)stream;
+  const KvGeom g = kv_geom(m, kv, B, P);
+  if (!m->gexec || m->g_kv != kv || m->g_B != B || m->g_P != P) {
+    dg_status st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
+    if (st != DG_OK) return st;
+    m->g_kv = kv; m->g_B = B; m->g_P = P;
+  }
+  { LaunchScope ls(m, s, PH_CONTROL);
+    k_loop_init<<<B, 256, 0, s>>>(m->st, m->c.max_steps, B, m->canvas_cur, m->done, m->steps_used, m->ncom_out,
+                                  m->prev_amax, m->c.sample_seed, m->V); }
+  CU_TRY(cudaGraphLaunch(m->gexec, s));
+  CU_TRY(cudaMemcpyAsync(canvas_out, m->canvas_out, (size_t)B * kCanvas * sizeof(int), cudaMemcpyDeviceToDevice, s));
+  CU_TRY(cudaMemcpyAsync(steps_used, m->steps_used, (size_t)B * sizeof(int), cudaMemcpyDeviceToDevice, s));
+  CU_TRY(cudaMemcpyAsync(n_committed, m->ncom_out, (size_t)B * sizeof(int), cudaMemcpyDeviceToDevice, s));
+  return DG_OK;
+}
+
+dg_status dg_sync_status(dg_model* m, void* stream) {
+  if (!m) return DG_ERR_INVALID_ARG;
+  return latched(m, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+#include "dg_test_api.inc"

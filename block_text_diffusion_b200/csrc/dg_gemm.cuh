@@ -1,0 +1,237 @@
+// GEMMs of the denoising step.
+//
+// Every projection is computed "swap-AB": out[n][m] = alpha * sum_k A[m][k] B[n][k]
+// with A a weight matrix stored [out_features][in_features] (K-major) and B the
+// activations [tokens][in_features] (K-major).  Weights fill the 128-row M side
+// of tcgen05.mma, tokens the N side (16..256), so a 256-token canvas streams
+// every weight byte exactly once and a small expert group (16 rows) still uses
+// full-height MMA tiles.
+//
+// Work items.  Dense launches tile N by blockIdx; grouped (MoE) launches read
+// work items (group, b_row0, n_valid, out_row0) built on the device by the
+// permute kernel, one per (expert, token tile).  Split-K writes fp32 partials
+// to out + split * split_stride; consumers sum the splits in index order.
+#pragma once
+#include "dg_device.cuh"
+
+struct GemmArgs {
+  int M;                   // valid A rows per work item
+  int m_tiles;             // ceil(M / tile M)
+  int kb_total;            // number of 64-wide K blocks
+  int k_splits;            // split-K factor (k blocks divided evenly, last takes the rest)
+  int N;                   // dense: total B rows
+  int n_tile;              // dense: B rows per CTA
+  float alpha;
+  float* out;
+  long long ldo;           // out row stride (elements)
+  long long split_stride;  // elements between split-K partial outputs
+  const int4* work;        // grouped: (group, b_row0, n_valid, out_row0); nullptr = dense
+  int a_group_rows;        // grouped: A rows per group (a_row0 = group * a_group_rows)
+  const int* work_count;
+  const int* skip;         // optional device flag: nonzero -> every CTA returns at once
+  int* err;
+};
+
+struct GemmTile {
+  int m_tile, split, a_row0, b_row0, n_valid, out_row0;
+};
+
+__device__ __forceinline__ bool gemm_decode(const GemmArgs& p, GemmTile& t) {
+  const int bid = blockIdx.x;
+  t.m_tile = bid % p.m_tiles;
+  const int r = bid / p.m_tiles;
+  t.split = r % p.k_splits;
+  const int item = r / p.k_splits;
+  if (p.work) {
+    if (item >= *p.work_count) return false;
+    const int4 w = p.work[item];
+    t.a_row0 = w.x * p.a_group_rows; t.b_row0 = w.y; t.n_valid = w.z; t.out_row0 = w.w;
+  } else {
+    const int n0 = item * p.n_tile;
+    t.a_row0 = 0; t.b_row0 = n0; t.out_row0 = n0;
+    t.n_valid = min(p.n_tile, p.N - n0);
+  }
+  return t.n_valid > 0;
+}
+
+__device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
+  const int per = p.kb_total / p.k_splits;
+  kb0 = split * per;
+  kb1 = (split == p.k_splits - 1) ? p.kb_total : kb0 + per;
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM, bf16 in / fp32 out.  128 threads: warp 0 lane 0 issues TMA,
+// warp 1 lane 0 issues MMAs, then all four warps drain TMEM (warp w owns
+// accumulator rows 32w..32w+31).  A tiles 128 x 64, B tiles BN x 64 loaded
+// 16 rows per TMA box; STAGES-deep mbarrier ring.
+// ---------------------------------------------------------------------------
+constexpr int kBoxRowsB = 16;
+
+template <int BN, int STAGES>
+struct GemmTcCfg {
+  static constexpr int kABytes = 128 * 128;          // 128 rows x 64 bf16
+  static constexpr int kBBytes = BN * 128;           // BN rows x 64 bf16
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kTmemCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+  static constexpr int kSmem = STAGES * kStage + 1024;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(128, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          GemmArgs p) {
+  using C = GemmTcCfg<BN, STAGES>;
+  if (p.skip && *p.skip) return;
+  GemmTile t;
+  if (!gemm_decode(p, t)) return;
+  int kb0, kb1;
+  split_range(p, t.split, kb0, kb1);
+  const int nkb = kb1 - kb0;
+  const int n_mma = min(BN, (t.n_valid + 15) & ~15);
+  const int n_boxes = n_mma / kBoxRowsB;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], done_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const int m0 = t.m_tile * 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (i >= STAGES && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) {
+          abort_flag = 1;
+          break;
+        }
+        uint8_t* a_s = smem + s * C::kStage;
+        uint8_t* b_s = a_s + C::kABytes;
+        const int kx = (kb0 + i) * 64;
+        mbar_expect_tx(&full_bar[s], tx);
+        tma_load_2d(a_s, &tmA, kx, t.a_row0 + m0, &full_bar[s]);
+        for (int j = 0; j < n_boxes; ++j)
+          tma_load_2d(b_s + j * kBoxRowsB * 128, &tmB, kx, t.b_row0 + j * kBoxRowsB, &full_bar[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, n_mma);
+      bool ok = true;
+      for (int i = 0; i < nkb && ok; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&full_bar[s], ph, p.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+        const uint32_t b_addr = a_addr + C::kABytes;
+        const uint64_t ad = sdesc_sw128(a_addr), bd = sdesc_sw128(b_addr);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_bf16(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (i | kk) != 0);
+        tc_commit(&empty_bar[s]);
+      }
+      // Completes when every MMA above has finished (also on the abort path).
+      tc_commit(&done_bar);
+    }
+    __syncwarp();
+  }
+
+  // Epilogue: TMEM -> registers -> out[(out_row0 + n) * ldo + m0 + row].
+  const bool ok = mbar_wait(&done_bar, 0, p.err, DGDEV_TIMEOUT_EPI);
+  tc_fence_after();
+  if (ok && nkb > 0) {
+    const int row = warp * 32 + lane;
+    const bool m_ok = (m0 + row) < p.M;
+    float* outp = p.out + (long long)t.split * p.split_stride + (long long)t.out_row0 * p.ldo + m0 + row;
+    for (int c0 = 0; c0 < n_mma; c0 += 16) {
+      float v[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
+      if (m_ok) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < t.n_valid) outp[(long long)(c0 + j) * p.ldo] = v[j] * p.alpha;
+      }
+    }
+  } else if (nkb == 0 && ok) {
+    const int row = warp * 32 + lane;
+    if ((m0 + row) < p.M) {
+      float* outp = p.out + (long long)t.split * p.split_stride + (long long)t.out_row0 * p.ldo + m0 + row;
+      for (int n = 0; n < t.n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// fp32 SIMT GEMM with the same contract (the fp32 workload's projections):
+// 64 x 64 output tile per CTA, 256 threads, 4 x 4 outputs per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_gemm_f32(const float* __restrict__ A, long long lda, const float* __restrict__ B, long long ldb,
+           int K, GemmArgs p) {
+  if (p.skip && *p.skip) return;
+  GemmTile t;
+  if (!gemm_decode(p, t)) return;
+  int kb0, kb1;
+  split_range(p, t.split, kb0, kb1);
+  const int k_begin = kb0 * 64, k_end = min(K, kb1 * 64);
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int m0 = t.m_tile * 64;
+  float acc[4][4] = {};
+  for (int k0 = k_begin; k0 < k_end; k0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int kk = i % 16, r = i / 16;
+      const int k = k0 + kk;
+      const int am = m0 + r;
+      As[kk][r] = (k < k_end && am < p.M) ? A[(long long)(t.a_row0 + am) * lda + k] : 0.0f;
+      Bs[kk][r] = (k < k_end && r < t.n_valid) ? B[(long long)(t.b_row0 + r) * ldb + k] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* outp = p.out + (long long)t.split * p.split_stride;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= p.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = tx * 4 + j;
+      if (n < t.n_valid) outp[(long long)(t.out_row0 + n) * p.ldo + m] = acc[i][j] * p.alpha;
+    }
+  }
+}

@@ -1,0 +1,653 @@
+// Memory-bound and integer kernels of the denoising step.
+#pragma once
+#include "dg_device.cuh"
+
+// Device-resident loop state, read by every kernel that depends on the round.
+struct DevState {
+  int step;           // current round s
+  float t;            // diffusion time of the round (1 -> 0)
+  int n_steps;        // round budget N
+  int use_selfcond;   // 0 at round 0 (self-conditioning input is zero)
+  int active;         // number of canvases not yet stopped
+  int cond;           // 1 while the block loop should continue
+  int err;            // first device error code
+  int pad;
+};
+
+// ---------------------------------------------------------------------------
+// Weight initialisation: w = round(0.02 * sqrt(-2 ln u1) * cos(2 pi u2)),
+// u1/u2 from words 0/1 of Philox(key = seed, ctr = (j lo, j hi, tensor, 3)),
+// j the element's row-major index in its logical tensor.  `outer`/`inner`
+// place logical element j at physical index (j / inner) * outer + j % inner
+// + offset, which packs gate/up experts and the fused QKV matrix.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float init_value(uint64_t j, uint64_t seed, uint32_t tensor_id) {
+  const uint4 w = philox4x32_10(make_uint4((uint32_t)j, (uint32_t)(j >> 32), tensor_id, STREAM_WEIGHTS),
+                                (uint32_t)seed, (uint32_t)(seed >> 32));
+  const float u1 = uniform_open(w.x), u2 = uniform_open(w.y);
+  const float r = __fsqrt_rn(__fmul_rn(dg_logf(u1), -2.0f));
+  const float z = __fmul_rn(r, dg_cos2pif(u2));
+  return __fmul_rn(DG_F(0x3CA3D70Au), z);   // 0.02f
+}
+
+template <typename T>
+__global__ void k_init_weights(T* __restrict__ out, uint64_t n, uint64_t inner, uint64_t outer,
+                               uint64_t offset, uint64_t seed, uint32_t tensor_id) {
+  for (uint64_t j = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; j < n;
+       j += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t phys = (j / inner) * outer + (j % inner) + offset;
+    out[phys] = from_f<T>(init_value(j, seed, tensor_id));
+  }
+}
+
+// Transposed copy of a logical [rows][cols] tensor: out[c][r] = w(r * cols + c).
+template <typename T>
+__global__ void k_init_weights_t(T* __restrict__ out, uint64_t rows, uint64_t cols, uint64_t seed,
+                                 uint32_t tensor_id) {
+  const uint64_t n = rows * cols;
+  for (uint64_t p = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; p < n;
+       p += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t c = p / rows, r = p % rows;
+    out[p] = from_f<T>(init_value(r * cols + c, seed, tensor_id));
+  }
+}
+
+// RoPE table: (cos, sin) of pos * theta^(-2i/hd) in fp64, stored fp32.
+__global__ void k_rope_table(float2* __restrict__ tab, int n_pos, int half, int hd, double theta) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pos * half) return;
+  const int pos = i / half, c = i % half;
+  const double ang = (double)pos * pow(theta, -2.0 * c / hd);
+  double s, co;
+  sincos(ang, &s, &co);
+  tab[i] = make_float2((float)co, (float)s);
+}
+
+// Router bias b_e = -s ln(e + 1) (Zipf-skewed expert popularity), fp64.
+__global__ void k_router_bias(double* bias, int E, double s) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < E) bias[e] = s == 0.0 ? 0.0 : -s * log((double)(e + 1));
+}
+
+// ---------------------------------------------------------------------------
+// Embedding (+ self-conditioning add): h[t] = E[ids[t]] (+ s[t]).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_embed(const int* __restrict__ ids, const T* __restrict__ E, const T* __restrict__ sc,
+                        const int* __restrict__ use_sc, T* __restrict__ h, int d, int vocab,
+                        int* err) {
+  const int t = blockIdx.x;
+  int id = ids[t];
+  if (id < 0 || id >= vocab) { dev_error(err, DGDEV_BAD_INDEX); id = 0; }
+  const bool add = sc != nullptr && (use_sc == nullptr || *use_sc != 0);
+  const T* e = E + (long long)id * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float v = to_f(e[i]);
+    if (add) v = __fadd_rn(v, to_f(sc[(long long)t * d + i]));
+    h[(long long)t * d + i] = from_f<T>(v);
+  }
+}
+
+// RMSNorm (unit gain): x = h / sqrt(mean(h^2) + eps), one CTA per row.
+template <typename T>
+__global__ void k_rmsnorm(const T* __restrict__ h, T* __restrict__ x, int d, float eps) {
+  const long long row = blockIdx.x;
+  const T* hr = h + row * d;
+  float ss = 0.0f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) { const float v = to_f(hr[i]); ss = fmaf(v, v, ss); }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(red[0], (float)d), eps)));
+  for (int i = threadIdx.x; i < d; i += blockDim.x) x[row * d + i] = from_f<T>(to_f(hr[i]) * r);
+}
+
+// ---------------------------------------------------------------------------
+// After the QKV projection: sum split-K partials, rotate q and k by RoPE at
+// their absolute positions, round, and scatter q -> Q[t][Hq][hd],
+// k -> K cache [lbh][pos][hd], v -> V^T cache [lbh][hd][pos].
+// Token t of the launch is canvas b = t / n_per, local i = t % n_per,
+// position pos0 + i.
+// ---------------------------------------------------------------------------
+struct QkvPostArgs {
+  const float* ws;
+  long long split_stride;
+  int splits;
+  int Hq, Hkv, hd;
+  int n_per;        // tokens per canvas in this launch
+  int pos0;         // position of local token 0
+  int b0;           // first canvas index of this launch
+  int B;            // canvases in the KV cache
+  int layer;
+  int S;            // key slot stride of the cache
+  const float2* rope;
+};
+
+template <typename T>
+__global__ void k_qkv_post(QkvPostArgs a, T* __restrict__ Q, T* __restrict__ Kc, T* __restrict__ Vt) {
+  const int t = blockIdx.x;
+  const int b = a.b0 + t / a.n_per, i = t % a.n_per, pos = a.pos0 + i;
+  const int hd = a.hd, half = hd / 2;
+  const int nq = a.Hq * hd, nk = a.Hkv * hd;
+  const int ncol = nq + 2 * nk;
+  const float* w = a.ws + (long long)t * ncol;
+  auto load = [&](int c) {
+    float v = w[c];
+    for (int s = 1; s < a.splits; ++s) v += w[s * a.split_stride + c];
+    return v;
+  };
+  // rotary pairs of q and k heads
+  const int n_pairs = (a.Hq + a.Hkv) * half;
+  for (int u = threadIdx.x; u < n_pairs; u += blockDim.x) {
+    const int head = u / half, c = u % half;
+    const int base = head < a.Hq ? head * hd : nq + (head - a.Hq) * hd;
+    const float x0 = load(base + c), x1 = load(base + c + half);
+    const float2 cs = a.rope[(long long)pos * half + c];
+    const float y0 = x0 * cs.x - x1 * cs.y;
+    const float y1 = x0 * cs.y + x1 * cs.x;
+    if (head < a.Hq) {
+      T* q = Q + ((long long)(t) * a.Hq + head) * hd;
+      q[c] = from_f<T>(y0);
+      q[c + half] = from_f<T>(y1);
+    } else {
+      const int g = head - a.Hq;
+      const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + g;
+      T* k = Kc + (lbh * a.S + pos) * hd;
+      k[c] = from_f<T>(y0);
+      k[c + half] = from_f<T>(y1);
+    }
+  }
+  for (int u = threadIdx.x; u < nk; u += blockDim.x) {
+    const int g = u / hd, c = u % hd;
+    const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + g;
+    Vt[(lbh * hd + c) * a.S + pos] = from_f<T>(load(nq + nk + u));
+  }
+}
+
+// h = round(h + sum_s ws[s]) over [rows][d].
+template <typename T>
+__global__ void k_residual(T* __restrict__ h, const float* __restrict__ ws, long long split_stride,
+                           int splits, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    float v = ws[i];
+    for (int s = 1; s < splits; ++s) v += ws[s * split_stride + i];
+    h[i] = from_f<T>(to_f(h[i]) + v);
+  }
+}
+
+// out = round(sum_s ws[s]) over n elements.
+template <typename T>
+__global__ void k_sum_round(T* __restrict__ out, const float* __restrict__ ws, long long split_stride,
+                            int splits, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    float v = ws[i];
+    for (int s = 1; s < splits; ++s) v += ws[s * split_stride + i];
+    out[i] = from_f<T>(v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Router: r_e = x . Wr[e] (+ b_e) in fp64 (products of stored values are
+// exact, so the top-k decision does not depend on the summation order), top-k
+// by value with ties to the lower expert id, gate weights = softmax over the
+// k selected logits.  One CTA per token.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void k_router(const T* __restrict__ x, const T* __restrict__ Wr, const double* __restrict__ bias,
+                         int d, int E, int k, int* __restrict__ ids, float* __restrict__ gate) {
+  extern __shared__ double rsm[];
+  double* xs = rsm;          // [d]
+  double* logit = rsm + d;   // [E]
+  const long long t = blockIdx.x;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) xs[i] = (double)to_f(x[t * d + i]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nw) {
+    const T* w = Wr + (long long)e * d;
+    double acc = 0.0;
+    for (int i = lane; i < d; i += 32) acc = fma((double)to_f(w[i]), xs[i], acc);
+    acc = warp_sum_d(acc);
+    if (lane == 0) logit[e] = acc + (bias ? bias[e] : 0.0);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double sel[64];
+    int sid[64];
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        bool taken = false;
+        for (int q = 0; q < j; ++q) taken |= (sid[q] == e);
+        if (taken) continue;
+        if (best < 0 || logit[e] > logit[best]) best = e;
+      }
+      sid[j] = best;
+      sel[j] = logit[best];
+    }
+    double den = 0.0;
+    for (int j = 0; j < k; ++j) den += exp(sel[j] - sel[0]);
+    for (int j = 0; j < k; ++j) {
+      ids[t * k + j] = sid[j];
+      gate[t * k + j] = (float)(exp(sel[j] - sel[0]) / den);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Permute: stable counting sort of the T*k (token, slot) pairs by expert.
+// perm[pos] = pair, inv[pair] = pos; work items (expert, first row, rows,
+// first row) cover each expert's rows in tiles of `bn`.  One CTA; warp w
+// places the pairs of experts w, w+32, ... in pair order (stable).
+// ---------------------------------------------------------------------------
+__global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int bn, int* __restrict__ perm,
+                          int* __restrict__ inv, int4* __restrict__ work, int* __restrict__ work_count,
+                          int* __restrict__ counts_out, int* err) {
+  extern __shared__ int psm[];
+  int* counts = psm;         // [E]
+  int* offs = psm + E;       // [E + 1]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int e = ids[p];
+    if (e < 0 || e >= E) { dev_error(err, DGDEV_BAD_INDEX); continue; }
+    atomicAdd(&counts[e], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0, nw = 0;
+    for (int e = 0; e < E; ++e) {
+      offs[e] = acc;
+      for (int r = 0; r < counts[e]; r += bn)
+        work[nw++] = make_int4(e, acc + r, min(bn, counts[e] - r), acc + r);
+      acc += counts[e];
+    }
+    offs[E] = acc;
+    *work_count = nw;
+  }
+  __syncthreads();
+  if (counts_out)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts_out[e] = counts[e];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nwarps) {
+    int base = offs[e];
+    for (int p0 = 0; p0 < n_pairs; p0 += 32) {
+      const int p = p0 + lane;
+      const bool hit = p < n_pairs && ids[p] == e;
+      const unsigned m = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        const int pos = base + __popc(m & ((1u << lane) - 1u));
+        perm[pos] = p;
+        inv[p] = pos;
+      }
+      base += __popc(m);
+    }
+  }
+}
+
+// xp[pos] = x[perm[pos] / k]: expert-ordered copy of the normalised rows.
+template <typename T>
+__global__ void k_gather(const T* __restrict__ x, const int* __restrict__ perm, int k, int d,
+                         T* __restrict__ xp) {
+  const int pos = blockIdx.x;
+  const long long src = perm[pos] / k;
+  const uint4* s = reinterpret_cast<const uint4*>(x + src * d);
+  uint4* o = reinterpret_cast<uint4*>(xp + (long long)pos * d);
+  const int nv = d * (int)sizeof(T) / 16;
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) o[i] = s[i];
+}
+
+// SwiGLU: a = round(silu(g) * u), g/u the gate and up halves of each row.
+template <typename T>
+__global__ void k_swiglu(const float* __restrict__ gu, int ff, long long n, T* __restrict__ a) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / ff, c = i % ff;
+    const float g = gu[r * 2 * ff + c], u = gu[r * 2 * ff + ff + c];
+    a[i] = from_f<T>(g / (1.0f + expf(-g)) * u);
+  }
+}
+
+// h[t] = round(h[t] + sum_slot gate[t][slot] * y[inv[t*k+slot]]), slots in order.
+template <typename T>
+__global__ void k_moe_combine(T* __restrict__ h, const float* __restrict__ y, const int* __restrict__ inv,
+                              const float* __restrict__ gate, int k, int d) {
+  const long long t = blockIdx.x;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc = 0.0f;
+    for (int j = 0; j < k; ++j) acc = fmaf(gate[t * k + j], y[(long long)inv[t * k + j] * d + i], acc);
+    h[t * d + i] = from_f<T>(to_f(h[t * d + i]) + acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Vocab sampler, one CTA per logit row (row = canvas * 256 + position).
+//  pass 1: row max + argmax, Gumbel-max token at 1/T (Philox per 4 logits);
+//  pass 2: e_v = exp(l_v - m); S, U summed exactly in Q40 int64;
+//  pass 3: p_v = e_v * (1/S) stored for self-conditioning.
+// H = ln(S) - U/S; all binary32 steps use the fixed-sequence math above.
+// ---------------------------------------------------------------------------
+struct SamplerArgs {
+  const float* logits;
+  int vocab;
+  int positions;        // rows per canvas (256)
+  uint64_t seed;
+  float temp_start, temp_end;
+  const DevState* state;
+  int step_override;    // >= 0: use this round instead of state->step
+  float t_override;     // used when step_override >= 0
+  float* H;
+  int* tok;
+  int* amax;
+  long long* s_q;       // optional
+  long long* u_q;       // optional
+};
+
+struct ArgBest {
+  float v;
+  int i;
+};
+__device__ __forceinline__ ArgBest arg_better(ArgBest a, ArgBest b) {
+  if (b.i < 0) return a;
+  if (a.i < 0) return b;
+  if (b.v > a.v || (b.v == a.v && b.i < a.i)) return b;
+  return a;
+}
+__device__ __forceinline__ ArgBest warp_argmax(ArgBest x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    ArgBest y;
+    y.v = __shfl_xor_sync(0xffffffffu, x.v, o);
+    y.i = __shfl_xor_sync(0xffffffffu, x.i, o);
+    x = arg_better(x, y);
+  }
+  return x;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(512) k_sampler(SamplerArgs a, T* __restrict__ probs) {
+  const long long row = blockIdx.x;
+  const int canvas = (int)(row / a.positions), pos = (int)(row % a.positions);
+  const int step = a.step_override >= 0 ? a.step_override : a.state->step;
+  const float t = a.step_override >= 0 ? a.t_override : a.state->t;
+  const float temp = __fadd_rn(a.temp_end, __fmul_rn(__fsub_rn(a.temp_start, a.temp_end), t));
+  const float inv_t = __fdiv_rn(1.0f, temp);
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32) ^ (uint32_t)canvas;
+  const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab);
+  const int n4 = a.vocab / 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  __shared__ ArgBest red_m[32], red_g[32];
+  __shared__ long long red_s[32], red_u[32];
+  __shared__ float sh_m;
+  __shared__ long long sh_s;
+
+  // pass 1
+  ArgBest bm{-INFINITY, -1}, bg{-INFINITY, -1};
+  for (int v4 = threadIdx.x; v4 < n4; v4 += blockDim.x) {
+    const float4 l = l4[v4];
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)v4, (uint32_t)pos, (uint32_t)step, STREAM_GUMBEL), k0, k1);
+    const float lv[4] = {l.x, l.y, l.z, l.w};
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int v = v4 * 4 + j;
+      bm = arg_better(bm, ArgBest{lv[j], v});
+      const float key = __fadd_rn(__fmul_rn(lv[j], inv_t), gumbel_of(wv[j]));
+      bg = arg_better(bg, ArgBest{key, v});
+    }
+  }
+  bm = warp_argmax(bm);
+  bg = warp_argmax(bg);
+  if (lane == 0) { red_m[warp] = bm; red_g[warp] = bg; }
+  __syncthreads();
+  if (warp == 0) {
+    ArgBest x = lane < nw ? red_m[lane] : ArgBest{-INFINITY, -1};
+    ArgBest y = lane < nw ? red_g[lane] : ArgBest{-INFINITY, -1};
+    x = warp_argmax(x);
+    y = warp_argmax(y);
+    if (lane == 0) {
+      sh_m = x.v;
+      a.amax[row] = x.i;
+      a.tok[row] = y.i;
+    }
+  }
+  __syncthreads();
+  const float m = sh_m;
+
+  // pass 2
+  long long sq = 0, uq = 0;
+  for (int v4 = threadIdx.x; v4 < n4; v4 += blockDim.x) {
+    const float4 l = l4[v4];
+    const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float dlt = __fsub_rn(lv[j], m);
+      const float e = dg_expf(dlt);
+      sq += __float2ll_rz(__fmul_rn(e, 1099511627776.0f));
+      uq += __float2ll_rz(__fmul_rn(__fmul_rn(e, dlt), 1099511627776.0f));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    uq += __shfl_xor_sync(0xffffffffu, uq, o);
+  }
+  if (lane == 0) { red_s[warp] = sq; red_u[warp] = uq; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long S = 0, U = 0;
+    for (int w = 0; w < nw; ++w) { S += red_s[w]; U += red_u[w]; }
+    const float sf = __ll2float_rn(S), uf = __ll2float_rn(U);
+    a.H[row] = __fsub_rn(dg_logf(__fmul_rn(sf, 9.094947017729282e-13f)), __fdiv_rn(uf, sf));
+    if (a.s_q) a.s_q[row] = S;
+    if (a.u_q) a.u_q[row] = U;
+    sh_s = S;
+  }
+  __syncthreads();
+
+  // pass 3
+  if (probs) {
+    const float inv_s = __fdiv_rn(1.0f, __fmul_rn(__ll2float_rn(sh_s), 9.094947017729282e-13f));
+    T* pr = probs + row * a.vocab;
+    for (int v4 = threadIdx.x; v4 < n4; v4 += blockDim.x) {
+      const float4 l = l4[v4];
+      const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) pr[v4 * 4 + j] = from_f<T>(__fmul_rn(dg_expf(__fsub_rn(lv[j], m)), inv_s));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Commit / re-noise / stop, one CTA of 256 threads per canvas.
+// Default: commit where H < bound.  Entropy-bounded: sort (trunc(H 2^32), i)
+// ascending, commit the longest prefix with exact sum <= trunc(bound 2^32),
+// at least one.  Stop: (mean mode) all committed or sum H < n * bound, or
+// (EB mode) sum H < n * bound and argmax == previous argmax (not at round 0);
+// the last round of the budget always stops.  Uncommitted positions get a
+// fresh uniform token (Philox stream 1).
+// In block-loop mode a stopped canvas is frozen: its outputs are written once.
+// ---------------------------------------------------------------------------
+struct CommitArgs {
+  const float* H;
+  const int* tok;
+  const int* amax;
+  int* prev_amax;          // [B*256] argmax of the previous round (updated)
+  int vocab;
+  uint64_t seed;
+  int commit_mode;
+  float commit_bound;
+  int stop_mode;
+  float stop_bound;
+  int max_steps;
+  DevState* state;
+  int step_override;       // >= 0: single-step mode with this round
+  // single-step outputs (any may be null)
+  uint8_t* commit;
+  int* canvas_next;
+  int* stop;
+  int* n_committed;
+  // block-loop state (null in single-step mode)
+  int* canvas_cur;         // [B*256] canvas fed to the next round
+  int* done;               // [B]
+  int* steps_used;         // [B]
+  int* n_committed_out;    // [B]
+  int* canvas_out;         // [B*256]
+};
+
+__global__ void __launch_bounds__(256) k_commit(CommitArgs a) {
+  const int b = blockIdx.x, i = threadIdx.x;
+  const int n = 256;
+  const int step = a.step_override >= 0 ? a.step_override : a.state->step;
+  const bool loop = a.done != nullptr;
+  if (loop && a.done[b]) return;
+  const long long idx = (long long)b * n + i;
+  const float h = a.H[idx];
+  const long long hq = __float2ll_rz(__fmul_rn(h, 4294967296.0f));
+  __shared__ long long key_h[256];
+  __shared__ int key_i[256];
+  __shared__ long long sum_red[8];
+  __shared__ int cnt_red[8], same_red[8];
+  __shared__ int commit_s[256];
+
+  int committed;
+  if (a.commit_mode == 0) {
+    committed = h < a.commit_bound;
+  } else {
+    key_h[i] = hq;
+    key_i[i] = i;
+    __syncthreads();
+    // bitonic sort of (hq, i) ascending
+    for (int kk = 2; kk <= n; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const bool up = (i & kk) == 0;
+          const long long ha = key_h[i], hb = key_h[ixj];
+          const int ia = key_i[i], ib = key_i[ixj];
+          const bool gt = ha > hb || (ha == hb && ia > ib);
+          if (gt == up) { key_h[i] = hb; key_h[ixj] = ha; key_i[i] = ib; key_i[ixj] = ia; }
+        }
+        __syncthreads();
+      }
+    }
+    // inclusive prefix sum of sorted entropies (exact int64)
+    const long long lim = __float2ll_rz(__fmul_rn(a.commit_bound, 4294967296.0f));
+    if (i == 0) {
+      long long acc = 0;
+      for (int r = 0; r < n; ++r) {
+        acc += key_h[r];
+        commit_s[key_i[r]] = (r == 0 || acc <= lim) ? 1 : 0;
+        if (r > 0 && acc > lim) {
+          for (int q = r + 1; q < n; ++q) commit_s[key_i[q]] = 0;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    committed = commit_s[i];
+  }
+
+  // reductions: count, sum of fixed-point entropies, argmax unchanged
+  const int same = (a.amax[idx] == a.prev_amax[idx]) ? 1 : 0;
+  long long s = hq;
+  int c = committed, sm = same;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    sm += __shfl_xor_sync(0xffffffffu, sm, o);
+  }
+  if ((i & 31) == 0) { sum_red[i >> 5] = s; cnt_red[i >> 5] = c; same_red[i >> 5] = sm; }
+  __syncthreads();
+  long long hsum = 0;
+  int ncom = 0, nsame = 0;
+  for (int w = 0; w < 8; ++w) { hsum += sum_red[w]; ncom += cnt_red[w]; nsame += same_red[w]; }
+  const long long bound_q = __float2ll_rz(__fmul_rn(a.stop_bound, 4294967296.0f));
+  const bool low = hsum < (long long)n * bound_q;
+  bool stop;
+  if (step >= a.max_steps - 1) stop = true;
+  else if (a.stop_mode == 0) stop = (ncom == n) || low;
+  else stop = step > 0 && low && nsame == n;
+
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32) ^ (uint32_t)b;
+  const uint4 w = philox4x32_10(make_uint4(0u, (uint32_t)i, (uint32_t)step, STREAM_RENOISE), k0, k1);
+  const int nxt = committed ? a.tok[idx] : token_from_word(w.x, a.vocab);
+
+  __syncthreads();
+  if (a.commit) a.commit[idx] = (uint8_t)committed;
+  if (a.canvas_next) a.canvas_next[idx] = nxt;
+  a.prev_amax[idx] = a.amax[idx];
+  if (i == 0) {
+    if (a.stop) a.stop[b] = stop ? 1 : 0;
+    if (a.n_committed) a.n_committed[b] = ncom;
+  }
+  if (loop) {
+    a.canvas_cur[idx] = nxt;
+    if (stop) {
+      a.canvas_out[idx] = a.tok[idx];
+      if (i == 0) {
+        a.done[b] = 1;
+        a.steps_used[b] = step + 1;
+        a.n_committed_out[b] = ncom;
+        atomicSub(&a.state->active, 1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Block-loop control.
+// ---------------------------------------------------------------------------
+// Start of a round: t = 1 - s/(N-1) in binary32 (t = 1 when N = 1).
+__global__ void k_round_begin(DevState* st) {
+  const int s = st->step, N = st->n_steps;
+  st->t = N <= 1 ? 1.0f : __fsub_rn(1.0f, __fdiv_rn((float)s, (float)(N - 1)));
+  st->use_selfcond = s > 0 ? 1 : 0;
+}
+
+// Single-step mode: set the round and time given by the caller.
+__global__ void k_set_round(DevState* st, int step, float t, int use_sc) {
+  st->step = step;
+  st->t = t;
+  st->use_selfcond = use_sc;
+}
+
+// Block-loop start: initial canvases from Philox stream 2, counters reset.
+__global__ void k_loop_init(DevState* st, int n_steps, int n_canvas, int* canvas_cur, int* done,
+                            int* steps_used, int* n_committed_out, int* prev_amax, uint64_t seed,
+                            int vocab) {
+  const int b = blockIdx.x, i = threadIdx.x;
+  const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32) ^ (uint32_t)b;
+  const uint4 w = philox4x32_10(make_uint4(0u, (uint32_t)i, 0u, STREAM_INIT_CANVAS), k0, k1);
+  canvas_cur[b * 256 + i] = token_from_word(w.x, vocab);
+  prev_amax[b * 256 + i] = -1;
+  if (i == 0) { done[b] = 0; steps_used[b] = 0; n_committed_out[b] = 0; }
+  if (b == 0 && i == 0) {
+    st->step = 0;
+    st->n_steps = n_steps;
+    st->active = n_canvas;
+    st->cond = 1;
+  }
+}
+
+// End of a round: advance and decide whether to continue.
+__global__ void k_round_end(DevState* st) {
+  st->step += 1;
+  st->cond = (st->active > 0 && st->step < st->n_steps && st->err == 0) ? 1 : 0;
+}
+
+__global__ void k_round_end_cond(DevState* st, cudaGraphConditionalHandle handle) {
+  st->step += 1;
+  const int c = (st->active > 0 && st->step < st->n_steps && st->err == 0) ? 1 : 0;
+  st->cond = c;
+  cudaGraphSetConditional(handle, c);
+}

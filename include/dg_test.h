@@ -1,0 +1,103 @@
+/*
+ * dg_test.h -- kernel-level entry points of the denoising-step library, used
+ * by the parity tests and the benchmark.  Same conventions as dg.h: device
+ * pointers unless marked "host", caller-owned buffers, asynchronous on
+ * `stream`, status codes, no exceptions.  Hooks marked "allocates" take
+ * temporary device memory and synchronise `stream` before returning.
+ */
+#ifndef DG_TEST_H
+#define DG_TEST_H
+
+#include "dg.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Fixed-sequence binary32 math of the sampler and the weight generator,
+ * elementwise over n values:
+ *   which 0: natural log of positive normal float `in`
+ *   which 1: e^x for float x <= 0 (0 below -86)
+ *   which 2: cos(2 pi u) for float u in (0,1)
+ *   which 3: Gumbel noise -ln(-ln u(w)) of uint32 words w
+ *   which 4: weight value 0.02 * BoxMuller(Philox(seed, (j, tensor_id, 3)))
+ *            for uint64 indices j in `in` (seed = aux0, tensor_id = aux1). */
+dg_status dg_test_math(int32_t which, const void* in, float* out, int64_t n, uint64_t aux0, uint32_t aux1,
+                       void* stream);
+
+/* Philox4x32-10 of n (counter[4], key[2]) records: in uint32 [n,6] ->
+ * out uint32 [n,4] (Salmon et al., SC'11). */
+dg_status dg_test_philox(const uint32_t* in, uint32_t* out, int64_t n, void* stream);
+
+/* The vocab sampler kernel on caller logits fp32 [rows, vocab] (row = canvas
+ * * positions + position; canvas = row / positions keys the Philox stream):
+ * entropy H, Gumbel-max token at T = temp_end + (temp_start - temp_end) t,
+ * argmax, exact fixed-point sums S_q/U_q (2^-40 units, may be NULL) and the
+ * probabilities (bf16 if probs_bf16 else fp32; may be NULL). */
+dg_status dg_test_sampler(const float* logits, int32_t rows, int32_t vocab, int32_t positions, uint64_t seed,
+                          int32_t step, float t, float temp_start, float temp_end, float* H, int32_t* tok,
+                          int32_t* amax, int64_t* s_q, int64_t* u_q, void* probs, int32_t probs_bf16,
+                          void* stream);
+
+/* The commit / re-noise / stop kernel for B canvases of 256 positions.
+ * prev_amax (in/out) holds the previous round's argmax and is overwritten. */
+dg_status dg_test_commit(const float* H, const int32_t* tok, const int32_t* amax, int32_t* prev_amax, int32_t B,
+                         int32_t vocab, uint64_t seed, int32_t step, int32_t max_steps, int32_t commit_mode,
+                         float commit_bound, int32_t stop_mode, float stop_bound, uint8_t* commit,
+                         int32_t* canvas_next, int32_t* stop, int32_t* n_committed, void* stream);
+
+/* Dense GEMM out[split][n][m] = alpha * sum_{k in split} A[m][k] B[n][k]
+ * (A [M,K], B [N,K] row-major, bf16 through tcgen05 when bf16 != 0, else
+ * fp32 SIMT); out holds k_splits partial slabs of N*M floats; bn in
+ * {32,64,128,256} is the token tile (bf16 only).  Allocates (tensor maps
+ * only; no device memory). */
+dg_status dg_test_gemm(const void* A, const void* B, float* out, int32_t M, int32_t N, int32_t K, int32_t bf16,
+                       float alpha, int32_t k_splits, int32_t bn, void* stream);
+
+/* Grouped GEMM as used by the experts: A [groups*M, K], B [rows, K] with
+ * rows ordered by group (counts host int32 [groups]); out [rows, M] fp32,
+ * out[r][m] = sum_k A[g(r)*M + m][k] B[r][k].  Allocates. */
+dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
+                               int32_t K, int32_t bf16, int32_t bn, float* out, void* stream);
+
+/* Attention kernels (tcgen05 for bf16, SIMT for fp32) plus the split
+ * combine, on plain layouts: q [n_canvas*n_q, Hq, hd], k and v
+ * [n_canvas, Hkv, n_keys, hd] -> out fp32 [n_canvas*n_q, Hq*hd].  Query i of
+ * a canvas sits at position q_pos0 + i; causal != 0 hides keys after it.
+ * Allocates. */
+dg_status dg_test_attention(const void* q, const void* k, const void* v, int32_t n_canvas, int32_t n_q,
+                            int32_t q_pos0, int32_t n_keys, int32_t causal, int32_t Hq, int32_t Hkv,
+                            int32_t head_dim, int32_t bf16, float* out, void* stream);
+
+/* Copy weight tensor `tensor_id` (0 = E [V,d], 1 = W_sc [d,d]; layer l:
+ * 16+16l + {0 Wq,1 Wk,2 Wv,3 Wo,4 Wr,5 Wg [E,ff,d],6 Wu,7 Wd [E,d,ff]})
+ * into dst in its logical row-major layout, model dtype. */
+dg_status dg_read_weight(const dg_model* model, int32_t tensor_id, void* dst, void* stream);
+
+/* Store prompt keys/values k, v [L, B, Hkv, P, hd] (model dtype; keys
+ * already rotated) into the library's cache layout inside `kv`. */
+dg_status dg_load_kv(dg_model* model, void* kv, int32_t B, int32_t P, const void* k, const void* v, void* stream);
+
+/* Run `reps` single denoising rounds (step 0, t = 1, self-conditioning on)
+ * with a CUDA event pair around every kernel launch on `stream`; returns
+ * per-phase total milliseconds and launch counts (host arrays of n_phases;
+ * phase names from dg_phase_name).  Synchronises. */
+dg_status dg_profile_step(dg_model* model, void* kv, int32_t B, int32_t P, int32_t reps, float* phase_ms,
+                          int32_t* phase_launches, int32_t n_phases, void* stream);
+
+/* Name of profile phase i, or NULL past the last one. */
+const char* dg_phase_name(int32_t i);
+
+/* Per-expert row counts of the most recent MoE layer launch (device int32
+ * [n_experts]); the number of nonzero entries is the distinct experts that
+ * layer streamed. */
+dg_status dg_expert_counts(const dg_model* model, int32_t* counts, void* stream);
+
+/* Kernel launches recorded in one captured block-loop round (graph body). */
+int32_t dg_launches_per_round(const dg_model* model);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_TEST_H */

@@ -1,0 +1,186 @@
+"""Step-level parity of the CUDA path against the oracle (B200 only).
+
+Tolerances (from the workload definitions): logits and entropy within 1e-4
+relative in the fp32 workload, within 2e-2 absolute in the bf16 workloads;
+sampled tokens and commit masks identical wherever the oracle's own decision
+is not within rounding of a tie (Gumbel-max margin, entropy vs bound), and at
+least 99% agreement overall; full block runs agree on >= 99% of tokens."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import block_text_diffusion_b200 as dg  # noqa: E402
+from block_text_diffusion_b200 import inputs as I  # noqa: E402
+from oracle import model as om, sampler as sp, numerics as nm  # noqa: E402
+
+F32 = np.float32
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    dg.lib()
+
+
+def cu(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.float().cpu().numpy() if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+def read_kv(model, kv, B, P):
+    """Decode the library's cache layout: K [L][B][Hkv][S][hd], V^T [L][B][Hkv][hd][S]."""
+    w = model.w
+    S = ((P + 256 + 63) // 64) * 64
+    esz = 2 if w.dtype == I.DTYPE_BF16 else 4
+    n = w.n_layers * B * w.n_kv_heads * S * w.head_dim
+    raw = kv[: 2 * n * esz].view(torch.bfloat16 if esz == 2 else torch.float32)
+    K = raw[:n].view(w.n_layers, B, w.n_kv_heads, S, w.head_dim)
+    Vt = raw[n:].view(w.n_layers, B, w.n_kv_heads, w.head_dim, S)
+    return host(K), host(Vt).transpose(0, 1, 2, 4, 3)
+
+
+def step_buffers(w, B):
+    dt = torch.bfloat16 if w.dtype == I.DTYPE_BF16 else torch.float32
+    z = lambda shape, t: torch.zeros(shape, dtype=t, device="cuda")
+    return dict(logits=z((B, 256, w.vocab), torch.float32), entropy=z((B, 256), torch.float32),
+                tokens=z((B, 256), torch.int32), argmax=z((B, 256), torch.int32), commit=z((B, 256), torch.uint8),
+                canvas_next=z((B, 256), torch.int32), selfcond_next=z((B, 256, w.d_model), dt),
+                stop=z(B, torch.int32), n_committed=z(B, torch.int32))
+
+
+def gumbel_margin(l32, inv_t, seed, canvas_id, step):
+    """Gap between the best and second-best Gumbel key per row (oracle side)."""
+    out = np.empty(l32.shape[0])
+    for i in range(l32.shape[0]):
+        g = sp.gumbel_noise(seed, canvas_id, i, step, l32.shape[1])
+        key = np.sort(l32[i].astype(np.float64) * float(inv_t) + g)
+        out[i] = key[-1] - key[-2]
+    return out
+
+
+def check_logits(got, ref, fp32):
+    if fp32:
+        scale = np.maximum(np.abs(ref), np.sqrt((ref ** 2).mean(axis=-1, keepdims=True)))
+        assert np.all(np.abs(got - ref) <= 1e-4 * scale), np.abs(got - ref).max()
+    else:
+        assert np.abs(got - ref).max() <= 2e-2, np.abs(got - ref).max()
+
+
+def compare_round(r_gpu, r_ora, w, step, t, fp32, canvas_id=0):
+    check_logits(r_gpu["logits"], r_ora["logits64"], fp32)
+    H_tol = 1e-4 * np.maximum(1.0, np.abs(r_ora["H"])) if fp32 else 2e-2
+    assert np.all(np.abs(r_gpu["entropy"] - r_ora["H"]) <= H_tol)
+    inv_t = F32(1.0) / sp.temperature(F32(t), w.temp_start, w.temp_end)
+    margin = gumbel_margin(r_ora["logits"], inv_t, w.sample_seed, canvas_id, step)
+    err = np.abs(r_gpu["logits"] - r_ora["logits64"]).max(axis=1)
+    safe = margin > 4 * err * float(inv_t) + 1e-6
+    assert np.array_equal(r_gpu["tokens"][safe], r_ora["tokens"][safe])
+    assert (r_gpu["tokens"] == r_ora["tokens"]).mean() >= 0.99
+    Hb = w.commit_bound
+    if w.commit_mode == 0:
+        safe_c = np.abs(r_ora["H"] - Hb) > np.max(H_tol) * 2
+        assert np.array_equal(r_gpu["commit"][safe_c], r_ora["commit"][safe_c])
+
+
+# --- tiny fp32 workload: weights, encode, one round, full block ------------------------
+@pytest.fixture(scope="module")
+def tiny():
+    w = I.TINY_FP32
+    return w, dg.Model(w), om.Model(w)
+
+
+def test_tiny_weights_bit_exact(tiny):
+    w, gm, om_ = tiny
+    shapes = {0: om_.embed, 1: om_.wsc}
+    for l, L in enumerate(om_.layers):
+        for j, name in enumerate(("wq", "wk", "wv", "wo", "wr", "wg", "wu", "wd")):
+            shapes[om.layer_tensor_id(l, name)] = getattr(L, name)
+    for tid, ref in shapes.items():
+        out = torch.empty(ref.shape, dtype=torch.float32, device="cuda")
+        gm.read_weight(tid, out)
+        assert np.array_equal(host(out).view(np.uint32), ref.view(np.uint32)), tid
+
+
+def test_tiny_encode_matches_oracle(tiny):
+    w, gm, om_ = tiny
+    P = w.prompt_len
+    prompt = I.prompt_ids(w.sample_seed, 1, P, w.vocab)
+    kv = gm.new_kv(1, P)
+    gm.encode_prompt(cu(prompt), kv)
+    K, V = read_kv(gm, kv, 1, P)
+    Ko, Vo = om.encode_prompt(om_, prompt[0])
+    assert np.allclose(K[:, 0, :, :P], Ko, rtol=1e-4, atol=1e-5)
+    assert np.allclose(V[:, 0, :, :P], Vo, rtol=1e-4, atol=1e-5)
+
+
+def test_tiny_round_and_block_match_oracle(tiny):
+    w, gm, om_ = tiny
+    P = w.prompt_len
+    prompt = I.prompt_ids(w.sample_seed, 1, P, w.vocab)
+    kv = gm.new_kv(1, P)
+    gm.encode_prompt(cu(prompt), kv)
+    Ko, Vo = om.encode_prompt(om_, prompt[0])
+    canvas = sp.initial_canvas(w.sample_seed, 0, 256, w.vocab)
+    out = step_buffers(w, 1)
+    gm.denoise_step(kv, P, cu(canvas[None]), None, 0, 1.0, out)
+    g = {k: host(v)[0] for k, v in out.items()}
+    r = om.denoise_step(om_, Ko, Vo, canvas, None, 0, F32(1.0))
+    compare_round(g, r, w, 0, 1.0, True)
+    assert np.allclose(g["selfcond_next"], r["selfcond_next"], rtol=1e-4, atol=1e-6)
+    # second round fed with the oracle's own self-conditioning and canvas
+    gm.denoise_step(kv, P, cu(r["canvas_next"][None]), cu(r["selfcond_next"][None].astype(F32)), 1,
+                    float(sp.schedule_t(1, w.max_steps)), out)
+    g2 = {k: host(v)[0] for k, v in out.items()}
+    r2 = om.denoise_step(om_, Ko, Vo, r["canvas_next"], r["selfcond_next"], 1, sp.schedule_t(1, w.max_steps),
+                         prev_amax=r["amax"])
+    compare_round(g2, r2, w, 1, float(sp.schedule_t(1, w.max_steps)), True)
+    # full block on the device loop
+    cout = torch.zeros((1, 256), dtype=torch.int32, device="cuda")
+    su = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gm.encode_prompt(cu(prompt), kv)
+    gm.generate_block(kv, 1, P, cout, su, nc)
+    gm.sync_status()
+    ref = om.generate_block(om_, Ko, Vo)
+    assert int(host(su)[0]) == ref["steps_used"]
+    assert (host(cout)[0] == ref["canvas"]).mean() >= 0.99
+    assert abs(int(host(nc)[0]) - ref["n_committed"]) <= 2
+
+
+# --- mid bf16 workload with a synthetic prompt cache -------------------------------------
+@pytest.fixture(scope="module")
+def mid():
+    w = I.MID_BF16
+    return w, dg.Model(w), om.Model(w)
+
+
+def test_mid_weights_sampled_bit_exact(mid):
+    w, gm, om_ = mid
+    for tid, ref in ((0, om_.embed), (om.layer_tensor_id(3, "wg"), om_.layers[3].wg),
+                     (om.layer_tensor_id(7, "wd"), om_.layers[7].wd), (om.layer_tensor_id(0, "wk"), om_.layers[0].wk)):
+        out = torch.empty(ref.shape, dtype=torch.bfloat16, device="cuda")
+        gm.read_weight(tid, out)
+        assert np.array_equal(host(out).view(np.uint32), ref.view(np.uint32)), tid
+
+
+def test_mid_round_matches_oracle(mid):
+    w, gm, om_ = mid
+    P = w.prompt_len
+    K, V = I.prompt_kv(9, w.n_layers, 1, w.n_kv_heads, P, w.head_dim, bf16=True)
+    kv = gm.new_kv(1, P)
+    gm.load_kv(kv, 1, P, cu(K).to(torch.bfloat16), cu(V).to(torch.bfloat16))
+    canvas = sp.initial_canvas(w.sample_seed, 0, 256, w.vocab)
+    out = step_buffers(w, 1)
+    gm.denoise_step(kv, P, cu(canvas[None]), None, 0, 1.0, out)
+    gm.sync_status()
+    g = {k: host(v)[0] for k, v in out.items()}
+    r = om.denoise_step(om_, K[:, 0], V[:, 0], canvas, None, 0, F32(1.0))
+    compare_round(g, r, w, 0, 1.0, False)
+    assert np.abs(g["selfcond_next"] - r["selfcond_next"]).max() <= 2e-2
