@@ -38,6 +38,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-reps", type=int, default=3)
+    ap.add_argument("--max-rounds", type=int, default=None,
+                    help="override the round budget (short runs for profiler launch lists)")
     return ap.parse_args()
 
 
@@ -127,6 +129,19 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def reduce_over_ranks(times, work, world, device):
+    """Whole-job numbers: the max of each time over ranks (the job ends when
+    the slowest rank ends) and the sum of each work count."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    w = torch.tensor(work, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()], [int(x) for x in w.tolist()]
+
+
 # --- our arm ------------------------------------------------------------------------------
 def run_ours(a):
     import numpy as np
@@ -147,6 +162,8 @@ def run_ours(a):
     B = a.batch or w.batch
     P = w.prompt_len
     w = w.replace(sample_seed=w.sample_seed + 1000 * rank)
+    if a.max_rounds:
+        w = w.replace(max_steps=a.max_rounds)
     model = dg.Model(w, max_canvases=B, max_prompt=P)
     stream = torch.cuda.current_stream()
     prompt_h = torch.from_numpy(I.prompt_ids(w.sample_seed, B, P, w.vocab)).pin_memory()
@@ -216,14 +233,8 @@ def run_ours(a):
     except AttributeError:
         pass
 
-    # reduce over ranks: max time, sum of work
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device="cuda")
-    wk = torch.tensor([n_rounds, n_com, e_rounds], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dist.all_reduce(wk, op=dist.ReduceOp.SUM)
-    ms, e2e_ms = float(t[0]), float(t[1])
-    n_rounds, n_com, e_rounds = (int(x) for x in wk.tolist())
+    (ms, e2e_ms), (n_rounds, n_com, e_rounds) = reduce_over_ranks(
+        [ms, e2e_ms], [n_rounds, n_com, e_rounds], world, "cuda")
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -69,8 +69,8 @@ def lib():
             "dg_test_philox": ([P, P, I64, P], I32),
             "dg_test_sampler": ([P, I32, I32, I32, U64, I32, F, F, F, P, P, P, P, P, P, I32, P], I32),
             "dg_test_commit": ([P, P, P, P, I32, I32, U64, I32, I32, I32, F, I32, F, P, P, P, P, P], I32),
-            "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, P], I32),
-            "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, P, P], I32),
+            "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, I32, P], I32),
+            "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
             "dg_test_attention": ([P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P], I32),
             "dg_read_weight": ([P, I32, P, P], I32),
             "dg_load_kv": ([P, P, I32, I32, P, P, P], I32),
@@ -221,20 +221,20 @@ def test_commit(H, tok, amax, prev_amax, vocab, seed, step, max_steps, commit_mo
                                 _ptr(canvas_next), _ptr(stop), _ptr(n_committed), _stream(stream)), "dg_test_commit")
 
 
-def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, stream=None):
+def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, persistent=False, stream=None):
     import torch
     M, K = A.shape
     N = B.shape[0]
     _check(lib().dg_test_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, 1 if A.dtype == torch.bfloat16 else 0,
-                              float(alpha), k_splits, bn, _stream(stream)), "dg_test_gemm")
+                              float(alpha), k_splits, bn, int(persistent), _stream(stream)), "dg_test_gemm")
 
 
-def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, stream=None):
+def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, stream=None):
     import torch
     K = A.shape[-1]
     c = (ctypes.c_int32 * groups)(*[int(x) for x in counts])
     _check(lib().dg_test_grouped_gemm(_ptr(A), _ptr(B), c, groups, M, K, 1 if A.dtype == torch.bfloat16 else 0,
-                                      bn, _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
+                                      bn, int(persistent), _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
 
 
 def test_attention(q, k, v, n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out, stream=None):

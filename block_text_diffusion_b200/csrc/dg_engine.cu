@@ -215,6 +215,7 @@ struct GemmCall {
   int a_group_rows = 0;
   int max_items = 0;
   int bn = 256;
+  bool persistent = false;           // walk tiles with one CTA per SM slot
 };
 
 template <int BN, int ST>
@@ -230,6 +231,26 @@ dg_status launch_tc(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   if (grid <= 0) return DG_OK;
   if (grid > 0x7FFFFFFFLL) return DG_ERR_UNSUPPORTED;
   k_gemm_tc<BN, ST><<<(unsigned)grid, 128, C::kSmem, s>>>(*g.tA, *g.tB, a);
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+template <int BN, int ST>
+dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
+  using C = GemmTcCfg<BN, ST>;
+  static bool attr = false;
+  if (!attr) {
+    CU_TRY(cudaFuncSetAttribute(k_gemm_tc_persistent<BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::kSmem));
+    attr = true;
+  }
+  const int items_dense = g.work ? 0 : cdiv(g.N, a.n_tile);
+  const long long max_tiles = (long long)a.m_tiles * a.k_splits * (g.work ? g.max_items : items_dense);
+  if (max_tiles <= 0) return DG_OK;
+  // CTAs per SM allowed by shared memory (228 KB per SM)
+  const int per_sm = std::max(1, (228 * 1024) / (C::kSmem + 2048));
+  const int grid = (int)std::min<long long>(max_tiles, (long long)kSMs * std::min(per_sm, 2));
+  k_gemm_tc_persistent<BN, ST><<<grid, 192, C::kSmem, s>>>(*g.tA, *g.tB, a, items_dense);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -261,6 +282,15 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   }
   a.m_tiles = cdiv(g.M, 128);
   a.n_tile = g.bn;
+  if (g.persistent) {
+    switch (g.bn) {
+      case 256: return launch_tc_persistent<256, 4>(g, a, s);
+      case 128: return launch_tc_persistent<128, 6>(g, a, s);
+      case 64: return launch_tc_persistent<64, 8>(g, a, s);
+      case 32: return launch_tc_persistent<32, 8>(g, a, s);
+      default: return DG_ERR_UNSUPPORTED;
+    }
+  }
   switch (g.bn) {
     case 256: return launch_tc<256, 4>(g, a, s);
     case 128: return launch_tc<128, 5>(g, a, s);
@@ -417,10 +447,10 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
   const int bn_g = m->bf ? (n_pairs / m->E <= 48 ? 64 : (n_pairs / m->E <= 100 ? 128 : 256)) : 64;
   const int max_items = m->E + cdiv(n_pairs, bn_g);
 
+  // Precondition: m->x holds RMSNorm(h) of the first layer (written by the
+  // embedding kernel); every layer leaves RMSNorm of its output in m->x.
   for (int l = 0; l < m->L; ++l) {
     const LayerW& w = m->layers[l];
-    { LaunchScope ls(m, s, PH_NORM);
-      k_rmsnorm<T><<<Tn, 256, 0, s>>>((const T*)m->h, (T*)m->x, d, m->c.rms_eps); }
     // QKV projection
     GemmCall qc;
     qc.tA = &w.tm_qkv; qc.tB = &m->tm_x; qc.A32 = (const float*)w.qkv; qc.B32 = (const float*)m->x;
@@ -490,12 +520,9 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     }
     DG_TRY(gemm(m, oc, PH_O_GEMM, s));
     { LaunchScope ls(m, s, PH_RESIDUAL);
-      const long long n = (long long)Tn * d;
-      k_residual<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(
-          (T*)m->h, m->ws, oc.split_stride, std::min(oc.splits, cdiv(nq, 64)), n); }
+      k_residual_norm<T><<<Tn, 256, 0, s>>>((T*)m->h, (T*)m->x, m->ws, oc.split_stride,
+                                            std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
     // MoE
-    { LaunchScope ls(m, s, PH_NORM);
-      k_rmsnorm<T><<<Tn, 256, 0, s>>>((const T*)m->h, (T*)m->x, d, m->c.rms_eps); }
     { LaunchScope ls(m, s, PH_ROUTER);
       const size_t sm = (size_t)(d + m->E) * sizeof(double);
       k_router<T><<<Tn, 256, sm, s>>>((const T*)m->x, (const T*)w.wr, m->rbias, d, m->E, m->k, m->ids,
@@ -521,7 +548,8 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.max_items = max_items; dn.bn = bn_g;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
-      k_moe_combine<T><<<Tn, 256, 0, s>>>((T*)m->h, m->ws, m->inv, m->gate, m->k, d); }
+      k_moe_combine_norm<T><<<Tn, 256, 0, s>>>((T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
+                                               m->c.rms_eps); }
   }
   CU_TRY(cudaGetLastError());
   return DG_OK;
@@ -550,11 +578,10 @@ template <typename T>
 dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_t s) {
   const int B = g.B, Tn = B * kCanvas, d = m->d, V = m->V;
   { LaunchScope ls(m, s, PH_EMBED);
-    k_embed<T><<<Tn, 256, 0, s>>>(io.canvas, (const T*)m->emb, (const T*)io.selfcond, io.use_sc, (T*)m->h, d,
-                                  V, &m->st->err); }
+    k_embed_norm<T><<<Tn, 256, 0, s>>>(io.canvas, (const T*)m->emb, (const T*)io.selfcond, io.use_sc, (T*)m->h,
+                                       (T*)m->x, d, V, m->c.rms_eps, &m->st->err); }
+  // the last layer leaves the final RMSNorm(h) in m->x
   DG_TRY(run_layers<T>(m, g, 0, B, kCanvas, g.P, g.P + kCanvas, false, s));
-  { LaunchScope ls(m, s, PH_NORM);
-    k_rmsnorm<T><<<Tn, 256, 0, s>>>((const T*)m->h, (T*)m->x, d, m->c.rms_eps); }
   // LM head (tied embedding) with the logit scale
   GemmCall lc;
   lc.tA = &m->tm_E; lc.tB = &m->tm_x; lc.A32 = (const float*)m->emb; lc.B32 = (const float*)m->x;
@@ -840,9 +867,10 @@ size_t dg_kv_bytes(const dg_model* m, int32_t B, int32_t P) {
 int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   if (!m) return 0;
   (void)B; (void)P;
-  // per layer: norm, qkv gemm, qkv post, attention, combine, o gemm, residual,
-  // norm, router, permute, gather, gate/up gemm, swiglu, down gemm, combine
-  return 15 * m->L + 1 /*embed*/ + 1 /*norm*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
+  // per layer: qkv gemm, qkv post, attention, attention combine, o gemm,
+  // residual+norm, router, permute, gather, gate/up gemm, swiglu, down gemm,
+  // combine+norm; then embed+norm, lm head, sampler, commit, 4 self-cond.
+  return 13 * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          4 /*self-conditioning*/;
 }
 
@@ -859,11 +887,12 @@ dg_status dg_encode_prompt(dg_model* m, const int32_t* prompt, int32_t B, int32_
       {
         LaunchScope ls(m, s, PH_EMBED);
         if (m->bf)
-          k_embed<bf16><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const bf16*)m->emb, nullptr, nullptr,
-                                         (bf16*)m->h, m->d, m->V, &m->st->err);
+          k_embed_norm<bf16><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const bf16*)m->emb, nullptr, nullptr,
+                                              (bf16*)m->h, (bf16*)m->x, m->d, m->V, m->c.rms_eps, &m->st->err);
         else
-          k_embed<float><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const float*)m->emb, nullptr, nullptr,
-                                          (float*)m->h, m->d, m->V, &m->st->err);
+          k_embed_norm<float><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const float*)m->emb, nullptr,
+                                               nullptr, (float*)m->h, (float*)m->x, m->d, m->V, m->c.rms_eps,
+                                               &m->st->err);
       }
       dg_status st = m->bf ? run_layers<bf16>(m, g, b, 1, n, c0, c0 + n, true, s)
                            : run_layers<float>(m, g, b, 1, n, c0, c0 + n, true, s);

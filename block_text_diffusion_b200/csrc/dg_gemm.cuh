@@ -185,6 +185,167 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 }
 
 // ---------------------------------------------------------------------------
+// Persistent variant for long tile lists (expert GEMMs, LM head): one CTA per
+// SM slot walks tiles blockIdx.x, +gridDim.x, ...  The TMA ring runs across
+// tile boundaries, and the accumulator is double-buffered in TMEM so the
+// epilogue of tile i overlaps the mainloop of tile i+1.
+// Warps: 0 = TMA producer, 1 = MMA issuer, 2..5 = epilogue (warp w drains
+// TMEM lanes 32*(w%4)..+31).  192 threads.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int gemm_total_tiles(const GemmArgs& p, int items_dense) {
+  const int items = p.work ? *p.work_count : items_dense;
+  return p.m_tiles * p.k_splits * items;
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     GemmArgs p, int items_dense) {
+  using C = GemmTcCfg<BN, STAGES>;
+  constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
+  constexpr int kAllocCols = 2 * kAccCols;             // two buffers (<= 512)
+  if (p.skip && *p.skip) return;
+  const int total = gemm_total_tiles(p, items_dense);
+  if ((int)blockIdx.x >= total) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], acc_full[2], acc_empty[2];
+  __shared__ uint32_t tmem_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, kAllocCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;   // global k-block counter across tiles (ring position)
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        GemmTile t;
+        // decode with blockIdx replaced by `tile`
+        t.m_tile = tile % p.m_tiles;
+        const int r = tile / p.m_tiles;
+        t.split = r % p.k_splits;
+        const int item = r / p.k_splits;
+        if (p.work) {
+          const int4 w = p.work[item];
+          t.a_row0 = w.x * p.a_group_rows; t.b_row0 = w.y; t.n_valid = w.z;
+        } else {
+          t.a_row0 = 0; t.b_row0 = item * p.n_tile; t.n_valid = min(p.n_tile, p.N - t.b_row0);
+        }
+        int kb0, kb1;
+        split_range(p, t.split, kb0, kb1);
+        const int n_boxes = min(BN, (t.n_valid + 15) & ~15) / kBoxRowsB;
+        const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (it >= STAGES && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) { ok = false; break; }
+          uint8_t* a_s = smem + s * C::kStage;
+          uint8_t* b_s = a_s + C::kABytes;
+          mbar_expect_tx(&full_bar[s], tx);
+          tma_load_2d(a_s, &tmA, kb * 64, t.a_row0 + t.m_tile * 128, &full_bar[s]);
+          for (int j = 0; j < n_boxes; ++j)
+            tma_load_2d(b_s + j * kBoxRowsB * 128, &tmB, kb * 64, t.b_row0 + j * kBoxRowsB, &full_bar[s]);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        const int m_t = tile % p.m_tiles;
+        const int r = tile / p.m_tiles;
+        const int split = r % p.k_splits;
+        const int item = r / p.k_splits;
+        const int n_valid = p.work ? p.work[item].z : min(p.n_tile, p.N - item * p.n_tile);
+        (void)m_t;
+        int kb0, kb1;
+        split_range(p, split, kb0, kb1);
+        const int n_mma = min(BN, (n_valid + 15) & ~15);
+        const uint32_t idesc = idesc_bf16(128, n_mma);
+        const int buf = local & 1;
+        // wait until the epilogue drained this buffer (use 2 tiles ago)
+        if (local >= 2 && !mbar_wait(&acc_empty[buf], ((local >> 1) & 1) ^ 1, p.err, DGDEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * kAccCols;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&full_bar[s], ph, p.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+          const uint64_t ad = sdesc_sw128(a_addr), bd = sdesc_sw128(a_addr + C::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          tc_commit(&empty_bar[s]);
+        }
+        tc_commit(&acc_full[buf]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      const int m_t = tile % p.m_tiles;
+      const int r = tile / p.m_tiles;
+      const int split = r % p.k_splits;
+      const int item = r / p.k_splits;
+      int n_valid, out_row0;
+      if (p.work) { const int4 w = p.work[item]; n_valid = w.z; out_row0 = w.w; }
+      else { out_row0 = item * p.n_tile; n_valid = min(p.n_tile, p.N - out_row0); }
+      int kb0, kb1;
+      split_range(p, split, kb0, kb1);
+      const int n_mma = min(BN, (n_valid + 15) & ~15);
+      const int buf = local & 1;
+      const bool ok = mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, DGDEV_TIMEOUT_EPI);
+      tc_fence_after();
+      const int m0 = m_t * 128;
+      const bool m_ok = (m0 + row) < p.M;
+      float* outp = p.out + (long long)split * p.split_stride + (long long)out_row0 * p.ldo + m0 + row;
+      if (ok && kb1 > kb0) {
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          float v[16];
+          tmem_ld16(tmem + buf * kAccCols + ((uint32_t)(quad * 32) << 16) + c0, v);
+          if (m_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c0 + j < n_valid) outp[(long long)(c0 + j) * p.ldo] = v[j] * p.alpha;
+          }
+        }
+      } else if (ok && m_ok) {
+        for (int n = 0; n < n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      if (!ok) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kAllocCols);
+}
+
+// ---------------------------------------------------------------------------
 // fp32 SIMT GEMM with the same contract (the fp32 workload's projections):
 // 64 x 64 output tile per CTA, 256 threads, 4 x 4 outputs per thread.
 // ---------------------------------------------------------------------------

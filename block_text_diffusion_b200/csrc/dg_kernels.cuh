@@ -88,6 +88,100 @@ __global__ void k_embed(const int* __restrict__ ids, const T* __restrict__ E, co
   }
 }
 
+// Block-wide sum of one float per thread (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float w = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+    w = warp_sum(w);
+    if (threadIdx.x == 0) red[0] = w;
+  }
+  __syncthreads();
+  const float s = red[0];
+  __syncthreads();
+  return s;
+}
+
+// Normalise the (already stored) row hr into xr: x = h / sqrt(mean(h^2) + eps).
+// Each thread reads back only the elements it wrote itself.
+template <typename T>
+__device__ __forceinline__ void rownorm_store(const T* hr, T* xr, int d, float eps, float ss, float* red) {
+  const float tot = block_sum(ss, red);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)d), eps)));
+  for (int i = threadIdx.x; i < d; i += blockDim.x) xr[i] = from_f<T>(to_f(hr[i]) * r);
+}
+
+// Embedding (+ self-conditioning add) fused with the first RMSNorm:
+// h[t] = E[ids[t]] (+ s[t]);  x[t] = RMSNorm(h[t]).
+template <typename T>
+__global__ void k_embed_norm(const int* __restrict__ ids, const T* __restrict__ E, const T* __restrict__ sc,
+                             const int* __restrict__ use_sc, T* __restrict__ h, T* __restrict__ x, int d,
+                             int vocab, float eps, int* err) {
+  __shared__ float red[32];
+  const long long t = blockIdx.x;
+  int id = ids[t];
+  if (id < 0 || id >= vocab) { dev_error(err, DGDEV_BAD_INDEX); id = 0; }
+  const bool add = sc != nullptr && (use_sc == nullptr || *use_sc != 0);
+  const T* e = E + (long long)id * d;
+  T* hr = h + t * d;
+  float ss = 0.0f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float v = to_f(e[i]);
+    if (add) v = __fadd_rn(v, to_f(sc[t * d + i]));
+    const T hv = from_f<T>(v);
+    hr[i] = hv;
+    const float f = to_f(hv);
+    ss = fmaf(f, f, ss);
+  }
+  rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
+}
+
+// Attention residual fused with the MoE RMSNorm:
+// h = round(h + sum_s ws[s]);  x = RMSNorm(h).  One CTA per row.
+template <typename T>
+__global__ void k_residual_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ ws,
+                                long long split_stride, int splits, int d, float eps) {
+  __shared__ float red[32];
+  const long long t = blockIdx.x;
+  T* hr = h + t * d;
+  const float* w = ws + t * d;
+  float ss = 0.0f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float v = w[i];
+    for (int s = 1; s < splits; ++s) v += w[s * split_stride + i];
+    const T hv = from_f<T>(to_f(hr[i]) + v);
+    hr[i] = hv;
+    const float f = to_f(hv);
+    ss = fmaf(f, f, ss);
+  }
+  rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
+}
+
+// MoE combine fused with the next RMSNorm (next layer's attention norm, or the
+// final norm after the last layer -- all norms have unit gain):
+// h[t] = round(h[t] + sum_slot gate[t][slot] * y[inv[t*k+slot]]) (slots in
+// order);  x[t] = RMSNorm(h[t]).
+template <typename T>
+__global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ y,
+                                   const int* __restrict__ inv, const float* __restrict__ gate, int k, int d,
+                                   float eps) {
+  __shared__ float red[32];
+  const long long t = blockIdx.x;
+  T* hr = h + t * d;
+  float ss = 0.0f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc = 0.0f;
+    for (int j = 0; j < k; ++j) acc = fmaf(gate[t * k + j], y[(long long)inv[t * k + j] * d + i], acc);
+    const T hv = from_f<T>(to_f(hr[i]) + acc);
+    hr[i] = hv;
+    const float f = to_f(hv);
+    ss = fmaf(f, f, ss);
+  }
+  rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
+}
+
 // RMSNorm (unit gain): x = h / sqrt(mean(h^2) + eps), one CTA per row.
 template <typename T>
 __global__ void k_rmsnorm(const T* __restrict__ h, T* __restrict__ x, int d, float eps) {

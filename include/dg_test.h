@@ -49,16 +49,17 @@ dg_status dg_test_commit(const float* H, const int32_t* tok, const int32_t* amax
 /* Dense GEMM out[split][n][m] = alpha * sum_{k in split} A[m][k] B[n][k]
  * (A [M,K], B [N,K] row-major, bf16 through tcgen05 when bf16 != 0, else
  * fp32 SIMT); out holds k_splits partial slabs of N*M floats; bn in
- * {32,64,128,256} is the token tile (bf16 only).  Allocates (tensor maps
- * only; no device memory). */
+ * {32,64,128,256} is the token tile (bf16 only); flags bit 0 selects the
+ * persistent tile-walking kernel.  Allocates (a 32-byte error word). */
 dg_status dg_test_gemm(const void* A, const void* B, float* out, int32_t M, int32_t N, int32_t K, int32_t bf16,
-                       float alpha, int32_t k_splits, int32_t bn, void* stream);
+                       float alpha, int32_t k_splits, int32_t bn, int32_t flags, void* stream);
 
 /* Grouped GEMM as used by the experts: A [groups*M, K], B [rows, K] with
  * rows ordered by group (counts host int32 [groups]); out [rows, M] fp32,
- * out[r][m] = sum_k A[g(r)*M + m][k] B[r][k].  Allocates. */
+ * out[r][m] = sum_k A[g(r)*M + m][k] B[r][k]; flags as dg_test_gemm.
+ * Allocates. */
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
-                               int32_t K, int32_t bf16, int32_t bn, float* out, void* stream);
+                               int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);
 
 /* Attention kernels (tcgen05 for bf16, SIMT for fp32) plus the split
  * combine, on plain layouts: q [n_canvas*n_q, Hq, hd], k and v

@@ -207,12 +207,13 @@ def _bound(a, b):
 @pytest.mark.parametrize("M,N,K,bn,splits", [
     (128, 16, 64, 32, 1), (256, 256, 512, 256, 1), (300, 200, 200, 256, 1), (1536, 256, 1024, 256, 4),
     (4096, 256, 2816, 256, 4), (1000, 40, 72, 64, 1), (640, 100, 4096, 128, 8), (128, 1, 64, 32, 1)])
-def test_gemm_bf16(M, N, K, bn, splits):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_gemm_bf16(M, N, K, bn, splits, persistent):
     g = np.random.default_rng(M + N + K)
     A = I._bf16_grid(g.standard_normal((M, K)).astype(F32))
     B = I._bf16_grid(g.standard_normal((N, K)).astype(F32))
     out = torch.zeros((splits, N, M), dtype=torch.float32, device="cuda")
-    dg.test_gemm(bf16_tensor(A), bf16_tensor(B), out, alpha=0.5, k_splits=splits, bn=bn)
+    dg.test_gemm(bf16_tensor(A), bf16_tensor(B), out, alpha=0.5, k_splits=splits, bn=bn, persistent=persistent)
     got = host(out).astype(np.float64).sum(axis=0)
     ref = 0.5 * (B.astype(np.float64) @ A.astype(np.float64).T)
     err = np.abs(got - ref)
@@ -238,7 +239,8 @@ def test_gemm_f32():
     (1024, 128, [7, 0, 70, 1], 128, True),
     (1024, 256, [0, 9, 64, 65, 1], 64, False),
 ])
-def test_grouped_gemm(M, K, counts, bn, bf):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     g = np.random.default_rng(sum(counts) + M)
     G = len(counts)
     rows = sum(counts)
@@ -249,7 +251,7 @@ def test_grouped_gemm(M, K, counts, bn, bf):
     At = bf16_tensor(A) if bf else cu(A)
     Bt = bf16_tensor(B) if bf else cu(B)
     out = torch.full((rows, M), float("nan"), dtype=torch.float32, device="cuda")
-    dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn)
+    dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn, persistent=persistent and bf)
     got = host(out).astype(np.float64)
     r0 = 0
     for e, c in enumerate(counts):
