@@ -151,8 +151,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
+    // tcgen05.ld/st are warp-collective: every branch around them is kept
+    // uniform across the warp (wait outcomes are agreed with __all_sync).
     for (int j = 0; j < nblk && ok; ++j) {
-      if (!mbar_wait(&s_full, j & 1, a.err, DGDEV_TIMEOUT_EPI)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full, j & 1, a.err, DGDEV_TIMEOUT_EPI))) { ok = false; break; }
       tc_fence_after();
       const int key0 = (kb_begin + j) * 128;
       // pass 1: block max (scaled to log2 units)
@@ -169,7 +171,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       }
       const float m_new = fmaxf(m_run, mx);
       // PV of the previous block must be done before P and O are touched
-      if (j > 0 && !mbar_wait(&o_done, (j - 1) & 1, a.err, DGDEV_TIMEOUT_EPI)) { ok = false; break; }
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done, (j - 1) & 1, a.err, DGDEV_TIMEOUT_EPI))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
       // pass 2: P = exp2(s - m_new) as bf16 into the swizzled tile
@@ -200,8 +205,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         *reinterpret_cast<uint4*>(rowp + (((ch0) ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4*>(rowp + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      // rescale the running output
-      if (j > 0 && alpha != 1.0f) {
+      // rescale the running output (skipped only when no row of the warp needs it)
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         for (int c0 = 0; c0 < 128; c0 += 16) {
           float v[16];
           tmem_ld16(tO + lane_off + c0, v);
@@ -217,7 +222,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       mbar_arrive(&p_full);
     }
     // epilogue: normalised partial O and log2-sum-exp of this split
-    if (ok && nblk > 0) ok = mbar_wait(&o_done, (nblk - 1) & 1, a.err, DGDEV_TIMEOUT_EPI);
+    if (ok && nblk > 0) ok = __all_sync(0xffffffffu, mbar_wait(&o_done, (nblk - 1) & 1, a.err, DGDEV_TIMEOUT_EPI));
     tc_fence_after();
     // TMEM loads are warp-collective: every lane loads, only valid rows store.
     const bool row_valid = tok < a.n_q;

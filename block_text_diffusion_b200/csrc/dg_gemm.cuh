@@ -157,7 +157,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   }
 
   // Epilogue: TMEM -> registers -> out[(out_row0 + n) * ldo + m0 + row].
-  const bool ok = mbar_wait(&done_bar, 0, p.err, DGDEV_TIMEOUT_EPI);
+  // tcgen05.ld is warp-collective: agree on the wait outcome across the warp.
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(&done_bar, 0, p.err, DGDEV_TIMEOUT_EPI));
   tc_fence_after();
   if (ok && nkb > 0) {
     const int row = warp * 32 + lane;
@@ -317,7 +318,8 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       split_range(p, split, kb0, kb1);
       const int n_mma = min(BN, (n_valid + 15) & ~15);
       const int buf = local & 1;
-      const bool ok = mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, DGDEV_TIMEOUT_EPI);
+      const bool ok =
+          __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, DGDEV_TIMEOUT_EPI));
       tc_fence_after();
       const int m0 = m_t * 128;
       const bool m_ok = (m0 + row) < p.M;
