@@ -78,6 +78,7 @@ def lib():
             "dg_phase_name": ([I32], ctypes.c_char_p),
             "dg_launches_per_round": ([P], I32),
             "dg_expert_counts": ([P, P, P], I32),
+            "dg_debug_trace": ([P, P, P], I32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -176,10 +177,21 @@ class Model:
     def load_kv(self, kv, B, P, k, v, stream=None):
         _check(lib().dg_load_kv(self.h, _ptr(kv), B, P, _ptr(k), _ptr(v), _stream(stream)), "dg_load_kv")
 
-    def touched_experts(self, counts, stream=None):
-        """Distinct experts the most recent MoE layer launch routed to."""
+    def debug_trace(self, h_trace=None, ids_trace=None):
+        """Record per-layer hidden states and routing of later eager calls."""
+        _check(lib().dg_debug_trace(self.h, _ptr(h_trace), _ptr(ids_trace)), "dg_debug_trace")
+
+    def expert_counts(self, counts, stream=None):
+        """Per-layer expert row counts [n_layers, n_experts] of the most recent call."""
         _check(lib().dg_expert_counts(self.h, _ptr(counts), _stream(stream)), "dg_expert_counts")
-        return int((counts > 0).sum().item())
+        return counts
+
+    def touched_experts(self, stream=None):
+        """Distinct experts each layer of the most recent call routed to (list)."""
+        import torch
+        c = torch.zeros((self.w.n_layers, self.w.n_experts), dtype=torch.int32, device="cuda")
+        self.expert_counts(c, stream)
+        return [int(x) for x in (c > 0).sum(dim=1).tolist()]
 
     def profile_step(self, kv, B, P, reps=3, stream=None):
         n = 32

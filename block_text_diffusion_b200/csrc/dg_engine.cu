@@ -116,6 +116,7 @@ struct dg_model {
   float* ws = nullptr;
   float *o_part = nullptr, *lse_part = nullptr;
   int *ids = nullptr, *perm = nullptr, *inv = nullptr, *work_count = nullptr, *counts = nullptr;
+  int* moe_splits = nullptr;         // [2] split-K of the gate|up and down GEMMs (set by permute)
   float* gate = nullptr;
   int4* work = nullptr;
   float *logits = nullptr, *H = nullptr;
@@ -134,6 +135,11 @@ struct dg_model {
   Prof prof;
   int launch_count = 0;
   int cur_phase = PH_CONTROL;
+
+  // optional per-layer trace of eager calls: h after the attention residual
+  // and after the MoE [L][2][T][d] (fp32), routing ids [L][T][k]
+  float* dbg_h = nullptr;
+  int* dbg_ids = nullptr;
 };
 
 namespace {
@@ -216,6 +222,7 @@ struct GemmCall {
   int max_items = 0;
   int bn = 256;
   bool persistent = false;           // walk tiles with one CTA per SM slot
+  const int* k_splits_dev = nullptr; // persistent: split-K count decided on the device (<= splits)
 };
 
 template <int BN, int ST>
@@ -269,6 +276,7 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   a.work = g.work;
   a.work_count = g.work_count;
   a.a_group_rows = g.a_group_rows;
+  a.k_splits_dev = g.persistent ? g.k_splits_dev : nullptr;
   a.err = &m->st->err;
   if (!m->bf) {
     a.m_tiles = cdiv(g.M, 64);
@@ -459,7 +467,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     {
       const int mt = m->bf ? cdiv(qc.M, 128) : cdiv(qc.M, 64);
       const int items = m->bf ? cdiv(Tn, qc.bn) : cdiv(Tn, 64);
-      qc.splits = pick_splits(mt, items, cdiv(d, 64), 8);
+      qc.splits = pick_splits(mt, items, cdiv(d, 64), 4);
       while (qc.splits > 1 && (size_t)qc.splits * Tn * m->nqkv > m->ws_elems) --qc.splits;
       qc.split_stride = (long long)Tn * m->nqkv;
     }
@@ -470,7 +478,8 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       qa.ws = m->ws; qa.split_stride = qc.split_stride; qa.splits = std::min(qc.splits, cdiv(d, 64));
       qa.Hq = m->hq; qa.Hkv = m->hkv; qa.hd = m->hd; qa.n_per = n_per; qa.pos0 = pos0; qa.b0 = b0;
       qa.B = g.B; qa.layer = l; qa.S = g.S; qa.rope = m->rope;
-      k_qkv_post<T><<<Tn, 256, 0, s>>>(qa, (T*)m->q, (T*)g.K, (T*)g.Vt);
+      const dim3 grid(cdiv(Tn, 64), m->hq + 2 * m->hkv);
+      k_qkv_post_tiled<T><<<grid, 256, 0, s>>>(qa, Tn, (T*)m->q, (T*)g.K, (T*)g.Vt);
     }
     // attention
     AttnArgs aa{};
@@ -514,7 +523,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     {
       const int mt = m->bf ? cdiv(d, 128) : cdiv(d, 64);
       const int items = m->bf ? cdiv(Tn, oc.bn) : cdiv(Tn, 64);
-      oc.splits = pick_splits(mt, items, cdiv(nq, 64), 8);
+      oc.splits = pick_splits(mt, items, cdiv(nq, 64), 4);
       while (oc.splits > 1 && (size_t)oc.splits * Tn * d > m->ws_elems) --oc.splits;
       oc.split_stride = (long long)Tn * d;
     }
@@ -522,34 +531,57 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     { LaunchScope ls(m, s, PH_RESIDUAL);
       k_residual_norm<T><<<Tn, 256, 0, s>>>((T*)m->h, (T*)m->x, m->ws, oc.split_stride,
                                             std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
+    if (m->dbg_h)
+      k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
     // MoE
     { LaunchScope ls(m, s, PH_ROUTER);
       const size_t sm = (size_t)(d + m->E) * sizeof(double);
       k_router<T><<<Tn, 256, sm, s>>>((const T*)m->x, (const T*)w.wr, m->rbias, d, m->E, m->k, m->ids,
                                        m->gate); }
+    // expert GEMM split-K factors are picked on the device from the routing
+    // (bf16 persistent path only; the fp32 path keeps one split)
+    const long long gu_stride = (long long)n_pairs * 2 * m->ff, dn_stride = (long long)n_pairs * d;
+    SplitPlan plan{};
+    plan.mt[0] = cdiv(2 * m->ff, 128); plan.kb[0] = cdiv(d, 64);
+    plan.mt[1] = cdiv(d, 128); plan.kb[1] = cdiv(m->ff, 64);
+    plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
+    plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
+    plan.out = m->moe_splits;
     { LaunchScope ls(m, s, PH_PERMUTE);
       k_permute<<<1, 1024, (2 * m->E + 1) * sizeof(int), s>>>(m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
-                                                             m->work, m->work_count, m->counts, &m->st->err); }
+                                                             m->work, m->work_count, m->counts + (size_t)l * m->E,
+                                                             plan, &m->st->err); }
     { LaunchScope ls(m, s, PH_GATHER);
       k_gather<T><<<n_pairs, 128, 0, s>>>((const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
     GemmCall gu;
     gu.tA = &w.tm_gu; gu.tB = &m->tm_xp; gu.A32 = (const float*)w.gu; gu.B32 = (const float*)m->xp;
     gu.lda = d; gu.ldb = d; gu.M = 2 * m->ff; gu.K = d; gu.out = m->ws; gu.ldo = 2 * m->ff;
     gu.work = m->work; gu.work_count = m->work_count; gu.a_group_rows = 2 * m->ff;
-    gu.max_items = max_items; gu.bn = bn_g;
+    gu.max_items = max_items; gu.bn = bn_g; gu.persistent = m->bf;
+    gu.split_stride = gu_stride; gu.k_splits_dev = m->bf ? m->moe_splits : nullptr;
+    gu.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
     { LaunchScope ls(m, s, PH_SWIGLU);
       const long long n = (long long)n_pairs * m->ff;
-      k_swiglu<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(m->ws, m->ff, n, (T*)m->act); }
+      k_swiglu<T><<<std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s>>>(m->ws, m->ff, n, (T*)m->act,
+                                                                        m->moe_splits, gu_stride); }
     GemmCall dn;
     dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
     dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;
     dn.work = m->work; dn.work_count = m->work_count; dn.a_group_rows = d;
-    dn.max_items = max_items; dn.bn = bn_g;
+    dn.max_items = max_items; dn.bn = bn_g; dn.persistent = m->bf;
+    dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
+    dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
       k_moe_combine_norm<T><<<Tn, 256, 0, s>>>((T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
-                                               m->c.rms_eps); }
+                                               m->c.rms_eps, m->moe_splits + 1, dn_stride); }
+    if (m->dbg_h) {
+      k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->h, m->dbg_h + (size_t)(2 * l + 1) * Tn * d,
+                                         (long long)Tn * d);
+      CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)l * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
+                             cudaMemcpyDeviceToDevice, s));
+    }
   }
   CU_TRY(cudaGetLastError());
   return DG_OK;
@@ -669,6 +701,12 @@ void release_graph(dg_model* m) {
 template <typename T>
 dg_status capture_block_graph(dg_model* m, const KvGeom& g) {
   release_graph(m);
+  // the diagnostic trace applies to eager calls only
+  struct NoTrace {
+    dg_model* m; float* h; int* ids;
+    explicit NoTrace(dg_model* mm) : m(mm), h(mm->dbg_h), ids(mm->dbg_ids) { m->dbg_h = nullptr; m->dbg_ids = nullptr; }
+    ~NoTrace() { m->dbg_h = h; m->dbg_ids = ids; }
+  } no_trace(m);
   cudaStream_t cs = m->cap_stream;
   cudaGraph_t graph;
   CU_TRY(cudaGraphCreate(&graph, 0));
@@ -785,6 +823,8 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
     w = std::max(w, Tk * 2 * m->ff);
     w = std::max(w, Tk * d);
     w = std::max(w, 16 * (size_t)m->T_cap * d);
+    // room for up to 8 split-K slabs of the expert GEMMs at small batch
+    w = std::max(w, 8 * std::min<size_t>((size_t)m->T_cap * m->k, 4096) * std::max<size_t>(2 * m->ff, d));
     m->ws_elems = w;
     m->part_rows_cap = 8 * Tw * (size_t)m->hq;
   }
@@ -824,7 +864,8 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   A((void**)&m->inv, Tk * sizeof(int));
   A((void**)&m->work, ((size_t)m->E + Tk / 16 + 8) * sizeof(int4));
   A((void**)&m->work_count, sizeof(int));
-  A((void**)&m->counts, (size_t)m->E * sizeof(int));
+  A((void**)&m->moe_splits, 2 * sizeof(int));
+  A((void**)&m->counts, (size_t)m->L * m->E * sizeof(int));
   A((void**)&m->logits, (size_t)m->T_cap * V * sizeof(float));
   A((void**)&m->H, (size_t)m->T_cap * sizeof(float));
   A((void**)&m->tok, (size_t)m->T_cap * sizeof(int));

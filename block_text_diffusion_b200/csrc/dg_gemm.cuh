@@ -28,6 +28,7 @@ struct GemmArgs {
   const int4* work;        // grouped: (group, b_row0, n_valid, out_row0); nullptr = dense
   int a_group_rows;        // grouped: A rows per group (a_row0 = group * a_group_rows)
   const int* work_count;
+  const int* k_splits_dev; // persistent kernel: split-K factor chosen on the device (overrides k_splits)
   const int* skip;         // optional device flag: nonzero -> every CTA returns at once
   int* err;
 };
@@ -201,11 +202,13 @@ __device__ __forceinline__ int gemm_total_tiles(const GemmArgs& p, int items_den
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     GemmArgs p, int items_dense) {
+                     GemmArgs p_in, int items_dense) {
   using C = GemmTcCfg<BN, STAGES>;
   constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
   constexpr int kAllocCols = 2 * kAccCols;             // two buffers (<= 512)
-  if (p.skip && *p.skip) return;
+  if (p_in.skip && *p_in.skip) return;
+  GemmArgs p = p_in;
+  if (p.k_splits_dev) p.k_splits = max(1, min(*p.k_splits_dev, p.kb_total));
   const int total = gemm_total_tiles(p, items_dense);
   if ((int)blockIdx.x >= total) return;
 

@@ -113,6 +113,16 @@ __device__ __forceinline__ void rownorm_store(const T* hr, T* xr, int d, float e
   for (int i = threadIdx.x; i < d; i += blockDim.x) xr[i] = from_f<T>(to_f(hr[i]) * r);
 }
 
+// Same, for rows written in groups of 4 consecutive elements per thread.
+template <typename T>
+__device__ __forceinline__ void rownorm_store4(const T* hr, T* xr, int d, float eps, float ss, float* red) {
+  const float tot = block_sum(ss, red);
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)d), eps)));
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) xr[i + q] = from_f<T>(to_f(hr[i + q]) * r);
+}
+
 // Embedding (+ self-conditioning add) fused with the first RMSNorm:
 // h[t] = E[ids[t]] (+ s[t]);  x[t] = RMSNorm(h[t]).
 template <typename T>
@@ -148,38 +158,69 @@ __global__ void k_residual_norm(T* __restrict__ h, T* __restrict__ x, const floa
   T* hr = h + t * d;
   const float* w = ws + t * d;
   float ss = 0.0f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float v = w[i];
-    for (int s = 1; s < splits; ++s) v += w[s * split_stride + i];
-    const T hv = from_f<T>(to_f(hr[i]) + v);
-    hr[i] = hv;
-    const float f = to_f(hv);
-    ss = fmaf(f, f, ss);
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
+    float4 v = *reinterpret_cast<const float4*>(w + i);
+    for (int s = 1; s < splits; ++s) {
+      const float4 v2 = *reinterpret_cast<const float4*>(w + s * split_stride + i);
+      v.x += v2.x; v.y += v2.y; v.z += v2.z; v.w += v2.w;
+    }
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const T hv = from_f<T>(to_f(hr[i + q]) + vv[q]);
+      hr[i + q] = hv;
+      const float f = to_f(hv);
+      ss = fmaf(f, f, ss);
+    }
   }
-  rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
+  rownorm_store4<T>(hr, x + t * d, d, eps, ss, red);
 }
 
 // MoE combine fused with the next RMSNorm (next layer's attention norm, or the
 // final norm after the last layer -- all norms have unit gain):
 // h[t] = round(h[t] + sum_slot gate[t][slot] * y[inv[t*k+slot]]) (slots in
 // order);  x[t] = RMSNorm(h[t]).
+// y holds `splits` partial slabs (split_stride apart; count read from the
+// device) that are summed before weighting.  Vectorised by 4 (d % 64 == 0).
 template <typename T>
 __global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ y,
                                    const int* __restrict__ inv, const float* __restrict__ gate, int k, int d,
-                                   float eps) {
+                                   float eps, const int* __restrict__ splits_dev, long long split_stride) {
   __shared__ float red[32];
+  __shared__ long long rows[64];
+  __shared__ float gw[64];
   const long long t = blockIdx.x;
+  const int ns = splits_dev ? *splits_dev : 1;
+  if (threadIdx.x < k) {
+    rows[threadIdx.x] = (long long)inv[t * k + threadIdx.x] * d;
+    gw[threadIdx.x] = gate[t * k + threadIdx.x];
+  }
+  __syncthreads();
   T* hr = h + t * d;
   float ss = 0.0f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float acc = 0.0f;
-    for (int j = 0; j < k; ++j) acc = fmaf(gate[t * k + j], y[(long long)inv[t * k + j] * d + i], acc);
-    const T hv = from_f<T>(to_f(hr[i]) + acc);
-    hr[i] = hv;
-    const float f = to_f(hv);
-    ss = fmaf(f, f, ss);
+  for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const float* yp = y + rows[j] + i;
+      float4 v = *reinterpret_cast<const float4*>(yp);
+      for (int s = 1; s < ns; ++s) {
+        const float4 v2 = *reinterpret_cast<const float4*>(yp + s * split_stride);
+        v.x += v2.x; v.y += v2.y; v.z += v2.z; v.w += v2.w;
+      }
+      acc[0] = fmaf(gw[j], v.x, acc[0]);
+      acc[1] = fmaf(gw[j], v.y, acc[1]);
+      acc[2] = fmaf(gw[j], v.z, acc[2]);
+      acc[3] = fmaf(gw[j], v.w, acc[3]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const T hv = from_f<T>(to_f(hr[i + q]) + acc[q]);
+      hr[i + q] = hv;
+      const float f = to_f(hv);
+      ss = fmaf(f, f, ss);
+    }
   }
-  rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
+  rownorm_store4<T>(hr, x + t * d, d, eps, ss, red);
 }
 
 // RMSNorm (unit gain): x = h / sqrt(mean(h^2) + eps), one CTA per row.
@@ -265,6 +306,73 @@ __global__ void k_qkv_post(QkvPostArgs a, T* __restrict__ Q, T* __restrict__ Kc,
   }
 }
 
+// out = float(in) over n elements (diagnostic copies).
+template <typename T>
+__global__ void k_cast_f32(const T* __restrict__ in, float* __restrict__ out, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    out[i] = to_f(in[i]);
+}
+
+// Tiled variant: one CTA per (64-token tile, head), head in [0, Hq + 2 Hkv)
+// (q heads, then k heads, then v heads).  q/k rows are written contiguously;
+// a v tile is transposed through shared memory so each V^T row segment of 64
+// positions is one 128-byte store.  A tile never spans two canvases
+// (n_per % 64 == 0, or a single canvas per launch).
+template <typename T>
+__global__ void __launch_bounds__(256) k_qkv_post_tiled(QkvPostArgs a, int n_tok, T* __restrict__ Q,
+                                                        T* __restrict__ Kc, T* __restrict__ Vt) {
+  __shared__ float vt[128][65];
+  const int t0 = blockIdx.x * 64;
+  const int head = blockIdx.y;
+  const int hd = a.hd, half = hd / 2;
+  const int nq = a.Hq * hd, nk = a.Hkv * hd, ncol = nq + 2 * nk;
+  auto load = [&](long long t, int c) {
+    const float* w = a.ws + t * ncol + c;
+    float v = w[0];
+    for (int s = 1; s < a.splits; ++s) v += w[s * a.split_stride];
+    return v;
+  };
+  if (head < a.Hq + a.Hkv) {
+    const int base = head < a.Hq ? head * hd : nq + (head - a.Hq) * hd;
+    for (int u = threadIdx.x; u < 64 * half; u += blockDim.x) {
+      const int tl = u / half, c = u % half;
+      const int t = t0 + tl;
+      if (t >= n_tok) continue;
+      const int b = a.b0 + t / a.n_per, pos = a.pos0 + t % a.n_per;
+      const float x0 = load(t, base + c), x1 = load(t, base + c + half);
+      const float2 cs = a.rope[(long long)pos * half + c];
+      const float y0 = x0 * cs.x - x1 * cs.y;
+      const float y1 = x0 * cs.y + x1 * cs.x;
+      T* dst;
+      if (head < a.Hq) {
+        dst = Q + ((long long)t * a.Hq + head) * hd;
+      } else {
+        const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + (head - a.Hq);
+        dst = Kc + (lbh * a.S + pos) * hd;
+      }
+      dst[c] = from_f<T>(y0);
+      dst[c + half] = from_f<T>(y1);
+    }
+  } else {
+    const int g = head - a.Hq - a.Hkv;
+    const int base = nq + nk + g * hd;
+    for (int u = threadIdx.x; u < 64 * hd; u += blockDim.x) {
+      const int tl = u / hd, c = u % hd;
+      const int t = t0 + tl;
+      vt[c][tl] = (t < n_tok) ? load(t, base + c) : 0.0f;
+    }
+    __syncthreads();
+    const int tfirst = t0;
+    const int b = a.b0 + tfirst / a.n_per, pos0 = a.pos0 + tfirst % a.n_per;
+    const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + g;
+    const int valid = min(64, n_tok - t0);
+    for (int u = threadIdx.x; u < hd * 64; u += blockDim.x) {
+      const int c = u / 64, tl = u % 64;
+      if (tl < valid) Vt[(lbh * hd + c) * a.S + pos0 + tl] = from_f<T>(vt[c][tl]);
+    }
+  }
+}
+
 // h = round(h + sum_s ws[s]) over [rows][d].
 template <typename T>
 __global__ void k_residual(T* __restrict__ h, const float* __restrict__ ws, long long split_stride,
@@ -313,25 +421,36 @@ __global__ void k_router(const T* __restrict__ x, const T* __restrict__ Wr, cons
     if (lane == 0) logit[e] = acc + (bias ? bias[e] : 0.0);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double sel[64];
-    int sid[64];
+  if (warp == 0) {
+    // k rounds of a warp argmax (ties to the lower expert id); a chosen
+    // expert's logit is replaced by -inf in shared memory.
+    __shared__ double sel[64];
+    __shared__ int sid[64];
     for (int j = 0; j < k; ++j) {
-      int best = -1;
-      for (int e = 0; e < E; ++e) {
-        bool taken = false;
-        for (int q = 0; q < j; ++q) taken |= (sid[q] == e);
-        if (taken) continue;
-        if (best < 0 || logit[e] > logit[best]) best = e;
+      double bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int e = lane; e < E; e += 32) {
+        const double v = logit[e];
+        if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
       }
-      sid[j] = best;
-      sel[j] = logit[best];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if (lane == 0) {
+        sid[j] = bi;
+        sel[j] = bv;
+        logit[bi] = -INFINITY;
+      }
+      __syncwarp();
     }
-    double den = 0.0;
-    for (int j = 0; j < k; ++j) den += exp(sel[j] - sel[0]);
-    for (int j = 0; j < k; ++j) {
-      ids[t * k + j] = sid[j];
-      gate[t * k + j] = (float)(exp(sel[j] - sel[0]) / den);
+    if (lane < k) {
+      double den = 0.0;
+      for (int j = 0; j < k; ++j) den += exp(sel[j] - sel[0]);
+      ids[t * k + lane] = sid[lane];
+      gate[t * k + lane] = (float)(exp(sel[lane] - sel[0]) / den);
     }
   }
 }
@@ -342,9 +461,17 @@ __global__ void k_router(const T* __restrict__ x, const T* __restrict__ Wr, cons
 // first row) cover each expert's rows in tiles of `bn`.  One CTA; warp w
 // places the pairs of experts w, w+32, ... in pair order (stable).
 // ---------------------------------------------------------------------------
+// Split-K factors of the two expert GEMMs, chosen here on the device from the
+// number of work items so that their tiles fill about eight waves of SMs:
+// splits_out[g] for g = 0 (gate|up) and 1 (down) from (m tiles, k blocks, cap).
+struct SplitPlan {
+  int mt[2], kb[2], cap[2];
+  int* out;
+};
+
 __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int bn, int* __restrict__ perm,
                           int* __restrict__ inv, int4* __restrict__ work, int* __restrict__ work_count,
-                          int* __restrict__ counts_out, int* err) {
+                          int* __restrict__ counts_out, SplitPlan plan, int* err) {
   extern __shared__ int psm[];
   int* counts = psm;         // [E]
   int* offs = psm + E;       // [E + 1]
@@ -366,6 +493,13 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
     }
     offs[E] = acc;
     *work_count = nw;
+    if (plan.out) {
+      for (int g = 0; g < 2; ++g) {
+        int s = (8 * 148) / max(1, plan.mt[g] * nw);
+        s = min(s, max(1, plan.kb[g] / 4));
+        plan.out[g] = max(1, min(s, plan.cap[g]));
+      }
+    }
   }
   __syncthreads();
   if (counts_out)
@@ -399,14 +533,29 @@ __global__ void k_gather(const T* __restrict__ x, const int* __restrict__ perm, 
   for (int i = threadIdx.x; i < nv; i += blockDim.x) o[i] = s[i];
 }
 
-// SwiGLU: a = round(silu(g) * u), g/u the gate and up halves of each row.
+// SwiGLU: a = round(silu(g) * u), g/u the gate and up halves of each row,
+// each summed over the split-K partials (count read from the device).
 template <typename T>
-__global__ void k_swiglu(const float* __restrict__ gu, int ff, long long n, T* __restrict__ a) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+__global__ void k_swiglu(const float* __restrict__ gu, int ff, long long n, T* __restrict__ a,
+                         const int* __restrict__ splits_dev, long long split_stride) {
+  const int ns = splits_dev ? *splits_dev : 1;
+  const long long n4 = n / 4;   // ff is a multiple of 64
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {
-    const long long r = i / ff, c = i % ff;
-    const float g = gu[r * 2 * ff + c], u = gu[r * 2 * ff + ff + c];
-    a[i] = from_f<T>(g / (1.0f + expf(-g)) * u);
+    const long long e = i * 4, r = e / ff, c = e % ff;
+    const float* gp = gu + r * 2 * ff + c;
+    float4 g = *reinterpret_cast<const float4*>(gp);
+    float4 u = *reinterpret_cast<const float4*>(gp + ff);
+    for (int s = 1; s < ns; ++s) {
+      const float4 g2 = *reinterpret_cast<const float4*>(gp + s * split_stride);
+      const float4 u2 = *reinterpret_cast<const float4*>(gp + s * split_stride + ff);
+      g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
+      u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+    }
+    a[e] = from_f<T>(g.x / (1.0f + expf(-g.x)) * u.x);
+    a[e + 1] = from_f<T>(g.y / (1.0f + expf(-g.y)) * u.y);
+    a[e + 2] = from_f<T>(g.z / (1.0f + expf(-g.z)) * u.z);
+    a[e + 3] = from_f<T>(g.w / (1.0f + expf(-g.w)) * u.w);
   }
 }
 

@@ -89,10 +89,17 @@ dg_status dg_profile_step(dg_model* model, void* kv, int32_t B, int32_t P, int32
 /* Name of profile phase i, or NULL past the last one. */
 const char* dg_phase_name(int32_t i);
 
-/* Per-expert row counts of the most recent MoE layer launch (device int32
- * [n_experts]); the number of nonzero entries is the distinct experts that
- * layer streamed. */
+/* Per-layer, per-expert row counts of the most recent call (device int32
+ * [n_layers][n_experts]); the nonzero entries of row l are the distinct
+ * experts layer l streamed. */
 dg_status dg_expert_counts(const dg_model* model, int32_t* counts, void* stream);
+
+/* Diagnostic trace of later eager calls (dg_denoise_step, dg_encode_prompt):
+ * for every layer l, h after the attention residual -> h_trace[l][0][T][d]
+ * and after the MoE -> h_trace[l][1][T][d] (fp32), and the routing ids ->
+ * ids_trace[l][T][top_k] (T = tokens of the call).  Both NULL turns it off;
+ * the block-loop graph never traces.  Buffers are the caller's. */
+dg_status dg_debug_trace(dg_model* model, float* h_trace, int32_t* ids_trace);
 
 /* Kernel launches recorded in one captured block-loop round (graph body). */
 int32_t dg_launches_per_round(const dg_model* model);

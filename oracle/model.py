@@ -220,10 +220,79 @@ def _proj(x, w):
     return x @ np.asarray(w, dtype=np.float64).T
 
 
-def block(model, layer, h, positions, k_prefix, v_prefix, causal):
+def router_margin(x, wr, top_k, zipf_s=0.0):
+    """Gap between the k-th and (k+1)-th largest router logit per token (how
+    close the top-k decision is to a tie; +inf when k = E).  Diagnostic only."""
+    r = np.asarray(x, dtype=np.float64) @ np.asarray(wr, dtype=np.float64).T
+    if zipf_s:
+        r = r + (-zipf_s * np.log(np.arange(wr.shape[0], dtype=np.float64) + 1.0))[None, :]
+    if top_k >= r.shape[1]:
+        return np.full(r.shape[0], np.inf)
+    s = -np.sort(-r, axis=1)
+    return s[:, top_k - 1] - s[:, top_k]
+
+
+def routing_alternatives(r_row, top_k, delta):
+    """Every top-k selection that is correct within `delta` of rounding.
+
+    r_row: router logits of one token (bias included).  The primary selection
+    is the k largest (ties to the lower id).  When the decision boundary is
+    within delta -- a selected expert whose logit is less than delta above the
+    best unselected one -- swapping that pair gives another selection that
+    rounding of the inputs can legitimately produce.  Returns a list of
+    (ids, gate weights) with the primary first; ids in descending-logit slot
+    order, gate weights the softmax over the selected logits."""
+    r = np.asarray(r_row, dtype=np.float64)
+    E = r.size
+    order = sorted(range(E), key=lambda e: (-r[e], e))
+    sel, rest = order[:top_k], order[top_k:]
+    sets = [sel]
+    if rest:
+        best_out = r[rest[0]]
+        worst_in = r[sel[-1]]
+        c_in = [e for e in sel if r[e] - best_out < delta]
+        c_out = [e for e in rest if worst_in - r[e] < delta]
+        for a in c_in:
+            for b in c_out:
+                alt = [e for e in sel if e != a] + [b]
+                sets.append(sorted(alt, key=lambda e: (-r[e], e)))
+    out = []
+    for s in sets:
+        v = r[s]
+        ex = np.exp(v - v.max())
+        out.append((np.array(s, dtype=np.int32), ex / ex.sum()))
+    return out
+
+
+def token_logits_with_routing(model, layer, h_attn_row, ids, gates):
+    """Logits of one token of a single-layer model whose MoE uses the given
+    selection: h = store(h_attn + sum_j g_j FFN_{e_j}(x)), x = store(RMSNorm(h_attn)),
+    logits = logit_scale * store(RMSNorm(h)) E^T.  Diagnostic / parity helper."""
+    cfg = model.cfg
+    h = np.asarray(h_attn_row, dtype=np.float64)[None, :]
+    x = model.store(rmsnorm(h, cfg.rms_eps))
+    y = np.zeros_like(h)
+    for e, g in zip(ids, gates):
+        a = model.store(silu(x @ layer.wg[e].astype(np.float64).T) * (x @ layer.wu[e].astype(np.float64).T))
+        y += g * (a @ layer.wd[e].astype(np.float64).T)
+    h = model.store(h + y)
+    xf = model.store(rmsnorm(h, cfg.rms_eps))
+    return (cfg.logit_scale * _proj(xf, model.embed))[0]
+
+
+def router_logits(x, wr, zipf_s=0.0):
+    """Router logits x Wr^T (+ Zipf bias), float64."""
+    r = np.asarray(x, dtype=np.float64) @ np.asarray(wr, dtype=np.float64).T
+    if zipf_s:
+        r = r + (-zipf_s * np.log(np.arange(wr.shape[0], dtype=np.float64) + 1.0))[None, :]
+    return r
+
+
+def block(model, layer, h, positions, k_prefix, v_prefix, causal, trace=None):
     """One pre-norm transformer block over n tokens.  k_prefix/v_prefix are
     cached keys/values [n_prefix, Hkv, hd] the tokens also attend to.  Returns
-    (h_out, k_new, v_new) with k_new/v_new the stored keys/values of the tokens."""
+    (h_out, k_new, v_new) with k_new/v_new the stored keys/values of the tokens.
+    `trace` (a list) receives the intermediate states for diagnostics."""
     cfg = model.cfg
     n = h.shape[0]
     hq, hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
@@ -237,7 +306,12 @@ def block(model, layer, h, positions, k_prefix, v_prefix, causal):
     h = model.store(h + _proj(o.reshape(n, hq * hd), layer.wo))
     x2 = model.store(rmsnorm(h, cfg.rms_eps))
     y, ids, w = moe(model, layer, x2)
+    if trace is not None:
+        trace.append(dict(h_attn=h.copy(), ids=ids, margin=router_margin(x2, layer.wr, cfg.top_k, cfg.zipf_s),
+                          router=router_logits(x2, layer.wr, cfg.zipf_s)))
     h = model.store(h + y)
+    if trace is not None:
+        trace[-1]["h_out"] = h.copy()
     return h, k, v
 
 
@@ -258,7 +332,7 @@ def encode_prompt(model, prompt):
 
 
 # --- one denoising step ----------------------------------------------------------
-def forward_canvas(model, K, V, canvas, selfcond):
+def forward_canvas(model, K, V, canvas, selfcond, trace=None):
     """Bidirectional canvas pass.  K, V: prompt cache [L, Hkv, P, hd];
     canvas [256] ids; selfcond [256, d] or None.  Returns float64 logits
     [256, vocab] and the canvas keys/values written per layer."""
@@ -272,7 +346,7 @@ def forward_canvas(model, K, V, canvas, selfcond):
     for l, layer in enumerate(model.layers):
         kp = K[l].transpose(1, 0, 2).astype(np.float64)
         vp = V[l].transpose(1, 0, 2).astype(np.float64)
-        h, k, v = block(model, layer, h, pos, kp, vp, causal=False)
+        h, k, v = block(model, layer, h, pos, kp, vp, causal=False, trace=trace)
         kv_new.append((k, v))
     x = model.store(rmsnorm(h, cfg.rms_eps))
     logits = cfg.logit_scale * _proj(x, model.embed)
@@ -287,12 +361,13 @@ def self_condition(model, probs):
     return model.store(_proj(u, model.wsc))
 
 
-def denoise_step(model, K, V, canvas, selfcond, step, t, canvas_id=0, prev_amax=None, max_steps=None):
+def denoise_step(model, K, V, canvas, selfcond, step, t, canvas_id=0, prev_amax=None, max_steps=None,
+                 trace=None):
     """One round for one canvas.  Returns a dict with logits (float64 and the
     binary32 values the sampler reads), entropy, sampled tokens, argmax,
     commit mask, next canvas, next self-conditioning, stop flag and count."""
     cfg = model.cfg
-    logits64, _ = forward_canvas(model, K, V, canvas, selfcond)
+    logits64, _ = forward_canvas(model, K, V, canvas, selfcond, trace=trace)
     l32 = logits64.astype(F32)
     T = sp.temperature(t, cfg.temp_start, cfg.temp_end)
     inv_t = F32(1.0) / T

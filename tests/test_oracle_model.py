@@ -314,3 +314,35 @@ def test_bf16_storage_rounds_values(micro):
     # bf16 spacing at 1 is 2^-7; exact ties go to the even mantissa
     x = np.array([1.0 + 2 ** -9, 1.0 + 3 * 2 ** -9, -3.14159, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8])
     assert np.array_equal(m.store(x), [1.0, 1.0 + 2 ** -7, -3.140625, 1.0, 1.0 + 2 ** -6])
+
+
+def test_routing_alternatives_pins():
+    g = np.random.default_rng(7)
+    r = g.standard_normal(16)
+    alts = om.routing_alternatives(r, 4, 1e-9)
+    assert len(alts) == 1
+    prim_ids, prim_w = alts[0]
+    assert list(prim_ids) == list(np.argsort(-r, kind="stable")[:4]) and np.isclose(prim_w.sum(), 1.0)
+    # construct a near tie at the boundary: 4th and 5th largest 1e-4 apart
+    s = np.argsort(-r, kind="stable")
+    r2 = r.copy()
+    r2[s[4]] = r2[s[3]] - 1e-4
+    alts = om.routing_alternatives(r2, 4, 1e-3)
+    assert len(alts) == 2
+    assert set(alts[1][0]) == (set(s[:3]) | {s[4]})
+    assert np.isclose(alts[1][1].sum(), 1.0)
+
+
+def test_token_logits_with_routing_reproduces_forward(micro):
+    cfg, model, _ = micro
+    one = om.Model.__new__(om.Model)
+    one.cfg, one.embed, one.wsc, one.layers = cfg.replace(n_layers=1), model.embed, model.wsc, model.layers[:1]
+    K, V = I.prompt_kv(4, 1, 1, cfg.n_kv_heads, 6, cfg.head_dim, bf16=False)
+    c = I.canvas_ids(5, 1, cfg.vocab)[0]
+    trace = []
+    logits, _ = om.forward_canvas(one, K[:, 0], V[:, 0], c, None, trace=trace)
+    for t in (0, 17, 255):
+        ids, w = om.routing_alternatives(trace[0]["router"][t], cfg.top_k, 1e-12)[0]
+        row = om.token_logits_with_routing(one, one.layers[0], trace[0]["h_attn"][t], ids, w)
+        assert np.allclose(row, logits[t], rtol=1e-12, atol=1e-12)
+        assert list(ids) == list(trace[0]["ids"][t])
