@@ -292,11 +292,14 @@ __global__ void k_attn_f32(const float* __restrict__ Q, const float* __restrict_
   if (lane == 0) a.lse_part[gw] = m + log2f(l);
 }
 
-// Merge split partials: o = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M).
+// Merge split partials: o = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),
+// splits in index order.  One warp per (token, head) row; hd % 32 == 0.
 template <typename T>
 __global__ void k_attn_combine(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                                int n_splits, long long rows, int hd, T* __restrict__ out) {
-  const long long row = blockIdx.x;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
   float M = -INFINITY;
   for (int s = 0; s < n_splits; ++s) M = fmaxf(M, lse_part[s * rows + row]);
   float den = 0.0f;
@@ -304,12 +307,20 @@ __global__ void k_attn_combine(const float* __restrict__ o_part, const float* __
     const float l = lse_part[s * rows + row];
     den += (l == -INFINITY) ? 0.0f : exp2f(l - M);
   }
-  for (int c = threadIdx.x; c < hd; c += blockDim.x) {
-    float acc = 0.0f;
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  for (int c0 = lane * 4; c0 < hd; c0 += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < n_splits; ++s) {
       const float l = lse_part[s * rows + row];
-      if (l != -INFINITY) acc += exp2f(l - M) * o_part[(s * rows + row) * hd + c];
+      if (l == -INFINITY) continue;
+      const float wgt = exp2f(l - M);
+      const float4 o = *reinterpret_cast<const float4*>(o_part + (s * rows + row) * hd + c0);
+      acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
     }
-    out[row * hd + c] = from_f<T>(den > 0.0f ? acc / den : 0.0f);
+    T* dst = out + row * hd + c0;
+    dst[0] = from_f<T>(acc.x * inv);
+    dst[1] = from_f<T>(acc.y * inv);
+    dst[2] = from_f<T>(acc.z * inv);
+    dst[3] = from_f<T>(acc.w * inv);
   }
 }

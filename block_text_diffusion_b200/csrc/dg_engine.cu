@@ -90,7 +90,7 @@ struct Prof {
 
 struct LayerW {
   void *qkv = nullptr, *wo = nullptr, *wr = nullptr, *gu = nullptr, *wd = nullptr;
-  CUtensorMap tm_qkv, tm_wo, tm_gu, tm_wd;
+  CUtensorMap tm_qkv, tm_wo, tm_gu, tm_wd, tm_wr;
 };
 
 struct dg_model {
@@ -107,7 +107,7 @@ struct dg_model {
   void *emb = nullptr, *embT = nullptr, *Wsc = nullptr;
   std::vector<LayerW> layers;
   float2* rope = nullptr;
-  double* rbias = nullptr;
+  float* rbias = nullptr;
   CUtensorMap tm_E, tm_ET, tm_Wsc;
 
   void *h = nullptr, *x = nullptr, *q = nullptr, *o = nullptr, *xp = nullptr, *act = nullptr;
@@ -398,6 +398,7 @@ dg_status build_maps(dg_model* m) {
     ok &= map2d(&w.tm_wo, w.wo, d, (uint64_t)m->hq * m->hd, 128);
     ok &= map2d(&w.tm_gu, w.gu, (uint64_t)m->E * 2 * m->ff, d, 128);
     ok &= map2d(&w.tm_wd, w.wd, (uint64_t)m->E * d, m->ff, 128);
+    ok &= map2d(&w.tm_wr, w.wr, (uint64_t)m->E, d, 128);
   }
   const uint64_t Tw = m->Tw, Tk = (uint64_t)m->Tw * m->k;
   ok &= map2d(&m->tm_x, m->x, Tw, d, kBoxRowsB);
@@ -513,7 +514,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       CU_TRY(cudaGetLastError());
     }
     { LaunchScope ls(m, s, PH_ATTN_COMBINE);
-      k_attn_combine<T><<<(unsigned)rows, 128, 0, s>>>(m->o_part, m->lse_part, aa.n_splits, rows, m->hd,
+      k_attn_combine<T><<<(unsigned)cdiv(rows, 8), 256, 0, s>>>(m->o_part, m->lse_part, aa.n_splits, rows, m->hd,
                                                         (T*)m->o); }
     // output projection + residual
     GemmCall oc;
@@ -534,10 +535,22 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     if (m->dbg_h)
       k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
     // MoE
+    // router logits r = x Wr^T as a small GEMM (fp32 accumulation), then top-k
+    GemmCall rc;
+    rc.tA = &w.tm_wr; rc.tB = &m->tm_x; rc.A32 = (const float*)w.wr; rc.B32 = (const float*)m->x;
+    rc.lda = d; rc.ldb = d; rc.M = m->E; rc.K = d; rc.N = Tn; rc.out = m->ws; rc.ldo = m->E;
+    rc.bn = dense_bn(Tn);
+    {
+      const int mt = m->bf ? cdiv(m->E, 128) : cdiv(m->E, 64);
+      const int items = m->bf ? cdiv(Tn, rc.bn) : cdiv(Tn, 64);
+      rc.splits = pick_splits(mt, items, cdiv(d, 64), 8);
+      while (rc.splits > 1 && (size_t)rc.splits * Tn * m->E > m->ws_elems) --rc.splits;
+      rc.split_stride = (long long)Tn * m->E;
+    }
+    DG_TRY(gemm(m, rc, PH_ROUTER, s));
     { LaunchScope ls(m, s, PH_ROUTER);
-      const size_t sm = (size_t)(d + m->E) * sizeof(double);
-      k_router<T><<<Tn, 256, sm, s>>>((const T*)m->x, (const T*)w.wr, m->rbias, d, m->E, m->k, m->ids,
-                                       m->gate); }
+      k_router_topk<<<cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s>>>(
+          m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, m->E, m->k, Tn, m->ids, m->gate); }
     // expert GEMM split-K factors are picked on the device from the routing
     // (bf16 persistent path only; the fp32 path keeps one split)
     const long long gu_stride = (long long)n_pairs * 2 * m->ff, dn_stride = (long long)n_pairs * d;
@@ -548,7 +561,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
     plan.out = m->moe_splits;
     { LaunchScope ls(m, s, PH_PERMUTE);
-      k_permute<<<1, 1024, (2 * m->E + 1) * sizeof(int), s>>>(m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
+      k_permute<<<1, permute_threads(m->E), permute_smem(m->E), s>>>(m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
                                                              m->work, m->work_count, m->counts + (size_t)l * m->E,
                                                              plan, &m->st->err); }
     { LaunchScope ls(m, s, PH_GATHER);
@@ -845,7 +858,7 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   }
   const int max_pos = cfg->max_prompt + kCanvas;
   A((void**)&m->rope, (size_t)max_pos * (m->hd / 2) * sizeof(float2));
-  A((void**)&m->rbias, (size_t)m->E * sizeof(double));
+  A((void**)&m->rbias, (size_t)m->E * sizeof(float));
   A(&m->h, Tw * d * es);
   A(&m->x, Tw * d * es);
   A(&m->q, Tw * nq * es);
@@ -889,7 +902,7 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   if (st == DG_OK) {
     const int n = max_pos * (m->hd / 2);
     k_rope_table<<<cdiv(n, 256), 256, 0, s>>>(m->rope, max_pos, m->hd / 2, m->hd, (double)cfg->rope_theta);
-    k_router_bias<<<cdiv(m->E, 128), 128, 0, s>>>(m->rbias, m->E, (double)cfg->zipf_s);
+    k_router_bias_f32<<<cdiv(m->E, 128), 128, 0, s>>>(m->rbias, m->E, cfg->zipf_s);
     if (cudaGetLastError() != cudaSuccess) st = DG_ERR_CUDA;
   }
   if (st == DG_OK) st = build_maps(m);
@@ -909,9 +922,10 @@ int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   if (!m) return 0;
   (void)B; (void)P;
   // per layer: qkv gemm, qkv post, attention, attention combine, o gemm,
-  // residual+norm, router, permute, gather, gate/up gemm, swiglu, down gemm,
-  // combine+norm; then embed+norm, lm head, sampler, commit, 4 self-cond.
-  return 13 * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
+  // residual+norm, router gemm, router top-k, permute, gather, gate/up gemm,
+  // swiglu, down gemm, combine+norm; then embed+norm, lm head, sampler,
+  // commit, 4 self-cond.
+  return 14 * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          4 /*self-conditioning*/;
 }
 

@@ -63,11 +63,6 @@ __global__ void k_rope_table(float2* __restrict__ tab, int n_pos, int half, int 
   tab[i] = make_float2((float)co, (float)s);
 }
 
-// Router bias b_e = -s ln(e + 1) (Zipf-skewed expert popularity), fp64.
-__global__ void k_router_bias(double* bias, int E, double s) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e < E) bias[e] = s == 0.0 ? 0.0 : -s * log((double)(e + 1));
-}
 
 // ---------------------------------------------------------------------------
 // Embedding (+ self-conditioning add): h[t] = E[ids[t]] (+ s[t]).
@@ -397,62 +392,61 @@ __global__ void k_sum_round(T* __restrict__ out, const float* __restrict__ ws, l
   }
 }
 
+
 // ---------------------------------------------------------------------------
-// Router: r_e = x . Wr[e] (+ b_e) in fp64 (products of stored values are
-// exact, so the top-k decision does not depend on the summation order), top-k
-// by value with ties to the lower expert id, gate weights = softmax over the
-// k selected logits.  One CTA per token.
+// Router top-k on logits produced by the router GEMM: r_e = sum over the
+// split-K partials of x . Wr[e] (fp32 accumulation) + b_e; the k largest
+// (ties to the lower expert id) in descending order; gate weights = softmax
+// over the k selected logits.  One warp per token.
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void k_router(const T* __restrict__ x, const T* __restrict__ Wr, const double* __restrict__ bias,
-                         int d, int E, int k, int* __restrict__ ids, float* __restrict__ gate) {
-  extern __shared__ double rsm[];
-  double* xs = rsm;          // [d]
-  double* logit = rsm + d;   // [E]
-  const long long t = blockIdx.x;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) xs[i] = (double)to_f(x[t * d + i]);
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nw) {
-    const T* w = Wr + (long long)e * d;
-    double acc = 0.0;
-    for (int i = lane; i < d; i += 32) acc = fma((double)to_f(w[i]), xs[i], acc);
-    acc = warp_sum_d(acc);
-    if (lane == 0) logit[e] = acc + (bias ? bias[e] : 0.0);
+__global__ void k_router_topk(const float* __restrict__ r, int splits, long long split_stride,
+                              const float* __restrict__ bias, int E, int k, int n_tok, int* __restrict__ ids,
+                              float* __restrict__ gate) {
+  extern __shared__ float rt[];   // [warps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long t = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= n_tok) return;
+  float* lg = rt + warp * E;
+  for (int e = lane; e < E; e += 32) {
+    float v = r[t * E + e];
+    for (int s = 1; s < splits; ++s) v += r[s * split_stride + t * E + e];
+    lg[e] = v + (bias ? bias[e] : 0.0f);
   }
-  __syncthreads();
-  if (warp == 0) {
-    // k rounds of a warp argmax (ties to the lower expert id); a chosen
-    // expert's logit is replaced by -inf in shared memory.
-    __shared__ double sel[64];
-    __shared__ int sid[64];
-    for (int j = 0; j < k; ++j) {
-      double bv = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int e = lane; e < E; e += 32) {
-        const double v = logit[e];
-        if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
-      }
+  __syncwarp();
+  float sel = 0.0f, top = 0.0f;
+  int sid = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      const float v = lg[e];
+      if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+    }
 #pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
-      if (lane == 0) {
-        sid[j] = bi;
-        sel[j] = bv;
-        logit[bi] = -INFINITY;
-      }
-      __syncwarp();
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    if (lane < k) {
-      double den = 0.0;
-      for (int j = 0; j < k; ++j) den += exp(sel[j] - sel[0]);
-      ids[t * k + lane] = sid[lane];
-      gate[t * k + lane] = (float)(exp(sel[lane] - sel[0]) / den);
-    }
+    if (j == 0) top = bv;
+    if (lane == j) { sel = bv; sid = bi; }
+    if (lane == 0) lg[bi] = -INFINITY;
+    __syncwarp();
   }
+  const float ex = lane < k ? expf(sel - top) : 0.0f;
+  float den = ex;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    ids[t * k + lane] = sid;
+    gate[t * k + lane] = ex / den;
+  }
+}
+
+// Router bias b_e = -s ln(e + 1) in fp32 (Zipf-skewed expert popularity).
+__global__ void k_router_bias_f32(float* bias, int E, float s) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < E) bias[e] = s == 0.0f ? 0.0f : (float)(-(double)s * log((double)(e + 1)));
 }
 
 // ---------------------------------------------------------------------------
@@ -472,24 +466,48 @@ struct SplitPlan {
 __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int bn, int* __restrict__ perm,
                           int* __restrict__ inv, int4* __restrict__ work, int* __restrict__ work_count,
                           int* __restrict__ counts_out, SplitPlan plan, int* err) {
+  // Warp w owns the contiguous pair range [w*chunk, (w+1)*chunk).  A pair's
+  // position is offs[e] (pairs of lower experts) + pairs of expert e in
+  // earlier warps + pairs of e earlier in this warp's range, which keeps the
+  // (token, slot) order within each expert.
   extern __shared__ int psm[];
-  int* counts = psm;         // [E]
-  int* offs = psm + E;       // [E + 1]
-  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+  const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* hist = psm;                  // [nwarps][E]
+  int* offs = psm + nwarps * E;     // [E + 1]
+  for (int i = threadIdx.x; i < nwarps * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
-    const int e = ids[p];
-    if (e < 0 || e >= E) { dev_error(err, DGDEV_BAD_INDEX); continue; }
-    atomicAdd(&counts[e], 1);
+  const int chunk = (n_pairs + nwarps - 1) / nwarps;
+  const int p_begin = min(n_pairs, warp * chunk), p_end = min(n_pairs, p_begin + chunk);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int* my = hist + warp * E;
+  for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+    const int p = p0 + lane;
+    int e = p < p_end ? ids[p] : -1;
+    if (e >= E || (p < p_end && e < 0)) { dev_error(err, DGDEV_BAD_INDEX); e = -1; }
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (same & lt_mask) == 0) my[e] += __popc(same);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert: exclusive prefix over warps; the total goes to offs[e]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int acc = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = acc;
+      acc += c;
+    }
+    offs[e] = acc;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0, nw = 0;
     for (int e = 0; e < E; ++e) {
+      const int c = offs[e];
+      if (counts_out) counts_out[e] = c;
       offs[e] = acc;
-      for (int r = 0; r < counts[e]; r += bn)
-        work[nw++] = make_int4(e, acc + r, min(bn, counts[e] - r), acc + r);
-      acc += counts[e];
+      for (int r = 0; r < c; r += bn) work[nw++] = make_int4(e, acc + r, min(bn, c - r), acc + r);
+      acc += c;
     }
     offs[E] = acc;
     *work_count = nw;
@@ -502,24 +520,26 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
     }
   }
   __syncthreads();
-  if (counts_out)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) counts_out[e] = counts[e];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nwarps) {
-    int base = offs[e];
-    for (int p0 = 0; p0 < n_pairs; p0 += 32) {
-      const int p = p0 + lane;
-      const bool hit = p < n_pairs && ids[p] == e;
-      const unsigned m = __ballot_sync(0xffffffffu, hit);
-      if (hit) {
-        const int pos = base + __popc(m & ((1u << lane) - 1u));
-        perm[pos] = p;
-        inv[p] = pos;
-      }
-      base += __popc(m);
+  for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+    const int p = p0 + lane;
+    int e = p < p_end ? ids[p] : -1;
+    if (e >= E) e = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int pos = offs[e] + my[e] + __popc(same & lt_mask);
+      perm[pos] = p;
+      inv[p] = pos;
     }
+    __syncwarp();
+    if (e >= 0 && (same & lt_mask) == 0) my[e] += __popc(same);
+    __syncwarp();
   }
 }
+
+// Threads of the permute kernel: whole warps, with the per-warp histograms
+// kept within 48 KB of shared memory.
+inline int permute_threads(int E) { return 32 * std::max(1, std::min(32, 12288 / std::max(1, E) - 2)); }
+inline size_t permute_smem(int E) { return ((size_t)(permute_threads(E) / 32) * E + E + 1) * sizeof(int); }
 
 // xp[pos] = x[perm[pos] / k]: expert-ordered copy of the normalised rows.
 template <typename T>
