@@ -79,6 +79,7 @@ def lib():
             "dg_launches_per_round": ([P], I32),
             "dg_expert_counts": ([P, P, P], I32),
             "dg_debug_trace": ([P, P, P], I32),
+            "dg_gemm_splitk_noalloc": ([P, P, P, I32, I32, I32, I32, P], I32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -255,3 +256,14 @@ def test_attention(q, k, v, n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out,
     _check(lib().dg_test_attention(_ptr(q), _ptr(k), _ptr(v), n_canvas, n_q, q_pos0, n_keys, int(causal), Hq,
                                    Hkv, hd, 1 if q.dtype == torch.bfloat16 else 0, _ptr(out), _stream(stream)),
            "dg_test_attention")
+
+
+def gemm_splitk_noalloc(A, B, out, k_splits=1, stream=None):
+    """out[n][m] = sum_k A[m][k] B[n][k] (bf16 in, fp32 out) through the
+    entry point that allocates no device memory (its split-K partial sums
+    live in a fixed-size array inside the library).  For callers that must
+    not call cudaMalloc: see dg_gemm_splitk_noalloc in include/dg.h."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check(lib().dg_gemm_splitk_noalloc(_ptr(A), _ptr(B), _ptr(out), M, N, K, k_splits, _stream(stream)),
+           "dg_gemm_splitk_noalloc")

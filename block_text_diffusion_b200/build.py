@@ -37,7 +37,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = [nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH, "-Xcompiler", "-fPIC", "-shared",
-           "-o", tmp, os.path.join(HERE, "csrc", "dg_engine.cu")]
+           "-o", tmp, os.path.join(HERE, "csrc", "dg_engine.cu"), os.path.join(HERE, "csrc", "dg_noalloc.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)

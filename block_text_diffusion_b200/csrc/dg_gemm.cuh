@@ -354,7 +354,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
 // fp32 SIMT GEMM with the same contract (the fp32 workload's projections):
 // 64 x 64 output tile per CTA, 256 threads, 4 x 4 outputs per thread.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
+static __global__ void __launch_bounds__(256)
 k_gemm_f32(const float* __restrict__ A, long long lda, const float* __restrict__ B, long long ldb,
            int K, GemmArgs p) {
   if (p.skip && *p.skip) return;

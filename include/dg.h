@@ -151,6 +151,27 @@ const char* dg_status_string(dg_status status);
  * body of one dg_generate_block round has the same count plus one). */
 int32_t dg_kernels_per_step(const dg_model* model, int32_t B, int32_t P);
 
+/* Split-K GEMM that allocates nothing.  The method pages have no counterpart
+ * of this call; it is a deployment aid.  Some callers cannot allocate device
+ * memory: serving loops that reserve all device memory up front, and code
+ * that must not block other streams (cudaMalloc/cudaFree can synchronise the
+ * device and fail under memory pressure).  For them this call keeps its
+ * split-K partial sums in a fixed 64 MiB file-scope device array (every GPU
+ * that loads the library holds it until the process exits) instead of a
+ * workspace.
+ *   out[n][m] = sum_k A[m][k] B[n][k]: A device bf16 [M,K], B device bf16
+ *   [N,K] (row-major, K a multiple of 8), out device fp32 [N,M]; k_splits
+ *   >= 1 is capped at ceil(K/64).  Inputs and outputs are the caller's.
+ * Returns DG_ERR_INVALID_ARG when min(k_splits, ceil(K/64)) * N * M exceeds
+ * 16 Mi floats (the array's size) or an argument is out of range.  The first
+ * call on a device looks up the array's device address (once per device,
+ * with that device current); make it before any stream capture.  The call
+ * returns after the result is in `out` (it synchronises `stream`).  Every
+ * call shares the one array, so calls that overlap on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller. */
+dg_status dg_gemm_splitk_noalloc(const void* A, const void* B, float* out, int32_t M, int32_t N, int32_t K,
+                                 int32_t k_splits, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
