@@ -42,6 +42,7 @@ constexpr int kAttnSmem = 32768 /*Q*/ + 2 * 65536 /*K,V x2*/ + 32768 /*P*/ + 102
 __global__ void __launch_bounds__(kAttnThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                 // 2 x [128 rows][128 B]
@@ -260,6 +261,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 // ---------------------------------------------------------------------------
 __global__ void k_attn_f32(const float* __restrict__ Q, const float* __restrict__ Kc,
                            const float* __restrict__ Vt, int S, int hd, AttnArgs a) {
+  pdl_enter();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = a.n_canvas * a.n_q * a.Hq;
@@ -297,6 +299,7 @@ __global__ void k_attn_f32(const float* __restrict__ Q, const float* __restrict_
 template <typename T>
 __global__ void k_attn_combine(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                                int n_splits, long long rows, int hd, T* __restrict__ out) {
+  pdl_enter();
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;

@@ -23,6 +23,15 @@ __device__ __forceinline__ void dev_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Programmatic dependent launch: every kernel of the step lets the next
+// kernel in the stream be scheduled at once, and waits for the previous
+// kernel (and its memory) before it touches global memory.  Without the
+// launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // dtype helpers
 // ---------------------------------------------------------------------------

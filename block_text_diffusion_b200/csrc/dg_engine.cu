@@ -161,6 +161,28 @@ dg_status cuda_status(cudaError_t e) {
     if (_e != cudaSuccess) return cuda_status(_e); \
   } while (0)
 
+// Launch with programmatic stream serialisation, so the next kernel's CTAs
+// are dispatched while this one drains (each kernel waits for its
+// predecessor with griddepcontrol.wait before touching global memory).
+// Errors surface through cudaGetLastError like a <<<>>> launch.
+bool g_use_pdl = true;
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_use_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 dg_status dalloc(dg_model* m, void** p, size_t bytes) {
   *p = nullptr;
   if (bytes == 0) bytes = 16;
@@ -237,7 +259,7 @@ dg_status launch_tc(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   const long long grid = (long long)a.m_tiles * a.k_splits * items;
   if (grid <= 0) return DG_OK;
   if (grid > 0x7FFFFFFFLL) return DG_ERR_UNSUPPORTED;
-  k_gemm_tc<BN, ST><<<(unsigned)grid, 128, C::kSmem, s>>>(*g.tA, *g.tB, a);
+  launch_pdl(k_gemm_tc<BN, ST>, (unsigned)grid, 128, C::kSmem, s, *g.tA, *g.tB, a);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -257,7 +279,7 @@ dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   // CTAs per SM allowed by shared memory (228 KB per SM)
   const int per_sm = std::max(1, (228 * 1024) / (C::kSmem + 2048));
   const int grid = (int)std::min<long long>(max_tiles, (long long)kSMs * std::min(per_sm, 2));
-  k_gemm_tc_persistent<BN, ST><<<grid, 192, C::kSmem, s>>>(*g.tA, *g.tB, a, items_dense);
+  launch_pdl(k_gemm_tc_persistent<BN, ST>, grid, 192, C::kSmem, s, *g.tA, *g.tB, a, items_dense);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -284,7 +306,7 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
     const int items = g.work ? g.max_items : cdiv(g.N, 64);
     const long long grid = (long long)a.m_tiles * a.k_splits * items;
     if (grid <= 0) return DG_OK;
-    k_gemm_f32<<<(unsigned)grid, 256, 0, s>>>(g.A32, g.lda, g.B32, g.ldb, g.K, a);
+    launch_pdl(k_gemm_f32, (unsigned)grid, 256, 0, s, g.A32, g.lda, g.B32, g.ldb, g.K, a);
     CU_TRY(cudaGetLastError());
     return DG_OK;
   }
@@ -480,7 +502,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       qa.Hq = m->hq; qa.Hkv = m->hkv; qa.hd = m->hd; qa.n_per = n_per; qa.pos0 = pos0; qa.b0 = b0;
       qa.B = g.B; qa.layer = l; qa.S = g.S; qa.rope = m->rope;
       const dim3 grid(cdiv(Tn, 64), m->hq + 2 * m->hkv);
-      k_qkv_post_tiled<T><<<grid, 256, 0, s>>>(qa, Tn, (T*)m->q, (T*)g.K, (T*)g.Vt);
+      launch_pdl(k_qkv_post_tiled<T>, grid, 256, 0, s, qa, Tn, (T*)m->q, (T*)g.K, (T*)g.Vt);
     }
     // attention
     AttnArgs aa{};
@@ -504,17 +526,17 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
           CU_TRY(cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem));
           attr = true;
         }
-        k_attn_tc<<<base * aa.n_splits, kAttnThreads, kAttnSmem, s>>>(am.q, am.k, am.v, aa);
+        launch_pdl(k_attn_tc, base * aa.n_splits, kAttnThreads, kAttnSmem, s, am.q, am.k, am.v, aa);
       } else {
         aa.q_tiles = 1; aa.n_splits = 1; aa.blocks_per_split = 1;
         const long long threads = rows * 32;
-        k_attn_f32<<<cdiv(threads, 256), 256, 0, s>>>((const float*)m->q, (const float*)g.K,
+        launch_pdl(k_attn_f32, cdiv(threads, 256), 256, 0, s, (const float*)m->q, (const float*)g.K,
                                                       (const float*)g.Vt, g.S, m->hd, aa);
       }
       CU_TRY(cudaGetLastError());
     }
     { LaunchScope ls(m, s, PH_ATTN_COMBINE);
-      k_attn_combine<T><<<(unsigned)cdiv(rows, 8), 256, 0, s>>>(m->o_part, m->lse_part, aa.n_splits, rows, m->hd,
+      launch_pdl(k_attn_combine<T>, (unsigned)cdiv(rows, 8), 256, 0, s, m->o_part, m->lse_part, aa.n_splits, rows, m->hd,
                                                         (T*)m->o); }
     // output projection + residual
     GemmCall oc;
@@ -530,10 +552,10 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     }
     DG_TRY(gemm(m, oc, PH_O_GEMM, s));
     { LaunchScope ls(m, s, PH_RESIDUAL);
-      k_residual_norm<T><<<Tn, 256, 0, s>>>((T*)m->h, (T*)m->x, m->ws, oc.split_stride,
+      launch_pdl(k_residual_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, oc.split_stride,
                                             std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
     if (m->dbg_h)
-      k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
+      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
     // MoE
     // router logits r = x Wr^T as a small GEMM (fp32 accumulation), then top-k
     GemmCall rc;
@@ -549,7 +571,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     }
     DG_TRY(gemm(m, rc, PH_ROUTER, s));
     { LaunchScope ls(m, s, PH_ROUTER);
-      k_router_topk<<<cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s>>>(
+      launch_pdl(k_router_topk, cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s, 
           m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, m->E, m->k, Tn, m->ids, m->gate); }
     // expert GEMM split-K factors are picked on the device from the routing
     // (bf16 persistent path only; the fp32 path keeps one split)
@@ -561,11 +583,11 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
     plan.out = m->moe_splits;
     { LaunchScope ls(m, s, PH_PERMUTE);
-      k_permute<<<1, permute_threads(m->E), permute_smem(m->E), s>>>(m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
+      launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
                                                              m->work, m->work_count, m->counts + (size_t)l * m->E,
                                                              plan, &m->st->err); }
     { LaunchScope ls(m, s, PH_GATHER);
-      k_gather<T><<<n_pairs, 128, 0, s>>>((const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
+      launch_pdl(k_gather<T>, n_pairs, 128, 0, s, (const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
     GemmCall gu;
     gu.tA = &w.tm_gu; gu.tB = &m->tm_xp; gu.A32 = (const float*)w.gu; gu.B32 = (const float*)m->xp;
     gu.lda = d; gu.ldb = d; gu.M = 2 * m->ff; gu.K = d; gu.out = m->ws; gu.ldo = 2 * m->ff;
@@ -576,7 +598,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
     { LaunchScope ls(m, s, PH_SWIGLU);
       const long long n = (long long)n_pairs * m->ff;
-      k_swiglu<T><<<std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s>>>(m->ws, m->ff, n, (T*)m->act,
+      launch_pdl(k_swiglu<T>, std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s, m->ws, m->ff, n, (T*)m->act,
                                                                         m->moe_splits, gu_stride); }
     GemmCall dn;
     dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
@@ -587,15 +609,15 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
-      k_moe_combine_norm<T><<<Tn, 256, 0, s>>>((T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
+      launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
                                                m->c.rms_eps, m->moe_splits + 1, dn_stride); }
     if (m->dbg_h) {
-      k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->h, m->dbg_h + (size_t)(2 * l + 1) * Tn * d,
+      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l + 1) * Tn * d,
                                          (long long)Tn * d);
       CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)l * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
                              cudaMemcpyDeviceToDevice, s));
       if (l == m->L - 1)   // the final normalised state (input of the LM head)
-        k_cast_f32<T><<<kSMs, 256, 0, s>>>((const T*)m->x, m->dbg_h + (size_t)(2 * m->L) * Tn * d,
+        launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->x, m->dbg_h + (size_t)(2 * m->L) * Tn * d,
                                            (long long)Tn * d);
     }
   }
@@ -626,7 +648,7 @@ template <typename T>
 dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_t s) {
   const int B = g.B, Tn = B * kCanvas, d = m->d, V = m->V;
   { LaunchScope ls(m, s, PH_EMBED);
-    k_embed_norm<T><<<Tn, 256, 0, s>>>(io.canvas, (const T*)m->emb, (const T*)io.selfcond, io.use_sc, (T*)m->h,
+    launch_pdl(k_embed_norm<T>, Tn, 256, 0, s, io.canvas, (const T*)m->emb, (const T*)io.selfcond, io.use_sc, (T*)m->h,
                                        (T*)m->x, d, V, m->c.rms_eps, &m->st->err); }
   // the last layer leaves the final RMSNorm(h) in m->x
   DG_TRY(run_layers<T>(m, g, 0, B, kCanvas, g.P, g.P + kCanvas, false, s));
@@ -644,7 +666,7 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     sa.temp_start = m->c.temp_start; sa.temp_end = m->c.temp_end; sa.state = m->st;
     sa.step_override = io.step_override; sa.t_override = io.t_override;
     sa.H = io.entropy; sa.tok = io.tokens; sa.amax = io.argmax;
-    k_sampler<T><<<Tn, 512, 0, s>>>(sa, io.selfcond_next ? (T*)m->probs : nullptr);
+    launch_pdl(k_sampler<T>, Tn, 512, 0, s, sa, io.selfcond_next ? (T*)m->probs : nullptr);
   }
   // commit / re-noise / stop
   {
@@ -662,7 +684,7 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
       ca.n_committed_out = m->ncom_out; ca.canvas_out = m->canvas_out;
     }
     ca.max_steps = io.loop ? m->c.max_steps : m->c.max_steps;
-    k_commit<<<B, 256, 0, s>>>(ca);
+    launch_pdl(k_commit, B, 256, 0, s, ca);
   }
   // self-conditioning for the next round: s' = round(round(p E) W_sc^T)
   if (io.selfcond_next) {
@@ -679,7 +701,7 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     DG_TRY(gemm(m, sc, PH_SC_GEMM, s));
     const long long n = (long long)Tn * d;
     { LaunchScope ls(m, s, PH_SC_ROUND);
-      k_sum_round<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(
+      launch_pdl(k_sum_round<T>, std::min(cdiv(n, 256), kSMs * 16), 256, 0, s, 
           (T*)m->u, m->ws, sc.split_stride, std::min(sc.splits, cdiv(V, 64)), n); }
     GemmCall s2;
     s2.tA = &m->tm_Wsc; s2.tB = &m->tm_u; s2.A32 = (const float*)m->Wsc; s2.B32 = (const float*)m->u;
@@ -693,7 +715,7 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     }
     DG_TRY(gemm(m, s2, PH_SC_GEMM, s));
     { LaunchScope ls(m, s, PH_SC_ROUND);
-      k_sum_round<T><<<std::min(cdiv(n, 256), kSMs * 16), 256, 0, s>>>(
+      launch_pdl(k_sum_round<T>, std::min(cdiv(n, 256), kSMs * 16), 256, 0, s, 
           (T*)io.selfcond_next, m->ws, s2.split_stride, std::min(s2.splits, cdiv(d, 64)), n); }
   }
   CU_TRY(cudaGetLastError());
@@ -743,7 +765,7 @@ dg_status capture_block_graph(dg_model* m, const KvGeom& g) {
   const int before = m->launch_count;
   {
     LaunchScope ls(m, cs, PH_CONTROL);
-    k_round_begin<<<1, 1, 0, cs>>>(m->st);
+    launch_pdl(k_round_begin, 1, 1, 0, cs, m->st);
   }
   RoundIO io{};
   io.canvas = m->canvas_cur;
@@ -756,7 +778,7 @@ dg_status capture_block_graph(dg_model* m, const KvGeom& g) {
   dg_status st = run_round<T>(m, g, io, cs);
   {
     LaunchScope ls(m, cs, PH_CONTROL);
-    k_round_end_cond<<<1, 1, 0, cs>>>(m->st, handle);
+    launch_pdl(k_round_end_cond, 1, 1, 0, cs, m->st, handle);
   }
   cudaGraph_t captured = nullptr;
   e = cudaStreamEndCapture(cs, &captured);
@@ -945,10 +967,10 @@ dg_status dg_encode_prompt(dg_model* m, const int32_t* prompt, int32_t B, int32_
       {
         LaunchScope ls(m, s, PH_EMBED);
         if (m->bf)
-          k_embed_norm<bf16><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const bf16*)m->emb, nullptr, nullptr,
+          launch_pdl(k_embed_norm<bf16>, n, 256, 0, s, prompt + (size_t)b * P + c0, (const bf16*)m->emb, nullptr, nullptr,
                                               (bf16*)m->h, (bf16*)m->x, m->d, m->V, m->c.rms_eps, &m->st->err);
         else
-          k_embed_norm<float><<<n, 256, 0, s>>>(prompt + (size_t)b * P + c0, (const float*)m->emb, nullptr,
+          launch_pdl(k_embed_norm<float>, n, 256, 0, s, prompt + (size_t)b * P + c0, (const float*)m->emb, nullptr,
                                                nullptr, (float*)m->h, (float*)m->x, m->d, m->V, m->c.rms_eps,
                                                &m->st->err);
       }
@@ -984,7 +1006,7 @@ dg_status dg_denoise_step(dg_model* m, void* kv, int32_t B, int32_t P, const int
   io.t_override = t;
   io.loop = false;
   { LaunchScope ls(m, s, PH_CONTROL);
-    k_set_round<<<1, 1, 0, s>>>(m->st, step, t, selfcond ? 1 : 0); }
+    launch_pdl(k_set_round, 1, 1, 0, s, m->st, step, t, selfcond ? 1 : 0); }
   return m->bf ? run_round<bf16>(m, g, io, s) : run_round<float>(m, g, io, s);
 }
 
@@ -996,6 +1018,13 @@ dg_status dg_generate_block(dg_model* m, void* kv, int32_t B, int32_t P, int32_t
   const KvGeom g = kv_geom(m, kv, B, P);
   if (!m->gexec || m->g_kv != kv || m->g_B != B || m->g_P != P) {
     dg_status st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
+    if (st != DG_OK && g_use_pdl) {
+      // a driver that cannot capture programmatic edges into the loop body:
+      // capture the same launches without the attribute
+      cudaGetLastError();
+      g_use_pdl = false;
+      st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
+    }
     if (st != DG_OK) return st;
     m->g_kv = kv; m->g_B = B; m->g_P = P;
   }

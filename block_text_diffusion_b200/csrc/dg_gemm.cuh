@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           GemmArgs p) {
   using C = GemmTcCfg<BN, STAGES>;
+  pdl_enter();
   if (p.skip && *p.skip) return;
   GemmTile t;
   if (!gemm_decode(p, t)) return;
@@ -206,6 +207,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   using C = GemmTcCfg<BN, STAGES>;
   constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
   constexpr int kAllocCols = 2 * kAccCols;             // two buffers (<= 512)
+  pdl_enter();
   if (p_in.skip && *p_in.skip) return;
   GemmArgs p = p_in;
   if (p.k_splits_dev) p.k_splits = max(1, min(*p.k_splits_dev, p.kb_total));
@@ -357,6 +359,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
 static __global__ void __launch_bounds__(256)
 k_gemm_f32(const float* __restrict__ A, long long lda, const float* __restrict__ B, long long ldb,
            int K, GemmArgs p) {
+  pdl_enter();
   if (p.skip && *p.skip) return;
   GemmTile t;
   if (!gemm_decode(p, t)) return;

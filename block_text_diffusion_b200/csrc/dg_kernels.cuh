@@ -64,25 +64,6 @@ __global__ void k_rope_table(float2* __restrict__ tab, int n_pos, int half, int 
 }
 
 
-// ---------------------------------------------------------------------------
-// Embedding (+ self-conditioning add): h[t] = E[ids[t]] (+ s[t]).
-// ---------------------------------------------------------------------------
-template <typename T>
-__global__ void k_embed(const int* __restrict__ ids, const T* __restrict__ E, const T* __restrict__ sc,
-                        const int* __restrict__ use_sc, T* __restrict__ h, int d, int vocab,
-                        int* err) {
-  const int t = blockIdx.x;
-  int id = ids[t];
-  if (id < 0 || id >= vocab) { dev_error(err, DGDEV_BAD_INDEX); id = 0; }
-  const bool add = sc != nullptr && (use_sc == nullptr || *use_sc != 0);
-  const T* e = E + (long long)id * d;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float v = to_f(e[i]);
-    if (add) v = __fadd_rn(v, to_f(sc[(long long)t * d + i]));
-    h[(long long)t * d + i] = from_f<T>(v);
-  }
-}
-
 // Block-wide sum of one float per thread (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
@@ -124,6 +105,7 @@ template <typename T>
 __global__ void k_embed_norm(const int* __restrict__ ids, const T* __restrict__ E, const T* __restrict__ sc,
                              const int* __restrict__ use_sc, T* __restrict__ h, T* __restrict__ x, int d,
                              int vocab, float eps, int* err) {
+  pdl_enter();
   __shared__ float red[32];
   const long long t = blockIdx.x;
   int id = ids[t];
@@ -148,6 +130,7 @@ __global__ void k_embed_norm(const int* __restrict__ ids, const T* __restrict__ 
 template <typename T>
 __global__ void k_residual_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ ws,
                                 long long split_stride, int splits, int d, float eps) {
+  pdl_enter();
   __shared__ float red[32];
   const long long t = blockIdx.x;
   T* hr = h + t * d;
@@ -181,6 +164,7 @@ template <typename T>
 __global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ y,
                                    const int* __restrict__ inv, const float* __restrict__ gate, int k, int d,
                                    float eps, const int* __restrict__ splits_dev, long long split_stride) {
+  pdl_enter();
   __shared__ float red[32];
   __shared__ long long rows[64];
   __shared__ float gw[64];
@@ -218,27 +202,6 @@ __global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const f
   rownorm_store4<T>(hr, x + t * d, d, eps, ss, red);
 }
 
-// RMSNorm (unit gain): x = h / sqrt(mean(h^2) + eps), one CTA per row.
-template <typename T>
-__global__ void k_rmsnorm(const T* __restrict__ h, T* __restrict__ x, int d, float eps) {
-  const long long row = blockIdx.x;
-  const T* hr = h + row * d;
-  float ss = 0.0f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) { const float v = to_f(hr[i]); ss = fmaf(v, v, ss); }
-  __shared__ float red[32];
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
-    v = warp_sum(v);
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(red[0], (float)d), eps)));
-  for (int i = threadIdx.x; i < d; i += blockDim.x) x[row * d + i] = from_f<T>(to_f(hr[i]) * r);
-}
-
 // ---------------------------------------------------------------------------
 // After the QKV projection: sum split-K partials, rotate q and k by RoPE at
 // their absolute positions, round, and scatter q -> Q[t][Hq][hd],
@@ -260,50 +223,10 @@ struct QkvPostArgs {
   const float2* rope;
 };
 
-template <typename T>
-__global__ void k_qkv_post(QkvPostArgs a, T* __restrict__ Q, T* __restrict__ Kc, T* __restrict__ Vt) {
-  const int t = blockIdx.x;
-  const int b = a.b0 + t / a.n_per, i = t % a.n_per, pos = a.pos0 + i;
-  const int hd = a.hd, half = hd / 2;
-  const int nq = a.Hq * hd, nk = a.Hkv * hd;
-  const int ncol = nq + 2 * nk;
-  const float* w = a.ws + (long long)t * ncol;
-  auto load = [&](int c) {
-    float v = w[c];
-    for (int s = 1; s < a.splits; ++s) v += w[s * a.split_stride + c];
-    return v;
-  };
-  // rotary pairs of q and k heads
-  const int n_pairs = (a.Hq + a.Hkv) * half;
-  for (int u = threadIdx.x; u < n_pairs; u += blockDim.x) {
-    const int head = u / half, c = u % half;
-    const int base = head < a.Hq ? head * hd : nq + (head - a.Hq) * hd;
-    const float x0 = load(base + c), x1 = load(base + c + half);
-    const float2 cs = a.rope[(long long)pos * half + c];
-    const float y0 = x0 * cs.x - x1 * cs.y;
-    const float y1 = x0 * cs.y + x1 * cs.x;
-    if (head < a.Hq) {
-      T* q = Q + ((long long)(t) * a.Hq + head) * hd;
-      q[c] = from_f<T>(y0);
-      q[c + half] = from_f<T>(y1);
-    } else {
-      const int g = head - a.Hq;
-      const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + g;
-      T* k = Kc + (lbh * a.S + pos) * hd;
-      k[c] = from_f<T>(y0);
-      k[c + half] = from_f<T>(y1);
-    }
-  }
-  for (int u = threadIdx.x; u < nk; u += blockDim.x) {
-    const int g = u / hd, c = u % hd;
-    const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + g;
-    Vt[(lbh * hd + c) * a.S + pos] = from_f<T>(load(nq + nk + u));
-  }
-}
-
 // out = float(in) over n elements (diagnostic copies).
 template <typename T>
 __global__ void k_cast_f32(const T* __restrict__ in, float* __restrict__ out, long long n) {
+  pdl_enter();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
     out[i] = to_f(in[i]);
 }
@@ -316,6 +239,7 @@ __global__ void k_cast_f32(const T* __restrict__ in, float* __restrict__ out, lo
 template <typename T>
 __global__ void __launch_bounds__(256) k_qkv_post_tiled(QkvPostArgs a, int n_tok, T* __restrict__ Q,
                                                         T* __restrict__ Kc, T* __restrict__ Vt) {
+  pdl_enter();
   __shared__ float vt[128][65];
   const int t0 = blockIdx.x * 64;
   const int head = blockIdx.y;
@@ -368,22 +292,11 @@ __global__ void __launch_bounds__(256) k_qkv_post_tiled(QkvPostArgs a, int n_tok
   }
 }
 
-// h = round(h + sum_s ws[s]) over [rows][d].
-template <typename T>
-__global__ void k_residual(T* __restrict__ h, const float* __restrict__ ws, long long split_stride,
-                           int splits, long long n) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x) {
-    float v = ws[i];
-    for (int s = 1; s < splits; ++s) v += ws[s * split_stride + i];
-    h[i] = from_f<T>(to_f(h[i]) + v);
-  }
-}
-
 // out = round(sum_s ws[s]) over n elements.
 template <typename T>
 __global__ void k_sum_round(T* __restrict__ out, const float* __restrict__ ws, long long split_stride,
                             int splits, long long n) {
+  pdl_enter();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
     float v = ws[i];
@@ -402,6 +315,7 @@ __global__ void k_sum_round(T* __restrict__ out, const float* __restrict__ ws, l
 __global__ void k_router_topk(const float* __restrict__ r, int splits, long long split_stride,
                               const float* __restrict__ bias, int E, int k, int n_tok, int* __restrict__ ids,
                               float* __restrict__ gate) {
+  pdl_enter();
   extern __shared__ float rt[];   // [warps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long t = (long long)blockIdx.x * (blockDim.x >> 5) + warp;
@@ -470,6 +384,7 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
   // position is offs[e] (pairs of lower experts) + pairs of expert e in
   // earlier warps + pairs of e earlier in this warp's range, which keeps the
   // (token, slot) order within each expert.
+  pdl_enter();
   extern __shared__ int psm[];
   const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* hist = psm;                  // [nwarps][E]
@@ -545,6 +460,7 @@ inline size_t permute_smem(int E) { return ((size_t)(permute_threads(E) / 32) * 
 template <typename T>
 __global__ void k_gather(const T* __restrict__ x, const int* __restrict__ perm, int k, int d,
                          T* __restrict__ xp) {
+  pdl_enter();
   const int pos = blockIdx.x;
   const long long src = perm[pos] / k;
   const uint4* s = reinterpret_cast<const uint4*>(x + src * d);
@@ -558,6 +474,7 @@ __global__ void k_gather(const T* __restrict__ x, const int* __restrict__ perm, 
 template <typename T>
 __global__ void k_swiglu(const float* __restrict__ gu, int ff, long long n, T* __restrict__ a,
                          const int* __restrict__ splits_dev, long long split_stride) {
+  pdl_enter();
   const int ns = splits_dev ? *splits_dev : 1;
   const long long n4 = n / 4;   // ff is a multiple of 64
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
@@ -576,18 +493,6 @@ __global__ void k_swiglu(const float* __restrict__ gu, int ff, long long n, T* _
     a[e + 1] = from_f<T>(g.y / (1.0f + expf(-g.y)) * u.y);
     a[e + 2] = from_f<T>(g.z / (1.0f + expf(-g.z)) * u.z);
     a[e + 3] = from_f<T>(g.w / (1.0f + expf(-g.w)) * u.w);
-  }
-}
-
-// h[t] = round(h[t] + sum_slot gate[t][slot] * y[inv[t*k+slot]]), slots in order.
-template <typename T>
-__global__ void k_moe_combine(T* __restrict__ h, const float* __restrict__ y, const int* __restrict__ inv,
-                              const float* __restrict__ gate, int k, int d) {
-  const long long t = blockIdx.x;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float acc = 0.0f;
-    for (int j = 0; j < k; ++j) acc = fmaf(gate[t * k + j], y[(long long)inv[t * k + j] * d + i], acc);
-    h[t * d + i] = from_f<T>(to_f(h[t * d + i]) + acc);
   }
 }
 
@@ -637,6 +542,7 @@ __device__ __forceinline__ ArgBest warp_argmax(ArgBest x) {
 
 template <typename T>
 __global__ void __launch_bounds__(512) k_sampler(SamplerArgs a, T* __restrict__ probs) {
+  pdl_enter();
   const long long row = blockIdx.x;
   const int canvas = (int)(row / a.positions), pos = (int)(row % a.positions);
   const int step = a.step_override >= 0 ? a.step_override : a.state->step;
@@ -767,6 +673,7 @@ struct CommitArgs {
 };
 
 __global__ void __launch_bounds__(256) k_commit(CommitArgs a) {
+  pdl_enter();
   const int b = blockIdx.x, i = threadIdx.x;
   const int n = 256;
   const int step = a.step_override >= 0 ? a.step_override : a.state->step;
@@ -872,6 +779,7 @@ __global__ void __launch_bounds__(256) k_commit(CommitArgs a) {
 // ---------------------------------------------------------------------------
 // Start of a round: t = 1 - s/(N-1) in binary32 (t = 1 when N = 1).
 __global__ void k_round_begin(DevState* st) {
+  pdl_enter();
   const int s = st->step, N = st->n_steps;
   st->t = N <= 1 ? 1.0f : __fsub_rn(1.0f, __fdiv_rn((float)s, (float)(N - 1)));
   st->use_selfcond = s > 0 ? 1 : 0;
@@ -879,6 +787,7 @@ __global__ void k_round_begin(DevState* st) {
 
 // Single-step mode: set the round and time given by the caller.
 __global__ void k_set_round(DevState* st, int step, float t, int use_sc) {
+  pdl_enter();
   st->step = step;
   st->t = t;
   st->use_selfcond = use_sc;
@@ -902,13 +811,9 @@ __global__ void k_loop_init(DevState* st, int n_steps, int n_canvas, int* canvas
   }
 }
 
-// End of a round: advance and decide whether to continue.
-__global__ void k_round_end(DevState* st) {
-  st->step += 1;
-  st->cond = (st->active > 0 && st->step < st->n_steps && st->err == 0) ? 1 : 0;
-}
-
+// End of a round: advance and set the loop's while-condition on the device.
 __global__ void k_round_end_cond(DevState* st, cudaGraphConditionalHandle handle) {
+  pdl_enter();
   st->step += 1;
   const int c = (st->active > 0 && st->step < st->n_steps && st->err == 0) ? 1 : 0;
   st->cond = c;
