@@ -54,8 +54,8 @@ def test_moe26b_one_layer_slice_matches_oracle():
     # one layer of the 26B-A4B shape (d 2816, 16/8 heads, 128 experts top-8,
     # vocab 262144) with its 2048-token prompt cache, against the oracle
     w = I.MOE26B_BF16.replace(n_layers=1, name="moe26b-L1")
-    g, r, trace, om_, gx = ts.run_bf16_round(w, w.prompt_len, 21)
-    ts.compare_bf16_round(g, r, trace, om_, w, gx)
+    g, r, trace, om_, gx, rn, trace_n = ts.run_bf16_round(w, w.prompt_len, 21)
+    ts.compare_bf16_round(g, r, trace, om_, w, gx, rn, trace_n)
 
 
 @pytest.mark.slow
@@ -110,31 +110,34 @@ def test_batch_two_canvases_match_oracle():
     gm.close()
     om_ = om.Model(w)
     for b in range(B):
-        trace = []
-        r = om.denoise_step(om_, K[:, b], V[:, b], canvas[b], None, 0, F32(1.0), canvas_id=b, trace=trace)
+        r, trace, rn, trace_n = ts.oracle_pair(w, K[:, b], V[:, b], canvas[b], canvas_id=b)
         gb = {k: v[b] for k, v in g.items() if v.ndim >= 1 and v.shape[0] == B}
-        ts.compare_bf16_round(gb, r, trace, om_, w, gx[b * 256:(b + 1) * 256], canvas_id=b)
+        ts.compare_bf16_round(gb, r, trace, om_, w, gx[b * 256:(b + 1) * 256], rn, trace_n, canvas_id=b)
     # the Zipf bias skews the load: expert 0 gets far more rows than the last
     assert cnt[0] > 4 * max(1, cnt[-1])
 
 
 def test_batch_32_equals_single_canvas_runs():
     # 32 canvases batched against the same canvases run one at a time (one
-    # layer, so a routing tie moves only its own token): the final normalised
-    # states agree within 2 bf16 ulps on at least 97% of each canvas's tokens
+    # layer, so a routing tie moves only its own token): batching changes
+    # only tile shapes and split-K orders, so the final normalised states
+    # differ by no more than the storage-noise envelope of canvas 0
     w = I.BATCH_ZIPF.replace(n_layers=1)
     B, P = 32, 2048
     gm = dg.Model(w, max_canvases=B, max_prompt=P)
     kv, K, V = synthetic_kv(gm, w, B, P, 41)
     canvas = np.stack([sp.initial_canvas(w.sample_seed, b, 256, w.vocab) for b in range(B)])
     g, gx = ts.traced_round(gm, w, kv, B, P, canvas)
+    _, trace, _, trace_n = ts.oracle_pair(w, K[:, 0], V[:, 0], canvas[0])
+    env = ts.quantiles(ts.rms_ulps(trace_n[-1]["x_final"], trace[-1]["x_final"]))
     for b in (0, 7, 31):
         kv1 = gm.new_kv(1, P)
         gm.load_kv(kv1, 1, P, cu(K[:, b:b + 1]).to(torch.bfloat16), cu(V[:, b:b + 1]).to(torch.bfloat16))
         _, gx1 = ts.traced_round(gm, w, kv1, 1, P, canvas[b:b + 1])
         xb = gx[b * 256:(b + 1) * 256]
-        du = np.abs(gx1 - xb) / ts.ulp_bf16(xb)
-        assert (du.max(axis=1) <= 2.0).mean() >= 0.97
+        du = ts.quantiles(ts.rms_ulps(gx1, xb))
+        print(f"canvas {b}: batched vs single {du}; envelope {env}")
+        assert du[0.5] <= 2 * env[0.5] + 1.0 and du[0.99] <= 2 * env[0.99] + 1.0
     gm.close()
 
 
@@ -144,8 +147,8 @@ def test_long_context_round_matches_oracle():
     # one layer of the long-context workload: 32768-token prompt cache,
     # logit scale 16
     w = I.LONG_CTX.replace(n_layers=1)
-    g, r, trace, om_, gx = ts.run_bf16_round(w, w.prompt_len, 51)
-    ts.compare_bf16_round(g, r, trace, om_, w, gx)
+    g, r, trace, om_, gx, rn, trace_n = ts.run_bf16_round(w, w.prompt_len, 51)
+    ts.compare_bf16_round(g, r, trace, om_, w, gx, rn, trace_n)
 
 
 @pytest.mark.slow
@@ -153,7 +156,12 @@ def test_long_context_round_matches_oracle():
 def test_long_context_block_loop_matches_oracle(layers):
     # the full device block loop of the fast-converging workload (logit scale
     # 16) against the oracle's loop: rounds used, committed count, and the
-    # committed tokens (>= 99%, the workload's multi-round criterion)
+    # committed tokens.  With one layer the loop converges in its first rounds
+    # and the committed tokens must agree on >= 99% (the workload's
+    # multi-round criterion).  With all 8 layers the random-init model does
+    # not converge within the budget, and any storage-rounding difference
+    # sends the sampled trajectory elsewhere; the oracle's own storage-noise
+    # run measures how far, and the device loop must stay within that.
     w = I.LONG_CTX.replace(n_layers=layers)
     P = w.prompt_len
     gm = dg.Model(w)
@@ -165,14 +173,25 @@ def test_long_context_block_loop_matches_oracle(layers):
     gm.sync_status()
     steps, ncom, canvas = int(ts.host(su)[0]), int(ts.host(nc)[0]), ts.host(out)[0]
     gm.close()
-    om_ = om.Model(w)
-    ref = om.generate_block(om_, K[:, 0], V[:, 0])
-    last = ref["trace"][-1]
-    committed = last["commit"] == 1
-    agree = (canvas[committed] == ref["canvas"][committed]).mean() if committed.any() else 1.0
+    ref = om.generate_block(om.Model(w), K[:, 0], V[:, 0])
+    committed = ref["trace"][-1]["commit"] == 1
+
+    def agreement(c):
+        return float((c[committed] == ref["canvas"][committed]).mean()) if committed.any() else 1.0
+    agree = agreement(canvas)
     print(f"long L{layers}: rounds gpu {steps} oracle {ref['steps_used']}; committed gpu {ncom} oracle "
           f"{ref['n_committed']}; committed-token agreement {agree:.4f}; all-token agreement "
           f"{(canvas == ref['canvas']).mean():.4f}")
-    assert steps == ref["steps_used"]
-    assert abs(ncom - ref["n_committed"]) <= max(2, ref["n_committed"] // 50)
-    assert agree >= 0.99
+    if layers == 1:
+        assert steps == ref["steps_used"]
+        assert abs(ncom - ref["n_committed"]) <= max(2, ref["n_committed"] // 50)
+        assert agree >= 0.99
+        return
+    rn = om.generate_block(ts.NoisyStore(w), K[:, 0], V[:, 0])
+    agree_n = agreement(rn["canvas"])
+    print(f"  noise envelope: rounds {rn['steps_used']}; committed {rn['n_committed']}; "
+          f"committed-token agreement {agree_n:.4f}")
+    assert abs(steps - ref["steps_used"]) <= 2 * abs(rn["steps_used"] - ref["steps_used"]) + 1
+    assert abs(ncom - ref["n_committed"]) <= 2 * abs(rn["n_committed"] - ref["n_committed"]) + \
+        max(2, ref["n_committed"] // 20)
+    assert agree >= agree_n - 0.05
