@@ -69,7 +69,6 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t 
 }
 
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
-constexpr int kSMs = 148;
 constexpr int kCanvas = 256;
 constexpr int kEncodeChunk = 4096;
 
@@ -475,7 +474,9 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
   AttnMaps am;
   if (m->bf && !attn_maps(m, g, n_keys, Tn, am)) return DG_ERR_CUDA;
   const int n_pairs = Tn * m->k;
-  const int bn_g = m->bf ? (n_pairs / m->E <= 48 ? 64 : (n_pairs / m->E <= 100 ? 128 : 256)) : 64;
+  // one work item per expert (up to 256 rows): each expert's weights are
+  // streamed once per split however many rows it received
+  const int bn_g = m->bf ? 256 : 64;
   const int max_items = m->E + cdiv(n_pairs, bn_g);
 
   // Precondition: m->x holds RMSNorm(h) of the first layer (written by the
@@ -501,8 +502,8 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       qa.ws = m->ws; qa.split_stride = qc.split_stride; qa.splits = std::min(qc.splits, cdiv(d, 64));
       qa.Hq = m->hq; qa.Hkv = m->hkv; qa.hd = m->hd; qa.n_per = n_per; qa.pos0 = pos0; qa.b0 = b0;
       qa.B = g.B; qa.layer = l; qa.S = g.S; qa.rope = m->rope;
-      const dim3 grid(cdiv(Tn, 64), m->hq + 2 * m->hkv);
-      launch_pdl(k_qkv_post_tiled<T>, grid, 256, 0, s, qa, Tn, (T*)m->q, (T*)g.K, (T*)g.Vt);
+      const long long work = (long long)Tn * (m->hq + m->hkv) * (m->hd / 8) + (long long)m->hkv * (m->hd / 4) * Tn;
+      launch_pdl(k_qkv_post<T>, cdiv(work, 256), 256, 0, s, qa, Tn, (T*)m->q, (T*)g.K, (T*)g.Vt);
     }
     // attention
     AttnArgs aa{};
@@ -666,7 +667,7 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     sa.temp_start = m->c.temp_start; sa.temp_end = m->c.temp_end; sa.state = m->st;
     sa.step_override = io.step_override; sa.t_override = io.t_override;
     sa.H = io.entropy; sa.tok = io.tokens; sa.amax = io.argmax;
-    launch_pdl(k_sampler<T>, Tn, 512, 0, s, sa, io.selfcond_next ? (T*)m->probs : nullptr);
+    CU_TRY(launch_sampler<T>(sa, io.selfcond_next ? (T*)m->probs : nullptr, Tn, s, g_use_pdl));
   }
   // commit / re-noise / stop
   {

@@ -65,9 +65,9 @@ __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& k
 // tcgen05 GEMM, bf16 in / fp32 out.  128 threads: warp 0 lane 0 issues TMA,
 // warp 1 lane 0 issues MMAs, then all four warps drain TMEM (warp w owns
 // accumulator rows 32w..32w+31).  A tiles 128 x 64, B tiles BN x 64 loaded
-// 16 rows per TMA box; STAGES-deep mbarrier ring.
+// 32 rows per TMA box; STAGES-deep mbarrier ring.
 // ---------------------------------------------------------------------------
-constexpr int kBoxRowsB = 16;
+constexpr int kBoxRowsB = 32;
 
 template <int BN, int STAGES>
 struct GemmTcCfg {
@@ -91,7 +91,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   split_range(p, t.split, kb0, kb1);
   const int nkb = kb1 - kb0;
   const int n_mma = min(BN, (t.n_valid + 15) & ~15);
-  const int n_boxes = n_mma / kBoxRowsB;
+  const int n_boxes = (n_mma + kBoxRowsB - 1) / kBoxRowsB;   // B rows loaded >= n_mma (extra rows unused)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -251,7 +251,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
         int kb0, kb1;
         split_range(p, t.split, kb0, kb1);
-        const int n_boxes = min(BN, (t.n_valid + 15) & ~15) / kBoxRowsB;
+        const int n_boxes = (min(BN, (t.n_valid + 15) & ~15) + kBoxRowsB - 1) / kBoxRowsB;
         const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;

@@ -231,64 +231,70 @@ __global__ void k_cast_f32(const T* __restrict__ in, float* __restrict__ out, lo
     out[i] = to_f(in[i]);
 }
 
-// Tiled variant: one CTA per (64-token tile, head), head in [0, Hq + 2 Hkv)
-// (q heads, then k heads, then v heads).  q/k rows are written contiguously;
-// a v tile is transposed through shared memory so each V^T row segment of 64
-// positions is one 128-byte store.  A tile never spans two canvases
-// (n_per % 64 == 0, or a single canvas per launch).
+// QKV post-processing: sum the split-K partials of the fused QKV GEMM, apply
+// rotate-half RoPE to q and k, store q (token-major) and k into the cache,
+// and v transposed into V^T.  Flat grid over two ranges:
+//   [0, n_qk):  thread = (token, q|k head, 4 rotation pairs c..c+3), float4
+//               loads of both halves, 8-byte stores;
+//   [n_qk, ..): thread = (v head, 4 channels, token), token fastest so each
+//               V^T row segment is written by consecutive lanes.
+// Partials are summed in split order.  hd % 8 == 0.
 template <typename T>
-__global__ void __launch_bounds__(256) k_qkv_post_tiled(QkvPostArgs a, int n_tok, T* __restrict__ Q,
-                                                        T* __restrict__ Kc, T* __restrict__ Vt) {
+__global__ void __launch_bounds__(256) k_qkv_post(QkvPostArgs a, int n_tok, T* __restrict__ Q,
+                                                  T* __restrict__ Kc, T* __restrict__ Vt) {
   pdl_enter();
-  __shared__ float vt[128][65];
-  const int t0 = blockIdx.x * 64;
-  const int head = blockIdx.y;
-  const int hd = a.hd, half = hd / 2;
+  const int hd = a.hd, half = hd / 2, q4 = half / 4;
   const int nq = a.Hq * hd, nk = a.Hkv * hd, ncol = nq + 2 * nk;
-  auto load = [&](long long t, int c) {
+  const long long n_qk = (long long)n_tok * (a.Hq + a.Hkv) * q4;
+  const long long n_v = (long long)a.Hkv * (hd / 4) * n_tok;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  auto load4 = [&](long long t, int c) {
     const float* w = a.ws + t * ncol + c;
-    float v = w[0];
-    for (int s = 1; s < a.splits; ++s) v += w[s * a.split_stride];
+    float4 v = *reinterpret_cast<const float4*>(w);
+    for (int s = 1; s < a.splits; ++s) {
+      const float4 u = *reinterpret_cast<const float4*>(w + s * a.split_stride);
+      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+    }
     return v;
   };
-  if (head < a.Hq + a.Hkv) {
+  if (i < n_qk) {
+    const int c = (int)(i % q4) * 4;
+    const long long r = i / q4;
+    const int head = (int)(r % (a.Hq + a.Hkv));
+    const long long t = r / (a.Hq + a.Hkv);
+    const int b = a.b0 + (int)(t / a.n_per), pos = a.pos0 + (int)(t % a.n_per);
     const int base = head < a.Hq ? head * hd : nq + (head - a.Hq) * hd;
-    for (int u = threadIdx.x; u < 64 * half; u += blockDim.x) {
-      const int tl = u / half, c = u % half;
-      const int t = t0 + tl;
-      if (t >= n_tok) continue;
-      const int b = a.b0 + t / a.n_per, pos = a.pos0 + t % a.n_per;
-      const float x0 = load(t, base + c), x1 = load(t, base + c + half);
-      const float2 cs = a.rope[(long long)pos * half + c];
-      const float y0 = x0 * cs.x - x1 * cs.y;
-      const float y1 = x0 * cs.y + x1 * cs.x;
-      T* dst;
-      if (head < a.Hq) {
-        dst = Q + ((long long)t * a.Hq + head) * hd;
-      } else {
-        const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + (head - a.Hq);
-        dst = Kc + (lbh * a.S + pos) * hd;
-      }
-      dst[c] = from_f<T>(y0);
-      dst[c + half] = from_f<T>(y1);
+    const float4 x0 = load4(t, base + c), x1 = load4(t, base + c + half);
+    const float4 r01 = *reinterpret_cast<const float4*>(a.rope + (long long)pos * half + c);
+    const float4 r23 = *reinterpret_cast<const float4*>(a.rope + (long long)pos * half + c + 2);
+    const float lo[4] = {x0.x, x0.y, x0.z, x0.w}, hi[4] = {x1.x, x1.y, x1.z, x1.w};
+    const float cs[4] = {r01.x, r01.z, r23.x, r23.z}, sn[4] = {r01.y, r01.w, r23.y, r23.w};
+    T* dst;
+    if (head < a.Hq) {
+      dst = Q + (t * a.Hq + head) * hd;
+    } else {
+      const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + (head - a.Hq);
+      dst = Kc + (lbh * a.S + pos) * hd;
     }
-  } else {
-    const int g = head - a.Hq - a.Hkv;
-    const int base = nq + nk + g * hd;
-    for (int u = threadIdx.x; u < 64 * hd; u += blockDim.x) {
-      const int tl = u / hd, c = u % hd;
-      const int t = t0 + tl;
-      vt[c][tl] = (t < n_tok) ? load(t, base + c) : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      dst[c + j] = from_f<T>(lo[j] * cs[j] - hi[j] * sn[j]);
+      dst[c + half + j] = from_f<T>(lo[j] * sn[j] + hi[j] * cs[j]);
     }
-    __syncthreads();
-    const int tfirst = t0;
-    const int b = a.b0 + tfirst / a.n_per, pos0 = a.pos0 + tfirst % a.n_per;
+  } else if (i < n_qk + n_v) {
+    const long long iv = i - n_qk;
+    const long long t = iv % n_tok;
+    const long long r = iv / n_tok;
+    const int c = (int)(r % (hd / 4)) * 4;
+    const int g = (int)(r / (hd / 4));
+    const int b = a.b0 + (int)(t / a.n_per), pos = a.pos0 + (int)(t % a.n_per);
+    const float4 v = load4(t, nq + nk + g * hd + c);
     const long long lbh = ((long long)a.layer * a.B + b) * a.Hkv + g;
-    const int valid = min(64, n_tok - t0);
-    for (int u = threadIdx.x; u < hd * 64; u += blockDim.x) {
-      const int c = u / 64, tl = u % 64;
-      if (tl < valid) Vt[(lbh * hd + c) * a.S + pos0 + tl] = from_f<T>(vt[c][tl]);
-    }
+    T* dst = Vt + (lbh * hd + c) * a.S + pos;
+    dst[0] = from_f<T>(v.x);
+    dst[a.S] = from_f<T>(v.y);
+    dst[2 * (long long)a.S] = from_f<T>(v.z);
+    dst[3 * (long long)a.S] = from_f<T>(v.w);
   }
 }
 
@@ -427,10 +433,23 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
     offs[E] = acc;
     *work_count = nw;
     if (plan.out) {
+      // Split-K factor per GEMM: the persistent kernel runs ceil(tiles / SMs)
+      // waves of tiles that each take 1/s of a full-K tile, and every split
+      // adds one fp32 partial slab (written, then read by the consumer).  In
+      // units of the time to stream the group's weights once:
+      //   cost(s) = ceil(mt * nw * s / SMs) / s + s * r,
+      //   r = partial bytes / weight bytes = (n_pairs * 4) / (nw * K * 2) * 2.
       for (int g = 0; g < 2; ++g) {
-        int s = (8 * 148) / max(1, plan.mt[g] * nw);
-        s = min(s, max(1, plan.kb[g] / 4));
-        plan.out[g] = max(1, min(s, plan.cap[g]));
+        const float r = 4.0f * (float)n_pairs / ((float)max(1, nw) * (float)(plan.kb[g] * 64));
+        const int s_max = max(1, min(plan.cap[g], plan.kb[g] / 4));
+        int best = 1;
+        float best_cost = 3.4e38f;
+        for (int s = 1; s <= s_max; ++s) {
+          const int waves = (plan.mt[g] * nw * s + kSMs - 1) / kSMs;
+          const float cost = (float)waves / (float)s + (float)s * r;
+          if (cost < best_cost) { best_cost = cost; best = s; }
+        }
+        plan.out[g] = best;
       }
     }
   }
@@ -540,28 +559,69 @@ __device__ __forceinline__ ArgBest warp_argmax(ArgBest x) {
   return x;
 }
 
+// Vocab-wide sampler pass.  One cluster of kSampCta CTAs per row; CTA r of
+// the cluster owns the contiguous vocab slice [r V/kSampCta, (r+1) V/kSampCta)
+// and keeps it in shared memory, so the logits are read from global memory
+// once.  Partial results are exchanged through distributed shared memory and
+// every CTA combines them in rank order (integer sums are exact, arg-maxima
+// break ties to the lower index), so all CTAs hold the same row values.
+//   pass 1: max / argmax of the logits, and the Gumbel-max key
+//           argmax_v (l_v / T + g_v), g_v = -ln(-ln u_v).  Since
+//           -ln u >= 1 - u, g_v <= -ln(1 - u_v) (1 - u_v is exact in binary32);
+//           the exact g_v is evaluated only where that bound plus a margin
+//           reaches the thread's best key, so the winner is unchanged.
+//   pass 2: e_v = exp(l_v - m) (own binary32 exp), S and U = sum e (l - m) as
+//           truncated Q40 int64; e_v replaces l_v in shared memory.
+//   pass 3: probabilities e_v / S in the storage dtype.
+// ---------------------------------------------------------------------------
+constexpr int kSampCta = 8;        // CTAs per row (one thread-block cluster)
+constexpr int kSampThreads = 256;
+
+struct SampPart {
+  ArgBest m, g;
+  long long s, u;
+};
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
+template <typename P>
+__device__ __forceinline__ const P* cluster_peer(const P* p, int rank) {
+  uint64_t out;
+  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"((uint64_t)p), "r"(rank));
+  return reinterpret_cast<const P*>(out);
+}
+
 template <typename T>
-__global__ void __launch_bounds__(512) k_sampler(SamplerArgs a, T* __restrict__ probs) {
+__global__ void __cluster_dims__(kSampCta, 1, 1) __launch_bounds__(kSampThreads)
+k_sampler(SamplerArgs a, T* __restrict__ probs) {
   pdl_enter();
-  const long long row = blockIdx.x;
+  extern __shared__ float4 sl4[];                 // this CTA's slice (logits, then e)
+  __shared__ SampPart part;
+  __shared__ ArgBest red_m[32], red_g[32];
+  __shared__ long long red_s[32], red_u[32];
+  uint32_t rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  const long long row = blockIdx.x / kSampCta;
   const int canvas = (int)(row / a.positions), pos = (int)(row % a.positions);
   const int step = a.step_override >= 0 ? a.step_override : a.state->step;
   const float t = a.step_override >= 0 ? a.t_override : a.state->t;
   const float temp = __fadd_rn(a.temp_end, __fmul_rn(__fsub_rn(a.temp_start, a.temp_end), t));
   const float inv_t = __fdiv_rn(1.0f, temp);
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32) ^ (uint32_t)canvas;
-  const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab);
-  const int n4 = a.vocab / 4;
+  const int n4 = a.vocab / (4 * kSampCta);        // float4 groups in this slice
+  const int g0 = (int)rank * n4;                  // first global float4 group
+  const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab) + g0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  __shared__ ArgBest red_m[32], red_g[32];
-  __shared__ long long red_s[32], red_u[32];
-  __shared__ float sh_m;
-  __shared__ long long sh_s;
 
   // pass 1
   ArgBest bm{-INFINITY, -1}, bg{-INFINITY, -1};
-  for (int v4 = threadIdx.x; v4 < n4; v4 += blockDim.x) {
-    const float4 l = l4[v4];
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 l = l4[i];
+    sl4[i] = l;
+    const int v4 = g0 + i;
     const uint4 w = philox4x32_10(make_uint4((uint32_t)v4, (uint32_t)pos, (uint32_t)step, STREAM_GUMBEL), k0, k1);
     const float lv[4] = {l.x, l.y, l.z, l.w};
     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
@@ -569,8 +629,14 @@ __global__ void __launch_bounds__(512) k_sampler(SamplerArgs a, T* __restrict__ 
     for (int j = 0; j < 4; ++j) {
       const int v = v4 * 4 + j;
       bm = arg_better(bm, ArgBest{lv[j], v});
-      const float key = __fadd_rn(__fmul_rn(lv[j], inv_t), gumbel_of(wv[j]));
-      bg = arg_better(bg, ArgBest{key, v});
+      const float lt = __fmul_rn(lv[j], inv_t);
+      // 1 - u exactly: u = (2 (x >> 9) + 1) 2^-24
+      const float one_minus_u = (float)(0x1000000u - (((wv[j] >> 9) << 1) | 1u)) * 5.9604644775390625e-8f;
+      const float g_ub = -__logf(one_minus_u);
+      if (bg.i < 0 || lt + g_ub + (1e-3f + 1e-5f * fabsf(bg.v)) >= bg.v) {
+        const float key = __fadd_rn(lt, gumbel_of(wv[j]));
+        bg = arg_better(bg, ArgBest{key, v});
+      }
     }
   }
   bm = warp_argmax(bm);
@@ -582,27 +648,35 @@ __global__ void __launch_bounds__(512) k_sampler(SamplerArgs a, T* __restrict__ 
     ArgBest y = lane < nw ? red_g[lane] : ArgBest{-INFINITY, -1};
     x = warp_argmax(x);
     y = warp_argmax(y);
-    if (lane == 0) {
-      sh_m = x.v;
-      a.amax[row] = x.i;
-      a.tok[row] = y.i;
-    }
+    if (lane == 0) { part.m = x; part.g = y; }
   }
-  __syncthreads();
-  const float m = sh_m;
+  cluster_sync_all();
+  ArgBest M{-INFINITY, -1}, G{-INFINITY, -1};
+  for (int r = 0; r < kSampCta; ++r) {
+    const SampPart* pr = cluster_peer(&part, r);
+    M = arg_better(M, ArgBest{pr->m.v, pr->m.i});
+    G = arg_better(G, ArgBest{pr->g.v, pr->g.i});
+  }
+  if (rank == 0 && threadIdx.x == 0) {
+    a.amax[row] = M.i;
+    a.tok[row] = G.i;
+  }
+  const float m = M.v;
 
   // pass 2
   long long sq = 0, uq = 0;
-  for (int v4 = threadIdx.x; v4 < n4; v4 += blockDim.x) {
-    const float4 l = l4[v4];
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 l = sl4[i];
     const float lv[4] = {l.x, l.y, l.z, l.w};
+    float ev[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float dlt = __fsub_rn(lv[j], m);
-      const float e = dg_expf(dlt);
-      sq += __float2ll_rz(__fmul_rn(e, 1099511627776.0f));
-      uq += __float2ll_rz(__fmul_rn(__fmul_rn(e, dlt), 1099511627776.0f));
+      ev[j] = dg_expf(dlt);
+      sq += __float2ll_rz(__fmul_rn(ev[j], 1099511627776.0f));
+      uq += __float2ll_rz(__fmul_rn(__fmul_rn(ev[j], dlt), 1099511627776.0f));
     }
+    sl4[i] = make_float4(ev[0], ev[1], ev[2], ev[3]);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -614,25 +688,59 @@ __global__ void __launch_bounds__(512) k_sampler(SamplerArgs a, T* __restrict__ 
   if (threadIdx.x == 0) {
     long long S = 0, U = 0;
     for (int w = 0; w < nw; ++w) { S += red_s[w]; U += red_u[w]; }
+    part.s = S;
+    part.u = U;
+  }
+  cluster_sync_all();
+  long long S = 0, U = 0;
+  for (int r = 0; r < kSampCta; ++r) {
+    const SampPart* pr = cluster_peer(&part, r);
+    S += pr->s;
+    U += pr->u;
+  }
+  // no CTA may leave (or reuse `part`) while another still reads it
+  cluster_sync_all();
+  if (rank == 0 && threadIdx.x == 0) {
     const float sf = __ll2float_rn(S), uf = __ll2float_rn(U);
     a.H[row] = __fsub_rn(dg_logf(__fmul_rn(sf, 9.094947017729282e-13f)), __fdiv_rn(uf, sf));
     if (a.s_q) a.s_q[row] = S;
     if (a.u_q) a.u_q[row] = U;
-    sh_s = S;
   }
-  __syncthreads();
 
   // pass 3
   if (probs) {
-    const float inv_s = __fdiv_rn(1.0f, __fmul_rn(__ll2float_rn(sh_s), 9.094947017729282e-13f));
-    T* pr = probs + row * a.vocab;
-    for (int v4 = threadIdx.x; v4 < n4; v4 += blockDim.x) {
-      const float4 l = l4[v4];
-      const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) pr[v4 * 4 + j] = from_f<T>(__fmul_rn(dg_expf(__fsub_rn(lv[j], m)), inv_s));
+    const float inv_s = __fdiv_rn(1.0f, __fmul_rn(__ll2float_rn(S), 9.094947017729282e-13f));
+    T* pr = probs + row * a.vocab + (long long)g0 * 4;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      const float4 e = sl4[i];
+      store4<T>(pr + (long long)i * 4, __fmul_rn(e.x, inv_s), __fmul_rn(e.y, inv_s), __fmul_rn(e.z, inv_s),
+                __fmul_rn(e.w, inv_s));
     }
   }
+}
+
+// Launch of the sampler over `rows` rows (vocab % (4 kSampCta) == 0).
+template <typename T>
+cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cudaStream_t s, bool pdl) {
+  const size_t smem = (size_t)sa.vocab / kSampCta * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_sampler<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * kSampCta));
+  cfg.blockDim = dim3(kSampThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_sampler<T>, sa, probs);
 }
 
 // ---------------------------------------------------------------------------

@@ -33,7 +33,8 @@ dg_status dg_test_philox(const uint32_t* in, uint32_t* out, int64_t n, void* str
  * * positions + position; canvas = row / positions keys the Philox stream):
  * entropy H, Gumbel-max token at T = temp_end + (temp_start - temp_end) t,
  * argmax, exact fixed-point sums S_q/U_q (2^-40 units, may be NULL) and the
- * probabilities (bf16 if probs_bf16 else fp32; may be NULL). */
+ * probabilities (bf16 if probs_bf16 else fp32; may be NULL).  vocab must be
+ * a multiple of 32 (DG_ERR_INVALID_ARG otherwise). */
 dg_status dg_test_sampler(const float* logits, int32_t rows, int32_t vocab, int32_t positions, uint64_t seed,
                           int32_t step, float t, float temp_start, float temp_end, float* H, int32_t* tok,
                           int32_t* amax, int64_t* s_q, int64_t* u_q, void* probs, int32_t probs_bf16,
