@@ -7,14 +7,10 @@
 //                           (K for S = Q K^T, V^T for O = P V) are K-major
 // S = slot stride >= P + 256, positions 0..P-1 prompt, P..P+255 canvas.
 //
-// tcgen05 kernel: one CTA = 128 query rows (128/G tokens x the G query heads
-// sharing one KV head) x one split of the key range.  Warp 4 issues TMA
-// (Q once, K/V blocks of 128 keys double-buffered), warp 5 issues the MMAs,
-// warps 0-3 run the online softmax: thread = query row = TMEM lane.
-// S = Q K^T lives in TMEM columns [0,128), O in [128,256).  P is written as
-// bf16 into shared memory in the 128B-swizzled K-major layout the MMA reads.
-// Each split writes its normalised partial O and log2-sum-exp; a combine
-// kernel merges the splits in index order.
+// tcgen05 kernel: S = Q K^T and O live in TMEM, P is written as bf16 into
+// shared memory in the 128B-swizzled K-major layout the MMA reads.  Each
+// split of the key range writes its normalised partial O and log2-sum-exp;
+// a combine kernel merges the splits in index order.
 #pragma once
 #include "dg_device.cuh"
 
@@ -27,7 +23,7 @@ struct AttnArgs {
   int Hq, Hkv;
   int q_tiles;          // ceil(n_q * G / 128)
   int n_splits;
-  int blocks_per_split; // KV blocks of 128 keys per split
+  int blocks_per_split; // KV blocks of 64 keys per split
   int lbh0;             // (layer * B + b0) * Hkv: outer index of canvas b0's head 0
   int n_canvas;         // canvases in this launch
   float scale_log2;     // log2(e) / sqrt(hd)
@@ -36,8 +32,45 @@ struct AttnArgs {
   int* err;
 };
 
-constexpr int kAttnThreads = 192;
-constexpr int kAttnSmem = 32768 /*Q*/ + 2 * 65536 /*K,V x2*/ + 32768 /*P*/ + 1024;
+// One CTA = two query tiles (A and B, 128 rows each: 128/G tokens x the G
+// query heads of one KV head) x one split of the key range, so every K/V
+// block fetched serves 256 query rows.  320 threads:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B (thread = query
+//              row = TMEM lane; warp w reaches lanes 32 (w % 4) ..);
+//   warp 8     TMA: Q of both tiles once, then K / V^T blocks of 64 keys
+//              through a 3-stage ring;
+//   warp 9     MMA issuer.
+// TMEM (512 columns): S_A [0,64), S_B [64,128), O_A [128,256), O_B [256,384).
+// The issuer alternates tiles -- S_B(j) and PV_A(j-1) run on the tensor core
+// while tile A's softmax works on block j, and the other way round -- so the
+// two softmax groups and the MMAs overlap.
+constexpr int kAttnThreads = 320;
+constexpr int kAttnBK = 64;                                   // keys per block
+constexpr int kAttnStages = 3;
+constexpr int kAttnQBytes = 32768;                            // one Q tile
+constexpr int kAttnKVBytes = 2 * 8192 + 16384;                // K (2 chunks) + V^T of one block
+constexpr int kAttnPBytes = 16384;                            // one P tile
+constexpr int kAttnSmem = 2 * kAttnQBytes + kAttnStages * kAttnKVBytes + 2 * kAttnPBytes + 1024;
+
+// Grid of the tensor-core attention: q_tiles tiles of 128 query rows, paired
+// per CTA; key range split so that pairs x splits fills the SMs about once
+// (one CTA per SM), capped by the partial-output rows available.
+struct AttnPlan {
+  int q_tiles, n_splits, blocks_per_split, ctas;
+};
+inline AttnPlan attn_plan(long long n_q, int G, int Hkv, int n_canvas, int n_keys, long long rows,
+                          long long part_rows_cap) {
+  AttnPlan p;
+  p.q_tiles = (int)((n_q * G + 127) / 128);
+  const int nblocks = (n_keys + kAttnBK - 1) / kAttnBK;
+  const int base = (p.q_tiles + 1) / 2 * Hkv * n_canvas;
+  int splits = std::max(1, std::min(nblocks, kSMs / std::max(1, base)));
+  while (splits > 1 && (long long)splits * rows > part_rows_cap) --splits;
+  p.blocks_per_split = (nblocks + splits - 1) / splits;
+  p.n_splits = (nblocks + p.blocks_per_split - 1) / p.blocks_per_split;
+  p.ctas = base * p.n_splits;
+  return p;
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -45,185 +78,182 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;                 // 2 x [128 rows][128 B]
-  uint8_t* sKV = smem + 32768;        // stage s: K (2 x 16 KB) then V (2 x 16 KB)
-  uint8_t* sP = smem + 32768 + 2 * 65536;
-  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], s_full, p_full, o_done;
+  uint8_t* sQ = smem;                                   // tile t at t * 32 KB
+  uint8_t* sKV = smem + 2 * kAttnQBytes;                // stage s: K chunk 0, K chunk 1, V^T
+  uint8_t* sP = sKV + kAttnStages * kAttnKVBytes;       // tile t at t * 16 KB
+  __shared__ __align__(8) uint64_t q_full, kv_full[kAttnStages], kv_empty[kAttnStages];
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_done[2];
   __shared__ uint32_t tmem_base;
 
   int bid = blockIdx.x;
   const int split = bid % a.n_splits; bid /= a.n_splits;
-  const int qt = bid % a.q_tiles; bid /= a.q_tiles;
+  const int n_pairs = (a.q_tiles + 1) / 2;
+  const int qp = bid % n_pairs; bid /= n_pairs;
   const int g = bid % a.Hkv;
   const int bc = bid / a.Hkv;                   // canvas within the launch
   const int tok_per_tile = 128 / a.G;
-  const int tok0 = qt * tok_per_tile;
+  const int tok0 = 2 * qp * tok_per_tile;       // first token of tile A (tile B follows)
   const int lbh = a.lbh0 + bc * a.Hkv + g;
 
-  // key blocks of this split (causal: only blocks reaching the tile's last query)
-  const int n_blocks_all = (a.n_keys + 127) / 128;
-  int kb_begin = split * a.blocks_per_split;
+  // key blocks of this split (causal: only blocks reaching the pair's last query)
+  const int n_blocks_all = (a.n_keys + kAttnBK - 1) / kAttnBK;
+  const int kb_begin = split * a.blocks_per_split;
   int kb_end = min(n_blocks_all, kb_begin + a.blocks_per_split);
   if (a.causal) {
-    const int last_pos = a.q_pos0 + min(a.n_q, tok0 + tok_per_tile) - 1;
-    kb_end = min(kb_end, last_pos / 128 + 1);
+    const int last_pos = a.q_pos0 + min(a.n_q, tok0 + 2 * tok_per_tile) - 1;
+    kb_end = min(kb_end, last_pos / kAttnBK + 1);
   }
   const int nblk = max(0, kb_end - kb_begin);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < 2; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    mbar_init(&s_full, 1);
-    mbar_init(&p_full, 128);
-    mbar_init(&o_done, 1);
+    for (int s = 0; s < kAttnStages; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int t = 0; t < 2; ++t) { mbar_init(&s_full[t], 1); mbar_init(&p_full[t], 128); mbar_init(&o_done[t], 1); }
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_base, 256);
+  if (warp == 0) tmem_alloc(&tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t idesc = idesc_bf16(128, 128);
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && nblk > 0) {
-      mbar_expect_tx(&q_full, 32768);
-      const int zq = bc * a.n_q + tok0;
-      tma_load_3d(sQ, &tmQ, 0, g * a.G, zq, &q_full);
-      tma_load_3d(sQ + 16384, &tmQ, 64, g * a.G, zq, &q_full);
+      mbar_expect_tx(&q_full, 2 * kAttnQBytes);
+      for (int t = 0; t < 2; ++t) {
+        const int zq = bc * a.n_q + tok0 + t * tok_per_tile;
+        tma_load_3d(sQ + t * kAttnQBytes, &tmQ, 0, g * a.G, zq, &q_full);
+        tma_load_3d(sQ + t * kAttnQBytes + 16384, &tmQ, 64, g * a.G, zq, &q_full);
+      }
       for (int j = 0; j < nblk; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, a.err, DGDEV_TIMEOUT_TMA)) break;
-        uint8_t* kv = sKV + s * 65536;
-        const int key0 = (kb_begin + j) * 128;
-        mbar_expect_tx(&kv_full[s], 65536);
+        const int s = j % kAttnStages;
+        if (j >= kAttnStages &&
+            !mbar_wait(&kv_empty[s], ((j / kAttnStages) & 1) ^ 1, a.err, DGDEV_TIMEOUT_TMA))
+          break;
+        uint8_t* kv = sKV + s * kAttnKVBytes;
+        const int key0 = (kb_begin + j) * kAttnBK;
+        mbar_expect_tx(&kv_full[s], kAttnKVBytes);
         tma_load_3d(kv, &tmK, 0, key0, lbh, &kv_full[s]);
-        tma_load_3d(kv + 16384, &tmK, 64, key0, lbh, &kv_full[s]);
-        tma_load_3d(kv + 32768, &tmV, key0, 0, lbh, &kv_full[s]);
-        tma_load_3d(kv + 49152, &tmV, key0 + 64, 0, lbh, &kv_full[s]);
+        tma_load_3d(kv + 8192, &tmK, 64, key0, lbh, &kv_full[s]);
+        tma_load_3d(kv + 16384, &tmV, key0, 0, lbh, &kv_full[s]);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && nblk > 0) {
       bool ok = mbar_wait(&q_full, 0, a.err, DGDEV_TIMEOUT_MMA);
-      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+      const uint32_t idesc_s = idesc_bf16(128, kAttnBK), idesc_o = idesc_bf16(128, 128);
       for (int j = 0; j <= nblk && ok; ++j) {
-        if (j > 0) {
-          // O += P_{j-1} V_{j-1}
-          if (!mbar_wait(&p_full, (j - 1) & 1, a.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sKV + ((j - 1) & 1) * 65536 + 32768);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = sdesc_sw128(p_addr + (kk >> 2) * 16384) + 2 * (kk & 3);
-            const uint64_t bd = sdesc_sw128(v_addr + (kk >> 2) * 16384) + 2 * (kk & 3);
-            tc_mma_bf16(tO, ad, bd, idesc, (j > 1 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(&o_done);
-          tc_commit(&kv_empty[(j - 1) & 1]);
+        if (j < nblk && !mbar_wait(&kv_full[j % kAttnStages], (j / kAttnStages) & 1, a.err, DGDEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
         }
-        if (j < nblk) {
-          // S = Q K_j^T
-          if (!mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sKV + (j & 1) * 65536);
+        tc_fence_after();
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j > 0) {
+            // O_t += P_t(j-1) V(j-1)
+            if (!mbar_wait(&p_full[t], (j - 1) & 1, a.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t p_addr = smem_u32(sP + t * kAttnPBytes);
+            const uint32_t v_addr = smem_u32(sKV + ((j - 1) % kAttnStages) * kAttnKVBytes + 16384);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * 16384) + 2 * (kk & 3);
-            const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * 16384) + 2 * (kk & 3);
-            tc_mma_bf16(tS, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma_bf16(tmem + 128 + t * 128, sdesc_sw128(p_addr) + 2 * kk, sdesc_sw128(v_addr) + 2 * kk,
+                          idesc_o, (j > 1 || kk > 0) ? 1u : 0u);
+            tc_commit(&o_done[t]);
+            if (t == 1) tc_commit(&kv_empty[(j - 1) % kAttnStages]);
           }
-          tc_commit(&s_full);
+          if (j < nblk) {
+            // S_t = Q_t K(j)^T
+            const uint32_t q_addr = smem_u32(sQ + t * kAttnQBytes);
+            const uint32_t k_addr = smem_u32(sKV + (j % kAttnStages) * kAttnKVBytes);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc_mma_bf16(tmem + t * kAttnBK, sdesc_sw128(q_addr + (kk >> 2) * 16384) + 2 * (kk & 3),
+                          sdesc_sw128(k_addr + (kk >> 2) * 8192) + 2 * (kk & 3), idesc_s, kk > 0 ? 1u : 0u);
+            tc_commit(&s_full[t]);
+          }
         }
       }
     }
     __syncwarp();
   } else {
-    // ---------------- softmax warps 0-3: thread = query row ----------------
-    const int r = threadIdx.x;                      // TMEM lane / Q row
-    const int tok = tok0 + r / a.G;
+    // ---------------- softmax: warps 0-3 tile A, 4-7 tile B ----------------
+    const int t = warp >> 2;
+    const int r = threadIdx.x & 127;                // TMEM lane / Q row of the tile
+    const int tok = tok0 + t * tok_per_tile + r / a.G;
     const int head = g * a.G + r % a.G;
     const int qpos = a.q_pos0 + tok;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t * kAttnBK + lane_off, tO = tmem + 128 + t * 128 + lane_off;
+    uint8_t* rowp = sP + t * kAttnPBytes + r * 128;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
     // tcgen05.ld/st are warp-collective: every branch around them is kept
     // uniform across the warp (wait outcomes are agreed with __all_sync).
     for (int j = 0; j < nblk && ok; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full, j & 1, a.err, DGDEV_TIMEOUT_EPI))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, a.err, DGDEV_TIMEOUT_EPI))) { ok = false; break; }
       tc_fence_after();
-      const int key0 = (kb_begin + j) * 128;
-      // pass 1: block max (scaled to log2 units)
-      float mx = -INFINITY;
-      for (int c0 = 0; c0 < 128; c0 += 16) {
-        float v[16];
-        tmem_ld16(tS + lane_off + c0, v);
+      const int key0 = (kb_begin + j) * kAttnBK;
+      float v[kAttnBK];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int key = key0 + c0 + q;
-          const bool vis = key < a.n_keys && (!a.causal || key <= qpos);
-          if (vis) mx = fmaxf(mx, v[q] * a.scale_log2);
-        }
+      for (int c0 = 0; c0 < kAttnBK; c0 += 16) {
+        float w16[16];
+        tmem_ld16(tS + c0, w16);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[c0 + q] = w16[q];
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kAttnBK; ++c) {
+        const int key = key0 + c;
+        const bool vis = key < a.n_keys && (!a.causal || key <= qpos);
+        v[c] = vis ? v[c] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, v[c]);
       }
       const float m_new = fmaxf(m_run, mx);
-      // PV of the previous block must be done before P and O are touched
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done, (j - 1) & 1, a.err, DGDEV_TIMEOUT_EPI))) {
+      // PV of the previous block must be done before P_t and O_t are touched
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, a.err, DGDEV_TIMEOUT_EPI))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
-      // pass 2: P = exp2(s - m_new) as bf16 into the swizzled tile
       float lsum = 0.0f;
-      for (int c0 = 0; c0 < 128; c0 += 16) {
-        float v[16];
-        tmem_ld16(tS + lane_off + c0, v);
-        uint32_t pk[8];
 #pragma unroll
-        for (int q = 0; q < 16; q += 2) {
-          float p2[2];
+      for (int ch = 0; ch < kAttnBK / 8; ++ch) {
+        uint32_t pk[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = key0 + c0 + q + u;
-            const bool vis = key < a.n_keys && (!a.causal || key <= qpos);
-            const float pv = (vis && m_new != -INFINITY) ? exp2f(v[q + u] * a.scale_log2 - m_new) : 0.0f;
-            const bf16 pb = __float2bfloat16_rn(pv);
-            lsum += __bfloat162float(pb);
-            p2[u] = __bfloat162float(pb);
-          }
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(p2[0], p2[1]);
+        for (int q = 0; q < 8; q += 2) {
+          const float p0 = m_new != -INFINITY ? exp2f(v[ch * 8 + q] - m_new) : 0.0f;
+          const float p1 = m_new != -INFINITY ? exp2f(v[ch * 8 + q + 1] - m_new) : 0.0f;
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+          lsum += __low2float(pr) + __high2float(pr);
           pk[q / 2] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        // 16 keys = two 16-byte chunks of row r in column block c0/64
-        const int cb = c0 >> 6;
-        const int ch0 = (c0 & 63) >> 3;
-        uint8_t* rowp = sP + cb * 16384 + r * 128;
-        *reinterpret_cast<uint4*>(rowp + (((ch0) ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(rowp + (((ch0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       // rescale the running output (skipped only when no row of the warp needs it)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
         for (int c0 = 0; c0 < 128; c0 += 16) {
-          float v[16];
-          tmem_ld16(tO + lane_off + c0, v);
+          float o16[16];
+          tmem_ld16(tO + c0, o16);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) v[q] *= alpha;
-          tmem_st16(tO + lane_off + c0, v);
+          for (int q = 0; q < 16; ++q) o16[q] *= alpha;
+          tmem_st16(tO + c0, o16);
         }
       }
       l_run = l_run * alpha + lsum;
       m_run = m_new;
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full);
+      mbar_arrive(&p_full[t]);
     }
     // epilogue: normalised partial O and log2-sum-exp of this split
-    if (ok && nblk > 0) ok = __all_sync(0xffffffffu, mbar_wait(&o_done, (nblk - 1) & 1, a.err, DGDEV_TIMEOUT_EPI));
+    if (ok && nblk > 0) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (nblk - 1) & 1, a.err, DGDEV_TIMEOUT_EPI));
     tc_fence_after();
     // TMEM loads are warp-collective: every lane loads, only valid rows store.
     const bool row_valid = tok < a.n_q;
@@ -234,15 +264,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const bool have = loaded && l_run > 0.0f;
     const float inv_l = have ? 1.0f / l_run : 0.0f;
     for (int c0 = 0; c0 < 128; c0 += 16) {
-      float v[16];
+      float o16[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) v[q] = 0.0f;
-      if (loaded) tmem_ld16(tO + lane_off + c0, v);
+      for (int q = 0; q < 16; ++q) o16[q] = 0.0f;
+      if (loaded) tmem_ld16(tO + c0, o16);
       if (row_valid) {
 #pragma unroll
         for (int q = 0; q < 16; q += 4) {
-          const float4 o4 = have ? make_float4(v[q] * inv_l, v[q + 1] * inv_l, v[q + 2] * inv_l,
-                                               v[q + 3] * inv_l)
+          const float4 o4 = have ? make_float4(o16[q] * inv_l, o16[q + 1] * inv_l, o16[q + 2] * inv_l,
+                                               o16[q + 3] * inv_l)
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
           *reinterpret_cast<float4*>(op + c0 + q) = o4;
         }
@@ -252,7 +282,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------

@@ -457,8 +457,8 @@ struct AttnMaps {
 bool attn_maps(const dg_model* m, const KvGeom& g, int n_keys, int T_q, AttnMaps& am) {
   const uint64_t hd = m->hd, lbh = (uint64_t)m->L * g.B * m->hkv;
   bool ok = map3d(&am.q, m->q, hd, m->hq, T_q, hd * 2, (uint64_t)m->hq * hd * 2, 64, m->G, 128 / m->G);
-  ok &= map3d(&am.k, g.K, hd, n_keys, lbh, hd * 2, (uint64_t)g.S * hd * 2, 64, 128, 1);
-  ok &= map3d(&am.v, g.Vt, n_keys, hd, lbh, (uint64_t)g.S * 2, (uint64_t)hd * g.S * 2, 64, 128, 1);
+  ok &= map3d(&am.k, g.K, hd, n_keys, lbh, hd * 2, (uint64_t)g.S * hd * 2, 64, kAttnBK, 1);
+  ok &= map3d(&am.v, g.Vt, n_keys, hd, lbh, (uint64_t)g.S * 2, (uint64_t)hd * g.S * 2, kAttnBK, 128, 1);
   return ok;
 }
 
@@ -515,19 +515,14 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     {
       LaunchScope ls(m, s, PH_ATTN);
       if (m->bf) {
-        aa.q_tiles = cdiv((long long)n_per * m->G, 128);
-        const int nblocks = cdiv(n_keys, 128);
-        const int base = aa.q_tiles * m->hkv * n_canvas;
-        int splits = std::max(1, std::min(nblocks, cdiv(2 * kSMs, base)));
-        while (splits > 1 && (size_t)splits * rows > m->part_rows_cap) --splits;
-        aa.blocks_per_split = cdiv(nblocks, splits);
-        aa.n_splits = cdiv(nblocks, aa.blocks_per_split);
+        const AttnPlan ap = attn_plan(n_per, m->G, m->hkv, n_canvas, n_keys, rows, (long long)m->part_rows_cap);
+        aa.q_tiles = ap.q_tiles; aa.n_splits = ap.n_splits; aa.blocks_per_split = ap.blocks_per_split;
         static bool attr = false;
         if (!attr) {
           CU_TRY(cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem));
           attr = true;
         }
-        launch_pdl(k_attn_tc, base * aa.n_splits, kAttnThreads, kAttnSmem, s, am.q, am.k, am.v, aa);
+        launch_pdl(k_attn_tc, ap.ctas, kAttnThreads, kAttnSmem, s, am.q, am.k, am.v, aa);
       } else {
         aa.q_tiles = 1; aa.n_splits = 1; aa.blocks_per_split = 1;
         const long long threads = rows * 32;

@@ -179,17 +179,29 @@ __global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const f
   float ss = 0.0f;
   for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const float* yp = y + rows[j] + i;
-      float4 v = *reinterpret_cast<const float4*>(yp);
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      // issue the loads of up to 8 slots before accumulating them in order
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j0 + j < k) v[j] = *reinterpret_cast<const float4*>(y + rows[j0 + j] + i);
       for (int s = 1; s < ns; ++s) {
-        const float4 v2 = *reinterpret_cast<const float4*>(yp + s * split_stride);
-        v.x += v2.x; v.y += v2.y; v.z += v2.z; v.w += v2.w;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j0 + j < k) {
+            const float4 v2 = *reinterpret_cast<const float4*>(y + rows[j0 + j] + i + s * split_stride);
+            v[j].x += v2.x; v[j].y += v2.y; v[j].z += v2.z; v[j].w += v2.w;
+          }
       }
-      acc[0] = fmaf(gw[j], v.x, acc[0]);
-      acc[1] = fmaf(gw[j], v.y, acc[1]);
-      acc[2] = fmaf(gw[j], v.z, acc[2]);
-      acc[3] = fmaf(gw[j], v.w, acc[3]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j0 + j < k) {
+          const float g = gw[j0 + j];
+          acc[0] = fmaf(g, v[j].x, acc[0]);
+          acc[1] = fmaf(g, v[j].y, acc[1]);
+          acc[2] = fmaf(g, v[j].z, acc[2]);
+          acc[3] = fmaf(g, v[j].w, acc[3]);
+        }
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
