@@ -75,7 +75,7 @@ inline AttnPlan attn_plan(long long n_q, int G, int Hkv, int n_canvas, int n_key
 __global__ void __launch_bounds__(kAttnThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
-  pdl_enter();
+  pdl_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                                   // tile t at t * 32 KB
@@ -113,6 +113,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&tmem_base, 512);
+  pdl_wait();   // q and the cache are written by the previous kernels
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

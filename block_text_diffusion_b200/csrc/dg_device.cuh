@@ -25,11 +25,19 @@ __device__ __forceinline__ void dev_error(int* err, int code) {
 
 // Programmatic dependent launch: every kernel of the step lets the next
 // kernel in the stream be scheduled at once, and waits for the previous
-// kernel (and its memory) before it touches global memory.  Without the
-// launch attribute both are no-ops.
-__device__ __forceinline__ void pdl_enter() {
+// kernel (and its memory) before it touches global memory the previous
+// kernels write.  Kernels with a prologue (barriers, tensor memory, weight
+// tiles, which no kernel of the step writes) run it before the wait.
+// Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  pdl_launch();
+  pdl_wait();
 }
 
 // ---------------------------------------------------------------------------

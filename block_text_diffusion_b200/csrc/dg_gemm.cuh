@@ -29,7 +29,6 @@ struct GemmArgs {
   int a_group_rows;        // grouped: A rows per group (a_row0 = group * a_group_rows)
   const int* work_count;
   const int* k_splits_dev; // persistent kernel: split-K factor chosen on the device (overrides k_splits)
-  const int* skip;         // optional device flag: nonzero -> every CTA returns at once
   int* err;
 };
 
@@ -83,10 +82,16 @@ __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           GemmArgs p) {
   using C = GemmTcCfg<BN, STAGES>;
-  pdl_enter();
-  if (p.skip && *p.skip) return;
+  pdl_launch();
+  // grouped work items come from the permute kernel: decode after the wait;
+  // dense tiles are pure index arithmetic and prefetch weight tiles first
+  const bool grouped = p.work != nullptr;
+  if (grouped) pdl_wait();
   GemmTile t;
-  if (!gemm_decode(p, t)) return;
+  if (!gemm_decode(p, t)) {
+    if (!grouped) pdl_wait();
+    return;
+  }
   int kb0, kb1;
   split_range(p, t.split, kb0, kb1);
   const int nkb = kb1 - kb0;
@@ -115,9 +120,19 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   const uint32_t tmem = tmem_base;
   const int m0 = t.m_tile * 128;
 
+  const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
+  // dense: the first ring slots' weight tiles are fetched before the wait
+  const int n_pre = grouped ? 0 : min(STAGES, nkb);
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < n_pre; ++i) {
+      mbar_expect_tx(&full_bar[i], tx);
+      tma_load_2d(smem + i * C::kStage, &tmA, (kb0 + i) * 64, t.a_row0 + m0, &full_bar[i]);
+    }
+  }
+  if (!grouped) pdl_wait();
+
   if (warp == 0) {
     if (lane == 0) {
-      const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
@@ -128,8 +143,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         uint8_t* a_s = smem + s * C::kStage;
         uint8_t* b_s = a_s + C::kABytes;
         const int kx = (kb0 + i) * 64;
-        mbar_expect_tx(&full_bar[s], tx);
-        tma_load_2d(a_s, &tmA, kx, t.a_row0 + m0, &full_bar[s]);
+        if (i >= n_pre) {
+          mbar_expect_tx(&full_bar[s], tx);
+          tma_load_2d(a_s, &tmA, kx, t.a_row0 + m0, &full_bar[s]);
+        }
         for (int j = 0; j < n_boxes; ++j)
           tma_load_2d(b_s + j * kBoxRowsB * 128, &tmB, kx, t.b_row0 + j * kBoxRowsB, &full_bar[s]);
       }
@@ -195,10 +212,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 // Warps: 0 = TMA producer, 1 = MMA issuer, 2..5 = epilogue (warp w drains
 // TMEM lanes 32*(w%4)..+31).  192 threads.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int gemm_total_tiles(const GemmArgs& p, int items_dense) {
-  const int items = p.work ? *p.work_count : items_dense;
-  return p.m_tiles * p.k_splits * items;
-}
+constexpr int kWorkSmem = 512;   // work items staged in shared memory (more are read from global)
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
@@ -207,17 +221,13 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   using C = GemmTcCfg<BN, STAGES>;
   constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
   constexpr int kAllocCols = 2 * kAccCols;             // two buffers (<= 512)
-  pdl_enter();
-  if (p_in.skip && *p_in.skip) return;
+  pdl_launch();
   GemmArgs p = p_in;
-  if (p.k_splits_dev) p.k_splits = max(1, min(*p.k_splits_dev, p.kb_total));
-  const int total = gemm_total_tiles(p, items_dense);
-  if ((int)blockIdx.x >= total) return;
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_base;
+  __shared__ int4 s_work[kWorkSmem];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
@@ -227,6 +237,16 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
     prefetch_tmap(&tmB);
   }
   if (warp == 0) tmem_alloc(&tmem_base, kAllocCols);
+  // the split factor and the work list are written by the permute kernel
+  pdl_wait();
+  if (p.k_splits_dev) p.k_splits = max(1, min(*p.k_splits_dev, p.kb_total));
+  const int n_items = p.work ? *p.work_count : items_dense;
+  const int total = p.m_tiles * p.k_splits * n_items;
+  // work items are read by all three roles once per tile: stage them on chip
+  const bool work_smem = p.work != nullptr && n_items <= kWorkSmem;
+  if (work_smem)
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) s_work[i] = p.work[i];
+  const int4* work = work_smem ? s_work : p.work;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -244,7 +264,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         t.split = r % p.k_splits;
         const int item = r / p.k_splits;
         if (p.work) {
-          const int4 w = p.work[item];
+          const int4 w = work[item];
           t.a_row0 = w.x * p.a_group_rows; t.b_row0 = w.y; t.n_valid = w.z;
         } else {
           t.a_row0 = 0; t.b_row0 = item * p.n_tile; t.n_valid = min(p.n_tile, p.N - t.b_row0);
@@ -276,7 +296,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int r = tile / p.m_tiles;
         const int split = r % p.k_splits;
         const int item = r / p.k_splits;
-        const int n_valid = p.work ? p.work[item].z : min(p.n_tile, p.N - item * p.n_tile);
+        const int n_valid = p.work ? work[item].z : min(p.n_tile, p.N - item * p.n_tile);
         (void)m_t;
         int kb0, kb1;
         split_range(p, split, kb0, kb1);
@@ -317,7 +337,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const int split = r % p.k_splits;
       const int item = r / p.k_splits;
       int n_valid, out_row0;
-      if (p.work) { const int4 w = p.work[item]; n_valid = w.z; out_row0 = w.w; }
+      if (p.work) { const int4 w = work[item]; n_valid = w.z; out_row0 = w.w; }
       else { out_row0 = item * p.n_tile; n_valid = min(p.n_tile, p.N - out_row0); }
       int kb0, kb1;
       split_range(p, split, kb0, kb1);
@@ -360,7 +380,6 @@ static __global__ void __launch_bounds__(256)
 k_gemm_f32(const float* __restrict__ A, long long lda, const float* __restrict__ B, long long ldb,
            int K, GemmArgs p) {
   pdl_enter();
-  if (p.skip && *p.skip) return;
   GemmTile t;
   if (!gemm_decode(p, t)) return;
   int kb0, kb1;

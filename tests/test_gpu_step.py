@@ -187,6 +187,11 @@ def oracle_pair(w, K, V, canvas, canvas_id=0):
     return r, trace, rn, trace_n
 
 
+def as_path_outputs(r):
+    """An oracle round's outputs under the CUDA path's names."""
+    return dict(logits=r["logits64"], entropy=r["H"], tokens=r["tokens"], selfcond_next=r["selfcond_next"])
+
+
 def deviation(x_a, x_b, g_a, g_b, stable):
     """Deviation of one round from another on the routing-stable tokens:
     final normalised state in bf16 steps at unit scale, logits, entropy,
@@ -244,7 +249,7 @@ def compare_bf16_round(g, r, trace, om_model, w, gx_final, rn, trace_n, min_stab
     lm_err = np.abs(g["logits"] - lm).max()
     assert lm_err <= 2e-2, lm_err
     dg_ = deviation(gx_final, xo, g, r, stable)
-    dn = deviation(xn, xo, rn, r, stable)
+    dn = deviation(xn, xo, as_path_outputs(rn), r, stable)
     print(f"stable {stable.mean():.3f}; LM head err {lm_err:.2e}; path vs oracle {dg_}; noise envelope {dn}")
     within_envelope(dg_, dn, SLACK)
     dl = np.abs(g["logits"] - r["logits64"]).max(axis=1)
