@@ -234,12 +234,13 @@ def test_commit(H, tok, amax, prev_amax, vocab, seed, step, max_steps, commit_mo
                                 _ptr(canvas_next), _ptr(stop), _ptr(n_committed), _stream(stream)), "dg_test_commit")
 
 
-def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, persistent=False, stream=None):
+def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, persistent=False, m256=False, stream=None):
     import torch
     M, K = A.shape
     N = B.shape[0]
+    flags = int(persistent) | (2 if m256 else 0)
     _check(lib().dg_test_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, 1 if A.dtype == torch.bfloat16 else 0,
-                              float(alpha), k_splits, bn, int(persistent), _stream(stream)), "dg_test_gemm")
+                              float(alpha), k_splits, bn, flags, _stream(stream)), "dg_test_gemm")
 
 
 def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, stream=None):

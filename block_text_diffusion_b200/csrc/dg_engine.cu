@@ -244,21 +244,22 @@ struct GemmCall {
   int bn = 256;
   bool persistent = false;           // walk tiles with one CTA per SM slot
   const int* k_splits_dev = nullptr; // persistent: split-K count decided on the device (<= splits)
+  bool m256 = false;                 // dense, bn 256: 256-row M tiles (two accumulators share B)
 };
 
-template <int BN, int ST>
+template <int BN, int ST, int MT = 1>
 dg_status launch_tc(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
-  using C = GemmTcCfg<BN, ST>;
+  using C = GemmTcCfg<BN, ST, MT>;
   static bool attr = false;
   if (!attr) {
-    CU_TRY(cudaFuncSetAttribute(k_gemm_tc<BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
+    CU_TRY(cudaFuncSetAttribute(k_gemm_tc<BN, ST, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
     attr = true;
   }
   const int items = g.work ? g.max_items : cdiv(g.N, a.n_tile);
   const long long grid = (long long)a.m_tiles * a.k_splits * items;
   if (grid <= 0) return DG_OK;
   if (grid > 0x7FFFFFFFLL) return DG_ERR_UNSUPPORTED;
-  launch_pdl(k_gemm_tc<BN, ST>, (unsigned)grid, 128, C::kSmem, s, *g.tA, *g.tB, a);
+  launch_pdl(k_gemm_tc<BN, ST, MT>, (unsigned)grid, 128, C::kSmem, s, *g.tA, *g.tB, a);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -319,6 +320,10 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
       case 32: return launch_tc_persistent<32, 8>(g, a, s);
       default: return DG_ERR_UNSUPPORTED;
     }
+  }
+  if (g.m256 && g.bn == 256 && !g.work) {
+    a.m_tiles = cdiv(g.M, 256);
+    return launch_tc<256, 3, 2>(g, a, s);
   }
   switch (g.bn) {
     case 256: return launch_tc<256, 4>(g, a, s);
@@ -653,6 +658,7 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
   lc.tA = &m->tm_E; lc.tB = &m->tm_x; lc.A32 = (const float*)m->emb; lc.B32 = (const float*)m->x;
   lc.lda = d; lc.ldb = d; lc.M = V; lc.K = d; lc.N = Tn; lc.alpha = m->c.logit_scale;
   lc.out = io.logits; lc.ldo = V; lc.bn = dense_bn(Tn); lc.splits = 1;
+  lc.m256 = cdiv(V, 256) >= kSMs;   // many 256-row tiles: share each x tile between two accumulators
   DG_TRY(gemm(m, lc, PH_LM_HEAD, s));
   // vocab sampler
   {
@@ -691,6 +697,10 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
       const int mt = m->bf ? cdiv(d, 128) : cdiv(d, 64);
       const int items = m->bf ? cdiv(Tn, sc.bn) : cdiv(Tn, 64);
       sc.splits = pick_splits(mt, items, cdiv(V, 64), 16);
+      // wide model, one canvas tile: 256-row tiles share each probability tile
+      // between two accumulators, with splits filling the SMs once
+      sc.m256 = m->bf && sc.bn == 256 && items == 1 && d >= 2048;
+      if (sc.m256) sc.splits = std::max(1, std::min(16, kSMs / cdiv(d, 256)));
       while (sc.splits > 1 && (size_t)sc.splits * Tn * d > m->ws_elems) --sc.splits;
       sc.split_stride = (long long)Tn * d;
     }

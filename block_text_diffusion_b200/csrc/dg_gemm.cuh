@@ -64,24 +64,27 @@ __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& k
 // tcgen05 GEMM, bf16 in / fp32 out.  128 threads: warp 0 lane 0 issues TMA,
 // warp 1 lane 0 issues MMAs, then all four warps drain TMEM (warp w owns
 // accumulator rows 32w..32w+31).  A tiles 128 x 64, B tiles BN x 64 loaded
-// 32 rows per TMA box; STAGES-deep mbarrier ring.
+// 32 rows per TMA box; STAGES-deep mbarrier ring.  MT = 2 gives a CTA two
+// 128-row accumulators that share every B tile (M tile 256): for the big
+// vocabulary GEMMs this halves how often the activations stream from L2.
 // ---------------------------------------------------------------------------
 constexpr int kBoxRowsB = 32;
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MT = 1>
 struct GemmTcCfg {
-  static constexpr int kABytes = 128 * 128;          // 128 rows x 64 bf16
+  static constexpr int kABytes = MT * 128 * 128;     // MT x (128 rows x 64 bf16)
   static constexpr int kBBytes = BN * 128;           // BN rows x 64 bf16
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kTmemCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int kSmem = STAGES * kStage + 1024;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MT = 1>
 __global__ void __launch_bounds__(128, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           GemmArgs p) {
-  using C = GemmTcCfg<BN, STAGES>;
+  using C = GemmTcCfg<BN, STAGES, MT>;
+  static_assert(MT * C::kTmemCols <= 512, "tensor memory holds 512 columns");
   pdl_launch();
   // grouped work items come from the permute kernel: decode after the wait;
   // dense tiles are pure index arithmetic and prefetch weight tiles first
@@ -113,12 +116,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 0) tmem_alloc(&tmem_base, C::kTmemCols);
+  if (warp == 0) tmem_alloc(&tmem_base, MT * C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const int m0 = t.m_tile * 128;
+  const int m0 = t.m_tile * 128 * MT;
 
   const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
   // dense: the first ring slots' weight tiles are fetched before the wait
@@ -126,7 +129,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < n_pre; ++i) {
       mbar_expect_tx(&full_bar[i], tx);
-      tma_load_2d(smem + i * C::kStage, &tmA, (kb0 + i) * 64, t.a_row0 + m0, &full_bar[i]);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+        tma_load_2d(smem + i * C::kStage + mt * 16384, &tmA, (kb0 + i) * 64, t.a_row0 + m0 + mt * 128,
+                    &full_bar[i]);
     }
   }
   if (!grouped) pdl_wait();
@@ -145,7 +151,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         const int kx = (kb0 + i) * 64;
         if (i >= n_pre) {
           mbar_expect_tx(&full_bar[s], tx);
-          tma_load_2d(a_s, &tmA, kx, t.a_row0 + m0, &full_bar[s]);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+            tma_load_2d(a_s + mt * 16384, &tmA, kx, t.a_row0 + m0 + mt * 128, &full_bar[s]);
         }
         for (int j = 0; j < n_boxes; ++j)
           tma_load_2d(b_s + j * kBoxRowsB * 128, &tmB, kx, t.b_row0 + j * kBoxRowsB, &full_bar[s]);
@@ -163,10 +171,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + s * C::kStage);
         const uint32_t b_addr = a_addr + C::kABytes;
-        const uint64_t ad = sdesc_sw128(a_addr), bd = sdesc_sw128(b_addr);
+        const uint64_t bd = sdesc_sw128(b_addr);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_bf16(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (i | kk) != 0);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+            tc_mma_bf16(tmem + mt * C::kTmemCols, sdesc_sw128(a_addr + mt * 16384) + 2 * kk, bd + 2 * kk, idesc,
+                        (i | kk) != 0);
         tc_commit(&empty_bar[s]);
       }
       // Completes when every MMA above has finished (also on the abort path).
@@ -179,29 +190,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   // tcgen05.ld is warp-collective: agree on the wait outcome across the warp.
   const bool ok = __all_sync(0xffffffffu, mbar_wait(&done_bar, 0, p.err, DGDEV_TIMEOUT_EPI));
   tc_fence_after();
-  if (ok && nkb > 0) {
-    const int row = warp * 32 + lane;
+  for (int mt = 0; mt < MT; ++mt) {
+    const int row = mt * 128 + warp * 32 + lane;
     const bool m_ok = (m0 + row) < p.M;
     float* outp = p.out + (long long)t.split * p.split_stride + (long long)t.out_row0 * p.ldo + m0 + row;
-    for (int c0 = 0; c0 < n_mma; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, v);
-      if (m_ok) {
+    if (ok && nkb > 0) {
+      for (int c0 = 0; c0 < n_mma; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + mt * C::kTmemCols + ((uint32_t)(warp * 32) << 16) + c0, v);
+        if (m_ok) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (c0 + j < t.n_valid) outp[(long long)(c0 + j) * p.ldo] = v[j] * p.alpha;
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < t.n_valid) outp[(long long)(c0 + j) * p.ldo] = v[j] * p.alpha;
+        }
       }
-    }
-  } else if (nkb == 0 && ok) {
-    const int row = warp * 32 + lane;
-    if ((m0 + row) < p.M) {
-      float* outp = p.out + (long long)t.split * p.split_stride + (long long)t.out_row0 * p.ldo + m0 + row;
+    } else if (nkb == 0 && ok && m_ok) {
       for (int n = 0; n < t.n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, MT * C::kTmemCols);
 }
 
 // ---------------------------------------------------------------------------

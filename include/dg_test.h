@@ -51,7 +51,8 @@ dg_status dg_test_commit(const float* H, const int32_t* tok, const int32_t* amax
  * (A [M,K], B [N,K] row-major, bf16 through tcgen05 when bf16 != 0, else
  * fp32 SIMT); out holds k_splits partial slabs of N*M floats; bn in
  * {32,64,128,256} is the token tile (bf16 only); flags bit 0 selects the
- * persistent tile-walking kernel.  Allocates (a 32-byte error word). */
+ * persistent tile-walking kernel, bit 1 (bn 256, not persistent) 256-row
+ * tiles with two accumulators.  Allocates (a 32-byte error word). */
 dg_status dg_test_gemm(const void* A, const void* B, float* out, int32_t M, int32_t N, int32_t K, int32_t bf16,
                        float alpha, int32_t k_splits, int32_t bn, int32_t flags, void* stream);
 

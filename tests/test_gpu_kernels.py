@@ -220,6 +220,21 @@ def test_gemm_bf16(M, N, K, bn, splits, persistent):
     assert np.all(err <= 2e-6 * 0.5 * _bound(B, A) + 1e-30), err.max()
 
 
+@pytest.mark.parametrize("M,N,K,splits", [
+    (256, 256, 512, 1), (300, 200, 200, 1), (785, 256, 1024, 3), (4096, 256, 2816, 4), (2000, 33, 4096, 16)])
+def test_gemm_bf16_256_row_tiles(M, N, K, splits):
+    # two accumulators per CTA sharing each B tile (the vocabulary GEMMs);
+    # ragged M (a tile whose second half is partly or wholly outside M)
+    g = np.random.default_rng(M * 7 + N + K)
+    A = I._bf16_grid(g.standard_normal((M, K)).astype(F32))
+    B = I._bf16_grid(g.standard_normal((N, K)).astype(F32))
+    out = torch.zeros((splits, N, M), dtype=torch.float32, device="cuda")
+    dg.test_gemm(bf16_tensor(A), bf16_tensor(B), out, alpha=0.5, k_splits=splits, bn=256, m256=True)
+    got = host(out).astype(np.float64).sum(axis=0)
+    ref = 0.5 * (B.astype(np.float64) @ A.astype(np.float64).T)
+    assert np.all(np.abs(got - ref) <= 2e-6 * 0.5 * _bound(B, A) + 1e-30), np.abs(got - ref).max()
+
+
 def test_gemm_f32():
     g = np.random.default_rng(5)
     M, N, K = 1000, 256, 300
