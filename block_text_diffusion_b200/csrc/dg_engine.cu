@@ -364,7 +364,8 @@ bool config_ok(const dg_config& c) {
   if (c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 || c.top_k > c.n_experts || c.top_k > 64)
     return false;
   if (c.d_ff < 64 || c.d_ff % 64) return false;
-  if (c.vocab < 64 || c.vocab % 64) return false;
+  // the sampler keeps a vocab / 8 slice of fp32 logits in one CTA's shared memory
+  if (c.vocab < 64 || c.vocab % 64 || c.vocab > 458752) return false;
   if (c.max_canvases < 1 || c.max_canvases > 4096 || c.max_prompt < 1 || c.max_prompt > (1 << 20)) return false;
   if (c.max_steps < 1) return false;
   if (c.commit_mode != DG_COMMIT_THRESH && c.commit_mode != DG_COMMIT_EB) return false;

@@ -735,12 +735,11 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
 template <typename T>
 cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cudaStream_t s, bool pdl) {
   const size_t smem = (size_t)sa.vocab / kSampCta * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_sampler<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  static size_t attr_bytes = 0;   // dynamic shared memory the kernel is currently allowed
+  if (smem > attr_bytes) {
+    const cudaError_t e = cudaFuncSetAttribute(k_sampler<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr_bytes = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * kSampCta));
