@@ -40,7 +40,33 @@ def parse():
     ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--max-rounds", type=int, default=None,
                     help="override the round budget (short runs for profiler launch lists)")
+    ap.add_argument("--no-fast-converging", action="store_true",
+                    help="skip the committed-tokens measurement on the fast-converging workload")
     return ap.parse_args()
+
+
+def measured_traffic(algorithmic_bytes):
+    """DRAM bytes per launch of the expert gate|up GEMM from the committed ncu
+    summary (captured on the mid workload and scaled by its measured ratio of
+    DRAM bytes to algorithmic bytes); None when the GEMM source changed since
+    the capture."""
+    import hashlib
+    src = os.path.join(ROOT, "block_text_diffusion_b200", "csrc", "dg_gemm.cuh")
+    summ = os.path.join(ROOT, "profiles", "expert_gemm_mid_ncu.md")
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        fields = {}
+        with open(summ) as f:
+            for line in f:
+                if line.startswith("- ") and ": " in line:
+                    k, v = line[2:].split(": ", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("dg_gemm.cuh sha256") != sha:
+            return None
+        return algorithmic_bytes * float(fields["DRAM bytes / algorithmic bytes"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def peaks():
@@ -232,6 +258,12 @@ def run_ours(a):
     # distinct experts each layer streamed in the profiled round (measured routing)
     touched = model.touched_experts()
 
+    # committed tokens on the fast-converging workload (logit scale 16), where
+    # random-init weights still commit: single-GPU runs only
+    fast = None
+    if world == 1 and not a.no_fast_converging:
+        fast = fast_converging(dg, I, torch)
+
     (ms, e2e_ms), (n_rounds, n_com, e_rounds) = reduce_over_ranks(
         [ms, e2e_ms], [n_rounds, n_com, e_rounds], world, "cuda")
     if world > 1:
@@ -273,17 +305,50 @@ def run_ours(a):
                           "roof_ms": step_roof_ms, "frac": step_roof_ms / per_round_ms,
                           "bytes": b_round, "flops": f_round, "touched_experts": touched},
         "roofline": {"bound": "hbm", "kernel": "expert_gate_up_gemm", "achieved": achieved, "peak": hbm,
-                     "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / hbm, "traffic": measured_traffic(gu_bytes),
                      "peak_source": src, "avg_launch_ms": gu_avg, "algorithmic_bytes": gu_bytes},
         "phases_ms_per_round": {k: v[0] / a.profile_reps for k, v in prof.items() if v[1]},
         "e2e": {"value": e_rounds / (e2e_ms * 1e-3), "unit": "denoise steps/s",
                 "h2d_bytes_per_step": B * P * 4 * world, "d2h_bytes_per_step": (B * 256 + 2 * B) * 4 * world,
                 "includes": "prompt H2D, causal prompt encode, block loop, result D2H"},
+        "fast_converging": fast,
         "gpu_launches": int(n_rounds / world * (kper + 1) + a.steps * (1 + 3)) * world,
         "clocks": clk.summary(),
     }
     model.close()
     return line
+
+
+def fast_converging(dg, I, torch, blocks=3):
+    """Committed canvas tokens per second of full blocks on the long-context
+    workload (32768-token prompt, logit scale 16), timed with device events."""
+    w = I.LONG_CTX
+    P = w.prompt_len
+    model = dg.Model(w, max_canvases=1, max_prompt=P)
+    stream = torch.cuda.current_stream()
+    kv = model.new_kv(1, P)
+    model.encode_prompt(torch.from_numpy(I.prompt_ids(w.sample_seed, 1, P, w.vocab)).cuda(), kv)
+    canvas = torch.zeros((1, 256), dtype=torch.int32, device="cuda")
+    steps = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ncom = torch.zeros(1, dtype=torch.int32, device="cuda")
+    model.generate_block(kv, 1, P, canvas, steps, ncom)
+    torch.cuda.synchronize()
+    rounds = torch.zeros((), dtype=torch.int64, device="cuda")
+    committed = torch.zeros((), dtype=torch.int64, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(blocks):
+        model.generate_block(kv, 1, P, canvas, steps, ncom)
+        rounds += steps.sum()
+        committed += ncom.sum()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    model.sync_status()
+    ms = e0.elapsed_time(e1)
+    model.close()
+    n_r, n_c = int(rounds.item()), int(committed.item())
+    return {"workload": w.name, "prompt_len": P, "blocks": blocks, "committed_tokens_per_s": n_c / (ms * 1e-3),
+            "committed_per_block": n_c / blocks, "rounds_per_block": n_r / blocks, "ms_per_block": ms / blocks}
 
 
 # --- CPU oracle (bounded sample) ---------------------------------------------------------

@@ -200,22 +200,40 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       tc_fence_after();
       const int key0 = (kb_begin + j) * kAttnBK;
       float v[kAttnBK];
+      {
+        uint32_t w[kAttnBK / 16][16];
 #pragma unroll
-      for (int c0 = 0; c0 < kAttnBK; c0 += 16) {
-        float w16[16];
-        tmem_ld16(tS + c0, w16);
+        for (int q = 0; q < kAttnBK / 16; ++q) tmem_ld16_nw(tS + q * 16, w[q]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) v[c0 + q] = w16[q];
+        for (int q = 0; q < kAttnBK / 16; ++q)
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[q * 16 + u] = __uint_as_float(w[q][u]);
       }
-      float mx = -INFINITY;
+      // scale to log2 units; keys past the end (or after the query, causal) get -inf
+      if (!a.causal && key0 + kAttnBK <= a.n_keys) {
 #pragma unroll
-      for (int c = 0; c < kAttnBK; ++c) {
-        const int key = key0 + c;
-        const bool vis = key < a.n_keys && (!a.causal || key <= qpos);
-        v[c] = vis ? v[c] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, v[c]);
+        for (int c = 0; c < kAttnBK; ++c) v[c] *= a.scale_log2;
+      } else {
+#pragma unroll
+        for (int c = 0; c < kAttnBK; ++c) {
+          const int key = key0 + c;
+          const bool vis = key < a.n_keys && (!a.causal || key <= qpos);
+          v[c] = vis ? v[c] * a.scale_log2 : -INFINITY;
+        }
       }
-      const float m_new = fmaxf(m_run, mx);
+      float mt[kAttnBK / 2];
+#pragma unroll
+      for (int c = 0; c < kAttnBK / 2; ++c) mt[c] = fmaxf(v[2 * c], v[2 * c + 1]);
+#pragma unroll
+      for (int w2 = kAttnBK / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int c = 0; c < w2; ++c) mt[c] = fmaxf(mt[c], mt[c + w2]);
+      const float mx = mt[0];
+      // The running reference max moves only when the block max exceeds it by
+      // more than 8 (a factor 256 in P), so O is rarely rescaled; the final
+      // normalisation uses the same reference, so the result is unchanged.
+      const float m_new = (m_run == -INFINITY || mx > m_run + 8.0f) ? mx : m_run;
       // PV of the previous block must be done before P_t and O_t are touched
       if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done[t], (j - 1) & 1, a.err, DGDEV_TIMEOUT_EPI))) {
         ok = false;
@@ -223,28 +241,42 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       }
       tc_fence_after();
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
-      float lsum = 0.0f;
+      float ls[kAttnBK / 8];
 #pragma unroll
       for (int ch = 0; ch < kAttnBK / 8; ++ch) {
         uint32_t pk[4];
+        float acc = 0.0f;
 #pragma unroll
         for (int q = 0; q < 8; q += 2) {
           const float p0 = m_new != -INFINITY ? exp2f(v[ch * 8 + q] - m_new) : 0.0f;
           const float p1 = m_new != -INFINITY ? exp2f(v[ch * 8 + q + 1] - m_new) : 0.0f;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-          lsum += __low2float(pr) + __high2float(pr);
+          acc += __low2float(pr) + __high2float(pr);
           pk[q / 2] = *reinterpret_cast<const uint32_t*>(&pr);
         }
+        ls[ch] = acc;
         *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+#pragma unroll
+      for (int w2 = kAttnBK / 16; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int c = 0; c < w2; ++c) ls[c] += ls[c + w2];
+      const float lsum = ls[0];
       // rescale the running output (skipped only when no row of the warp needs it)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-          float o16[16];
-          tmem_ld16(tO + c0, o16);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) o16[q] *= alpha;
-          tmem_st16(tO + c0, o16);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld16_nw(tO + half * 64 + q * 16, o[q]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 16; ++u) o[q][u] = __float_as_uint(__uint_as_float(o[q][u]) * alpha);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_st16_nw(tO + half * 64 + q * 16, o[q]);
+          tmem_wait_st();
         }
       }
       l_run = l_run * alpha + lsum;
@@ -264,19 +296,25 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const bool loaded = ok && nblk > 0;
     const bool have = loaded && l_run > 0.0f;
     const float inv_l = have ? 1.0f / l_run : 0.0f;
-    for (int c0 = 0; c0 < 128; c0 += 16) {
-      float o16[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) o16[q] = 0.0f;
-      if (loaded) tmem_ld16(tO + c0, o16);
+    for (int half = 0; half < 2; ++half) {
+      uint32_t o[4][16];
+      if (loaded) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld16_nw(tO + half * 64 + q * 16, o[q]);
+        tmem_wait_ld();
+      }
       if (row_valid) {
 #pragma unroll
-        for (int q = 0; q < 16; q += 4) {
-          const float4 o4 = have ? make_float4(o16[q] * inv_l, o16[q + 1] * inv_l, o16[q + 2] * inv_l,
-                                               o16[q + 3] * inv_l)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-          *reinterpret_cast<float4*>(op + c0 + q) = o4;
-        }
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int u = 0; u < 16; u += 4) {
+            const float4 o4 = have ? make_float4(__uint_as_float(o[q][u]) * inv_l, __uint_as_float(o[q][u + 1]) * inv_l,
+                                                 __uint_as_float(o[q][u + 2]) * inv_l,
+                                                 __uint_as_float(o[q][u + 3]) * inv_l)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(op + half * 64 + q * 16 + u) = o4;
+          }
       }
     }
     if (row_valid) a.lse_part[(long long)split * rows_total + row] = have ? m_run + log2f(l_run) : -INFINITY;

@@ -49,6 +49,18 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
 
+// Four consecutive values as floats (p 16-byte aligned for float, 8-byte for bf16).
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+template <> __device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+  return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+}
+
 // Four consecutive values (p 16-byte aligned for float, 8-byte for bf16).
 template <typename T> __device__ __forceinline__ void store4(T* p, float a, float b, float c, float d);
 template <> __device__ __forceinline__ void store4<float>(float* p, float a, float b, float c, float d) {
@@ -127,7 +139,11 @@ __device__ __forceinline__ float dg_logf(float x) {
 __device__ __forceinline__ float dg_expf(float x) {
   if (x < -86.0f) return 0.0f;
   const float t = __fmul_rn(x, DG_F(0x3FB8AA3Bu));
-  const float k = rintf(t);
+  // rint(t) for |t| < 2^22: adding 1.5 * 2^23 rounds to an integer (ties to
+  // even) in the low mantissa bits; subtracting it back is exact.  Integer
+  // arithmetic only: no conversion unit.
+  const float tk = __fadd_rn(t, 12582912.0f);
+  const float k = __fsub_rn(tk, 12582912.0f);
   const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(k, DG_F(0x3F317200u))),
                             __fmul_rn(k, DG_F(0x35BFBE8Eu)));
   float p = DG_F(0x39500D01u);                            // 1/7!
@@ -138,8 +154,20 @@ __device__ __forceinline__ float dg_expf(float x) {
   p = __fadd_rn(__fmul_rn(p, r), 0.5f);
   p = __fadd_rn(__fmul_rn(p, r), 1.0f);
   p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  const int ki = (int)k;
+  const int ki = __float_as_int(tk) - 0x4B400000;   // == (int)k
   return __fmul_rn(p, __uint_as_float((uint32_t)(ki + 127) << 23));
+}
+
+// trunc(x * 2^40) as int64 for |x| < 2^23, by exponent and mantissa shifts
+// (bit-identical to converting the exact product x * 2^40 toward zero).
+__device__ __forceinline__ long long q40_trunc(float x) {
+  const uint32_t b = __float_as_uint(x);
+  const int e = (int)((b >> 23) & 0xFFu);
+  if (e == 0) return 0;                               // zero (no subnormal inputs here)
+  const uint64_t m = (uint64_t)((b & 0x007FFFFFu) | 0x00800000u);
+  const int sh = e - 127 - 23 + 40;                   // x * 2^40 = m * 2^sh
+  const uint64_t v = sh >= 0 ? (m << sh) : (sh > -64 ? (m >> -sh) : 0ull);
+  return (b >> 31) ? -(long long)v : (long long)v;
 }
 
 // cos(2 pi u) for u in (0,1): fold to b in [0,1/8] by the cosine symmetries,
@@ -332,6 +360,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// Issue-only variants: several loads (or stores) in flight, then one wait.
+__device__ __forceinline__ void tmem_ld16_nw(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st16_nw(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"

@@ -126,7 +126,9 @@ __global__ void k_embed_norm(const int* __restrict__ ids, const T* __restrict__ 
 }
 
 // Attention residual fused with the MoE RMSNorm:
-// h = round(h + sum_s ws[s]);  x = RMSNorm(h).  One CTA per row.
+// h = round(h + sum_s ws[s]);  x = RMSNorm(h).  One CTA per row.  Rows of up
+// to 16 values per thread stay in registers, with every load issued before
+// the first use; longer rows take the strided loop.
 template <typename T>
 __global__ void k_residual_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ ws,
                                 long long split_stride, int splits, int d, float eps) {
@@ -135,6 +137,47 @@ __global__ void k_residual_norm(T* __restrict__ h, T* __restrict__ x, const floa
   const long long t = blockIdx.x;
   T* hr = h + t * d;
   const float* w = ws + t * d;
+  constexpr int G = 4;
+  if (d <= G * 4 * (int)blockDim.x) {
+    float4 v[G], hv[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int i = (threadIdx.x + g * blockDim.x) * 4;
+      if (i < d) { v[g] = *reinterpret_cast<const float4*>(w + i); hv[g] = load4<T>(hr + i); }
+    }
+    for (int s = 1; s < splits; ++s) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int i = (threadIdx.x + g * blockDim.x) * 4;
+        if (i < d) {
+          const float4 u = *reinterpret_cast<const float4*>(w + s * split_stride + i);
+          v[g].x += u.x; v[g].y += u.y; v[g].z += u.z; v[g].w += u.w;
+        }
+      }
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int i = (threadIdx.x + g * blockDim.x) * 4;
+      if (i < d) {
+        hv[g] = make_float4(to_f(from_f<T>(hv[g].x + v[g].x)), to_f(from_f<T>(hv[g].y + v[g].y)),
+                            to_f(from_f<T>(hv[g].z + v[g].z)), to_f(from_f<T>(hv[g].w + v[g].w)));
+        store4<T>(hr + i, hv[g].x, hv[g].y, hv[g].z, hv[g].w);
+        ss = fmaf(hv[g].x, hv[g].x, ss);
+        ss = fmaf(hv[g].y, hv[g].y, ss);
+        ss = fmaf(hv[g].z, hv[g].z, ss);
+        ss = fmaf(hv[g].w, hv[g].w, ss);
+      }
+    }
+    const float tot = block_sum(ss, red);
+    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)d), eps)));
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int i = (threadIdx.x + g * blockDim.x) * 4;
+      if (i < d) store4<T>(x + t * d + i, hv[g].x * r, hv[g].y * r, hv[g].z * r, hv[g].w * r);
+    }
+    return;
+  }
   float ss = 0.0f;
   for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
     float4 v = *reinterpret_cast<const float4*>(w + i);
@@ -572,19 +615,22 @@ __device__ __forceinline__ ArgBest warp_argmax(ArgBest x) {
 }
 
 // Vocab-wide sampler pass.  One cluster of kSampCta CTAs per row; CTA r of
-// the cluster owns the contiguous vocab slice [r V/kSampCta, (r+1) V/kSampCta)
-// and keeps it in shared memory, so the logits are read from global memory
-// once.  Partial results are exchanged through distributed shared memory and
-// every CTA combines them in rank order (integer sums are exact, arg-maxima
-// break ties to the lower index), so all CTAs hold the same row values.
+// the cluster owns the contiguous vocab slice [r V/kSampCta, (r+1) V/kSampCta).
+// Partial results are exchanged through distributed shared memory and every
+// CTA combines them in rank order (integer sums are exact, arg-maxima break
+// ties to the lower index), so all CTAs hold the same row values.
 //   pass 1: max / argmax of the logits, and the Gumbel-max key
 //           argmax_v (l_v / T + g_v), g_v = -ln(-ln u_v).  Since
-//           -ln u >= 1 - u, g_v <= -ln(1 - u_v) (1 - u_v is exact in binary32);
-//           the exact g_v is evaluated only where that bound plus a margin
-//           reaches the thread's best key, so the winner is unchanged.
+//           -ln u >= 1 - u, g_v <= -ln(1 - u_v) <= -E ln 2 with E the binary
+//           exponent of 1 - u_v (exact in binary32); the exact g_v is
+//           evaluated only where that bound plus a margin reaches the
+//           thread's best key, so the winner is unchanged.
 //   pass 2: e_v = exp(l_v - m) (own binary32 exp), S and U = sum e (l - m) as
-//           truncated Q40 int64; e_v replaces l_v in shared memory.
-//   pass 3: probabilities e_v / S in the storage dtype.
+//           truncated Q40 int64.
+//   pass 3: probabilities e_v / S in the storage dtype (e_v recomputed).
+// Passes 2 and 3 re-read the slice (from L2); nothing is staged in shared
+// memory, so several clusters share an SM.  The arithmetic uses no
+// conversion-unit instructions per element.
 // ---------------------------------------------------------------------------
 constexpr int kSampCta = 8;        // CTAs per row (one thread-block cluster)
 constexpr int kSampThreads = 256;
@@ -610,7 +656,6 @@ template <typename T>
 __global__ void __cluster_dims__(kSampCta, 1, 1) __launch_bounds__(kSampThreads)
 k_sampler(SamplerArgs a, T* __restrict__ probs) {
   pdl_enter();
-  extern __shared__ float4 sl4[];                 // this CTA's slice (logits, then e)
   __shared__ SampPart part;
   __shared__ ArgBest red_m[32], red_g[32];
   __shared__ long long red_s[32], red_u[32];
@@ -632,7 +677,6 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
   ArgBest bm{-INFINITY, -1}, bg{-INFINITY, -1};
   for (int i = threadIdx.x; i < n4; i += blockDim.x) {
     const float4 l = l4[i];
-    sl4[i] = l;
     const int v4 = g0 + i;
     const uint4 w = philox4x32_10(make_uint4((uint32_t)v4, (uint32_t)pos, (uint32_t)step, STREAM_GUMBEL), k0, k1);
     const float lv[4] = {l.x, l.y, l.z, l.w};
@@ -642,9 +686,13 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
       const int v = v4 * 4 + j;
       bm = arg_better(bm, ArgBest{lv[j], v});
       const float lt = __fmul_rn(lv[j], inv_t);
-      // 1 - u exactly: u = (2 (x >> 9) + 1) 2^-24
-      const float one_minus_u = (float)(0x1000000u - (((wv[j] >> 9) << 1) | 1u)) * 5.9604644775390625e-8f;
-      const float g_ub = -__logf(one_minus_u);
+      // 1 - u, u = (2 (x >> 9) + 1) 2^-24, exactly in binary32 from f =
+      // 1 + (x >> 9) 2^-23: (2 - f) - 2^-24.  Its binary exponent E (in
+      // [-24, -1]) gives g <= -E ln 2 (-E as a float through the 2^23 trick).
+      const float f = __uint_as_float(0x3F800000u | (wv[j] >> 9));
+      const float omu = __fsub_rn(__fsub_rn(2.0f, f), 5.9604644775390625e-8f);
+      const int negE = 127 - (int)(__float_as_uint(omu) >> 23);
+      const float g_ub = __fmul_rn(__fsub_rn(__int_as_float(0x4B000000 + negE), 8388608.0f), 0.69314718f);
       if (bg.i < 0 || lt + g_ub + (1e-3f + 1e-5f * fabsf(bg.v)) >= bg.v) {
         const float key = __fadd_rn(lt, gumbel_of(wv[j]));
         bg = arg_better(bg, ArgBest{key, v});
@@ -678,17 +726,15 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
   // pass 2
   long long sq = 0, uq = 0;
   for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-    const float4 l = sl4[i];
+    const float4 l = l4[i];
     const float lv[4] = {l.x, l.y, l.z, l.w};
-    float ev[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float dlt = __fsub_rn(lv[j], m);
-      ev[j] = dg_expf(dlt);
-      sq += __float2ll_rz(__fmul_rn(ev[j], 1099511627776.0f));
-      uq += __float2ll_rz(__fmul_rn(__fmul_rn(ev[j], dlt), 1099511627776.0f));
+      const float e = dg_expf(dlt);
+      sq += q40_trunc(e);
+      uq += q40_trunc(__fmul_rn(e, dlt));
     }
-    sl4[i] = make_float4(ev[0], ev[1], ev[2], ev[3]);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -724,9 +770,10 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
     const float inv_s = __fdiv_rn(1.0f, __fmul_rn(__ll2float_rn(S), 9.094947017729282e-13f));
     T* pr = probs + row * a.vocab + (long long)g0 * 4;
     for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-      const float4 e = sl4[i];
-      store4<T>(pr + (long long)i * 4, __fmul_rn(e.x, inv_s), __fmul_rn(e.y, inv_s), __fmul_rn(e.z, inv_s),
-                __fmul_rn(e.w, inv_s));
+      const float4 l = l4[i];
+      store4<T>(pr + (long long)i * 4, __fmul_rn(dg_expf(__fsub_rn(l.x, m)), inv_s),
+                __fmul_rn(dg_expf(__fsub_rn(l.y, m)), inv_s), __fmul_rn(dg_expf(__fsub_rn(l.z, m)), inv_s),
+                __fmul_rn(dg_expf(__fsub_rn(l.w, m)), inv_s));
     }
   }
 }
@@ -734,13 +781,7 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
 // Launch of the sampler over `rows` rows (vocab % (4 kSampCta) == 0).
 template <typename T>
 cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cudaStream_t s, bool pdl) {
-  const size_t smem = (size_t)sa.vocab / kSampCta * sizeof(float);
-  static size_t attr_bytes = 0;   // dynamic shared memory the kernel is currently allowed
-  if (smem > attr_bytes) {
-    const cudaError_t e = cudaFuncSetAttribute(k_sampler<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_bytes = smem;
-  }
+  const size_t smem = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * kSampCta));
   cfg.blockDim = dim3(kSampThreads);

@@ -54,7 +54,7 @@ enum { DG_STOP_MEAN = 0, DG_STOP_EB = 1 };
 /* Architecture + sampler.  Requirements checked by dg_init_weights:
  * canvas_len == 256; head_dim in {64, 128} (128 for DG_BF16); n_heads a
  * multiple of n_kv_heads with 128 % (n_heads / n_kv_heads) == 0;
- * d_model, d_ff multiples of 64; vocab a multiple of 64, at most 458752; top_k <= n_experts
+ * d_model, d_ff multiples of 64; vocab a multiple of 64; top_k <= n_experts
  * <= 1024, top_k <= 64; 1 <= max_canvases; max_prompt >= 1. */
 typedef struct dg_config {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim;
