@@ -243,12 +243,13 @@ def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, persistent=False, m256=F
                               float(alpha), k_splits, bn, flags, _stream(stream)), "dg_test_gemm")
 
 
-def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, stream=None):
+def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, sized_ring=False, stream=None):
     import torch
     K = A.shape[-1]
     c = (ctypes.c_int32 * groups)(*[int(x) for x in counts])
+    flags = int(persistent) | (2 if sized_ring else 0)
     _check(lib().dg_test_grouped_gemm(_ptr(A), _ptr(B), c, groups, M, K, 1 if A.dtype == torch.bfloat16 else 0,
-                                      bn, int(persistent), _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
+                                      bn, flags, _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
 
 
 def test_attention(q, k, v, n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out, stream=None):

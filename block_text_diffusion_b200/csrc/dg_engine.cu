@@ -147,7 +147,7 @@ struct dg_model {
   float* ws = nullptr;
   float *o_part = nullptr, *lse_part = nullptr;
   int *ids = nullptr, *perm = nullptr, *inv = nullptr, *work_count = nullptr, *counts = nullptr;
-  int* moe_splits = nullptr;         // [2] split-K of the gate|up and down GEMMs (set by permute)
+  int* moe_splits = nullptr;         // [3] split-K of the gate|up and down GEMMs, largest item rows (set by permute)
   float* gate = nullptr;
   int4* work = nullptr;
   float *logits = nullptr, *H = nullptr;
@@ -276,6 +276,7 @@ struct GemmCall {
   int bn = 256;
   bool persistent = false;           // walk tiles with one CTA per SM slot
   const int* k_splits_dev = nullptr; // persistent: split-K count decided on the device (<= splits)
+  const int* max_rows_dev = nullptr; // persistent grouped: rows of the largest work item (sizes the ring)
   bool m256 = false;                 // dense, bn 256: 256-row M tiles (two accumulators share B)
 };
 
@@ -331,6 +332,7 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   a.work_count = g.work_count;
   a.a_group_rows = g.a_group_rows;
   a.k_splits_dev = g.persistent ? g.k_splits_dev : nullptr;
+  a.max_rows_dev = g.persistent ? g.max_rows_dev : nullptr;
   a.err = &m->st->err;
   if (!m->bf) {
     a.m_tiles = cdiv(g.M, 64);
@@ -633,6 +635,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     gu.work = m->work; gu.work_count = m->work_count; gu.a_group_rows = 2 * m->ff;
     gu.max_items = max_items; gu.bn = bn_g; gu.persistent = m->bf;
     gu.split_stride = gu_stride; gu.k_splits_dev = m->bf ? m->moe_splits : nullptr;
+    gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     gu.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
     { LaunchScope ls(m, s, PH_SWIGLU);
@@ -645,6 +648,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.work = m->work; dn.work_count = m->work_count; dn.a_group_rows = d;
     dn.max_items = max_items; dn.bn = bn_g; dn.persistent = m->bf;
     dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
+    dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
@@ -947,7 +951,7 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   A((void**)&m->inv, Tk * sizeof(int));
   A((void**)&m->work, ((size_t)m->E + Tk / 16 + 8) * sizeof(int4));
   A((void**)&m->work_count, sizeof(int));
-  A((void**)&m->moe_splits, 2 * sizeof(int));
+  A((void**)&m->moe_splits, 4 * sizeof(int));
   A((void**)&m->counts, (size_t)m->L * m->E * sizeof(int));
   A((void**)&m->logits, (size_t)m->T_cap * V * sizeof(float));
   A((void**)&m->H, (size_t)m->T_cap * sizeof(float));

@@ -29,6 +29,7 @@ struct GemmArgs {
   int a_group_rows;        // grouped: A rows per group (a_row0 = group * a_group_rows)
   const int* work_count;
   const int* k_splits_dev; // persistent kernel: split-K factor chosen on the device (overrides k_splits)
+  const int* max_rows_dev; // persistent kernel: rows of the largest work item (sizes the ring stages)
   int* err;
 };
 
@@ -230,16 +231,20 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   using C = GemmTcCfg<BN, STAGES>;
   constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
   constexpr int kAllocCols = 2 * kAccCols;             // two buffers (<= 512)
+  // The ring holds STAGES full-size stages; when every work item has fewer
+  // rows than BN, stages shrink to A + the rows actually loaded and the ring
+  // holds more of them (more weight bytes in flight per SM).
+  constexpr int kMaxStages = 3 * STAGES;
   pdl_launch();
   GemmArgs p = p_in;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES], acc_full[2], acc_empty[2];
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ int4 s_work[kWorkSmem];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int s = 0; s < kMaxStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     fence_mbar_init();
     prefetch_tmap(&tmA);
@@ -250,6 +255,11 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   pdl_wait();
   if (p.k_splits_dev) p.k_splits = max(1, min(*p.k_splits_dev, p.kb_total));
   const int n_items = p.work ? *p.work_count : items_dense;
+  // ring geometry from the largest B tile any work item loads
+  int rows_max = BN;
+  if (p.max_rows_dev) rows_max = min(BN, max(kBoxRowsB, *p.max_rows_dev));
+  const int stage_bytes = C::kABytes + ((rows_max + kBoxRowsB - 1) / kBoxRowsB) * kBoxRowsB * 128;
+  const int n_stages = min(kMaxStages, (STAGES * C::kStage) / stage_bytes);
   const int total = p.m_tiles * p.k_splits * n_items;
   // work items are read by all three roles once per tile: stage them on chip
   const bool work_smem = p.work != nullptr && n_items <= kWorkSmem;
@@ -283,10 +293,10 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int n_boxes = (min(BN, (t.n_valid + 15) & ~15) + kBoxRowsB - 1) / kBoxRowsB;
         const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (it >= STAGES && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) { ok = false; break; }
-          uint8_t* a_s = smem + s * C::kStage;
+          const int s = it % n_stages;
+          const uint32_t ph = (it / n_stages) & 1;
+          if (it >= n_stages && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) { ok = false; break; }
+          uint8_t* a_s = smem + s * stage_bytes;
           uint8_t* b_s = a_s + C::kABytes;
           mbar_expect_tx(&full_bar[s], tx);
           tma_load_2d(a_s, &tmA, kb * 64, t.a_row0 + t.m_tile * 128, &full_bar[s]);
@@ -320,11 +330,11 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem + buf * kAccCols;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
+          const int s = it % n_stages;
+          const uint32_t ph = (it / n_stages) & 1;
           if (!mbar_wait(&full_bar[s], ph, p.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * C::kStage);
+          const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
           const uint64_t ad = sdesc_sw128(a_addr), bd = sdesc_sw128(a_addr + C::kABytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)

@@ -431,8 +431,8 @@ __global__ void k_router_bias_f32(float* bias, int E, float s) {
 // places the pairs of experts w, w+32, ... in pair order (stable).
 // ---------------------------------------------------------------------------
 // Split-K factors of the two expert GEMMs, chosen here on the device from the
-// number of work items so that their tiles fill about eight waves of SMs:
-// splits_out[g] for g = 0 (gate|up) and 1 (down) from (m tiles, k blocks, cap).
+// number of work items: out[g] for g = 0 (gate|up) and 1 (down) from (m tiles,
+// k blocks, cap); out[2] = rows of the largest work item.
 struct SplitPlan {
   int mt[2], kb[2], cap[2];
   int* out;
@@ -478,8 +478,10 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0, nw = 0;
+    int max_rows = 0;
     for (int e = 0; e < E; ++e) {
       const int c = offs[e];
+      max_rows = max(max_rows, min(c, bn));
       if (counts_out) counts_out[e] = c;
       offs[e] = acc;
       for (int r = 0; r < c; r += bn) work[nw++] = make_int4(e, acc + r, min(bn, c - r), acc + r);
@@ -506,6 +508,7 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
         }
         plan.out[g] = best;
       }
+      plan.out[2] = max_rows;
     }
   }
   __syncthreads();

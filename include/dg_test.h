@@ -58,7 +58,8 @@ dg_status dg_test_gemm(const void* A, const void* B, float* out, int32_t M, int3
 
 /* Grouped GEMM as used by the experts: A [groups*M, K], B [rows, K] with
  * rows ordered by group (counts host int32 [groups]); out [rows, M] fp32,
- * out[r][m] = sum_k A[g(r)*M + m][k] B[r][k]; flags as dg_test_gemm.
+ * out[r][m] = sum_k A[g(r)*M + m][k] B[r][k]; flags bit 0 as dg_test_gemm,
+ * bit 1 (persistent only) sizes the ring stages from the largest item.
  * Allocates. */
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
                                int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);

@@ -253,8 +253,9 @@ def test_gemm_f32():
     (2816, 128, [5, 0, 0, 130, 256, 257], 256, True),
     (1024, 128, [7, 0, 70, 1], 128, True),
     (1024, 256, [0, 9, 64, 65, 1], 64, False),
+    (1408, 2816, [17, 3, 0, 31, 12, 1, 9, 20], 256, True),
 ])
-@pytest.mark.parametrize("persistent", [False, True])
+@pytest.mark.parametrize("persistent", [False, True, "sized_ring"])
 def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     g = np.random.default_rng(sum(counts) + M)
     G = len(counts)
@@ -266,7 +267,10 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     At = bf16_tensor(A) if bf else cu(A)
     Bt = bf16_tensor(B) if bf else cu(B)
     out = torch.full((rows, M), float("nan"), dtype=torch.float32, device="cuda")
-    dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn, persistent=persistent and bf)
+    # "sized_ring": the persistent kernel's ring stages shrink to the largest
+    # item (more stages in flight), as the expert GEMMs run in the step
+    dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn, persistent=bool(persistent) and bf,
+                         sized_ring=persistent == "sized_ring" and bf)
     got = host(out).astype(np.float64)
     r0 = 0
     for e, c in enumerate(counts):
