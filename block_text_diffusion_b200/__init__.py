@@ -71,6 +71,7 @@ def lib():
             "dg_test_commit": ([P, P, P, P, I32, I32, U64, I32, I32, I32, F, I32, F, P, P, P, P, P], I32),
             "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, I32, P], I32),
             "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
+            "dg_test_router": ([P, P, P, I32, I32, I32, I32, P, P, P], I32),
             "dg_test_attention": ([P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P], I32),
             "dg_read_weight": ([P, I32, P, P], I32),
             "dg_load_kv": ([P, P, I32, I32, P, P, P], I32),
@@ -241,6 +242,14 @@ def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, persistent=False, m256=F
     flags = int(persistent) | (2 if m256 else 0)
     _check(lib().dg_test_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, 1 if A.dtype == torch.bfloat16 else 0,
                               float(alpha), k_splits, bn, flags, _stream(stream)), "dg_test_gemm")
+
+
+def test_router(x, wr, ids, gate, bias=None, stream=None):
+    T, d = x.shape
+    E = wr.shape[0]
+    k = ids.shape[1]
+    _check(lib().dg_test_router(_ptr(x), _ptr(wr), _ptr(bias) if bias is not None else None, T, d, E, k,
+                                _ptr(ids), _ptr(gate), _stream(stream)), "dg_test_router")
 
 
 def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, sized_ring=False, stream=None):

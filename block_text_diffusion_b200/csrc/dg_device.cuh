@@ -205,6 +205,20 @@ __device__ __forceinline__ float gumbel_of(uint32_t word) {
   return -dg_logf(-dg_logf(uniform_open(word)));
 }
 
+// Thread-block clusters: barrier over every thread of every CTA of the
+// cluster (release / acquire), and distributed shared memory addressing.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
+template <typename P>
+__device__ __forceinline__ const P* cluster_peer(const P* p, int rank) {
+  uint64_t out;
+  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"((uint64_t)p), "r"(rank));
+  return reinterpret_cast<const P*>(out);
+}
+
 // ---------------------------------------------------------------------------
 // Bounded waiting: every spin gives up after ~2 s of wall time (globaltimer)
 // and reports failure instead of hanging the GPU.

@@ -643,18 +643,6 @@ struct SampPart {
   long long s, u;
 };
 
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
-}
-
-// Address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
-template <typename P>
-__device__ __forceinline__ const P* cluster_peer(const P* p, int rank) {
-  uint64_t out;
-  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"((uint64_t)p), "r"(rank));
-  return reinterpret_cast<const P*>(out);
-}
-
 template <typename T>
 __global__ void __cluster_dims__(kSampCta, 1, 1) __launch_bounds__(kSampThreads)
 k_sampler(SamplerArgs a, T* __restrict__ probs) {

@@ -56,6 +56,15 @@ dg_status dg_test_commit(const float* H, const int32_t* tok, const int32_t* amax
 dg_status dg_test_gemm(const void* A, const void* B, float* out, int32_t M, int32_t N, int32_t K, int32_t bf16,
                        float alpha, int32_t k_splits, int32_t bn, int32_t flags, void* stream);
 
+/* The bf16 router kernel: logits r = x Wr^T (+ bias, fp32, may be NULL) for
+ * x bf16 [T, d] and Wr bf16 [E, d] (E <= 128, d % 64 == 0), then per token
+ * the k <= 32 largest logits (ties to the lower expert id) in descending
+ * order -> ids int32 [T, k], and their softmax -> gate fp32 [T, k]
+ * (Mixture-of-Experts FFN, DiffusionGemma technical-report explainer,
+ * section 二).  Allocates (a 32-byte error word); synchronises. */
+dg_status dg_test_router(const void* x, const void* wr, const float* bias, int32_t T, int32_t d, int32_t E,
+                         int32_t k, int32_t* ids, float* gate, void* stream);
+
 /* Grouped GEMM as used by the experts: A [groups*M, K], B [rows, K] with
  * rows ordered by group (counts host int32 [groups]); out [rows, M] fp32,
  * out[r][m] = sum_k A[g(r)*M + m][k] B[r][k]; flags bit 0 as dg_test_gemm,

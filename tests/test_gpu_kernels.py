@@ -281,6 +281,43 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
         r0 += c
 
 
+# --- router -----------------------------------------------------------------------------
+@pytest.mark.parametrize("T,d,E,k,zipf", [(256, 2816, 128, 8, 0.0), (77, 1024, 32, 4, 0.0),
+                                          (1024, 1024, 32, 4, 1.1), (40, 512, 100, 5, 0.0)])
+def test_router_kernel(T, d, E, k, zipf):
+    # top-k ids identical to the oracle's wherever the decision is farther
+    # from a tie than the fp32 accumulation error can move it; gates within
+    # 1e-4 of the fp64 softmax
+    g = np.random.default_rng(T + d + E)
+    x = I._bf16_grid(g.standard_normal((T, d)).astype(F32))
+    wr = I._bf16_grid((0.02 * g.standard_normal((E, d))).astype(F32))
+    bias = None
+    if zipf:
+        bias = cu((-zipf * np.log(np.arange(E, dtype=np.float64) + 1.0)).astype(F32))
+    ids = torch.zeros((T, k), dtype=torch.int32, device="cuda")
+    gate = torch.zeros((T, k), dtype=torch.float32, device="cuda")
+    dg.test_router(bf16_tensor(x), bf16_tensor(wr), ids, gate, bias=bias)
+    gi, gg = host(ids), host(gate)
+    oi, ow = om.router(x, wr, k, zipf_s=zipf)
+    r = x.astype(np.float64) @ wr.astype(np.float64).T
+    if zipf:
+        r += (-zipf * np.log(np.arange(E) + 1.0))[None, :]
+    # fp32 accumulation error bound, plus the binary32 rounding of the bias
+    err = 4e-6 * (np.abs(x.astype(np.float64)) @ np.abs(wr.astype(np.float64)).T).max(axis=1) + 1e-6 + 1e-5 * zipf
+    srt = -np.sort(-r, axis=1)
+    gaps = srt[:, :k] - srt[:, 1:k + 1]                       # adjacent gaps through the (k+1)-th
+    safe_set = gaps[:, k - 1] > 2 * err
+    safe_order = gaps.min(axis=1) > 2 * err
+    assert safe_order.mean() > 0.5
+    for t in range(T):
+        if safe_order[t]:
+            assert np.array_equal(gi[t], oi[t]), t
+        elif safe_set[t]:
+            assert set(gi[t]) == set(oi[t]), t
+    assert np.allclose(gg[safe_order], ow[safe_order], atol=1e-4)
+    assert np.allclose(gg.sum(axis=1), 1.0, atol=1e-5)
+
+
 # --- attention --------------------------------------------------------------------------
 def _attn_ref(q, k, v, n_canvas, n_q, q_pos0, causal, rows=None):
     out = []
