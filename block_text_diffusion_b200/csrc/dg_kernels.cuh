@@ -438,6 +438,34 @@ struct SplitPlan {
   int* out;
 };
 
+// Exclusive prefix sum of one int per thread over the block (blockDim a
+// multiple of 32); *total receives the block sum.  Uses wsum[32].
+__device__ __forceinline__ int block_scan_excl(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < nw) wsum[lane] = t;
+  }
+  __syncthreads();
+  const int base = warp > 0 ? wsum[warp - 1] : 0;
+  *total = wsum[nw - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
 __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int bn, int* __restrict__ perm,
                           int* __restrict__ inv, int4* __restrict__ work, int* __restrict__ work_count,
                           int* __restrict__ counts_out, SplitPlan plan, int* err) {
@@ -476,18 +504,33 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
     offs[e] = acc;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0, nw = 0;
-    int max_rows = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = offs[e];
-      max_rows = max(max_rows, min(c, bn));
+  // expert offsets and work items: block-wide exclusive scans of the expert
+  // row counts and item counts (chunks of blockDim experts, with carries)
+  __shared__ int wsum[32], s_max_rows;
+  if (threadIdx.x == 0) s_max_rows = 0;
+  int carry_rows = 0, carry_items = 0;
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    const int c = e < E ? offs[e] : 0;
+    const int it = (c + bn - 1) / bn;
+    int tot_rows, tot_items;
+    const int pr = block_scan_excl(c, wsum, &tot_rows);
+    const int pi = block_scan_excl(it, wsum, &tot_items);
+    if (e < E) {
+      const int acc = carry_rows + pr, nw0 = carry_items + pi;
       if (counts_out) counts_out[e] = c;
       offs[e] = acc;
-      for (int r = 0; r < c; r += bn) work[nw++] = make_int4(e, acc + r, min(bn, c - r), acc + r);
-      acc += c;
+      for (int j = 0; j < it; ++j)
+        work[nw0 + j] = make_int4(e, acc + j * bn, min(bn, c - j * bn), acc + j * bn);
+      if (c > 0) atomicMax(&s_max_rows, min(c, bn));
     }
-    offs[E] = acc;
+    carry_rows += tot_rows;
+    carry_items += tot_items;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int nw = carry_items;
+    offs[E] = carry_rows;
     *work_count = nw;
     if (plan.out) {
       // Split-K factor per GEMM: the persistent kernel runs ceil(tiles / SMs)
@@ -508,7 +551,7 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
         }
         plan.out[g] = best;
       }
-      plan.out[2] = max_rows;
+      plan.out[2] = s_max_rows;
     }
   }
   __syncthreads();
