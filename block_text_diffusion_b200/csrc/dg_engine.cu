@@ -278,6 +278,8 @@ struct GemmCall {
   bool persistent = false;           // walk tiles with one CTA per SM slot
   const int* k_splits_dev = nullptr; // persistent: split-K count decided on the device (<= splits)
   const int* max_rows_dev = nullptr; // persistent grouped: rows of the largest work item (sizes the ring)
+  void* act = nullptr;               // persistent gate|up: SwiGLU output (bf16) when the GEMM runs unsplit
+  int act_ld = 0;
   bool m256 = false;                 // dense, bn 256: 256-row M tiles (two accumulators share B)
 };
 
@@ -334,6 +336,8 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   a.a_group_rows = g.a_group_rows;
   a.k_splits_dev = g.persistent ? g.k_splits_dev : nullptr;
   a.max_rows_dev = g.persistent ? g.max_rows_dev : nullptr;
+  a.act = g.persistent ? g.act : nullptr;
+  a.act_ld = g.act_ld;
   a.err = &m->st->err;
   if (!m->bf) {
     a.m_tiles = cdiv(g.M, 64);
@@ -444,8 +448,11 @@ dg_status init_all_weights(dg_model* m, uint64_t seed, cudaStream_t s) {
     init_tensor<T>((T*)w.qkv, nk * d, nk * d, nk * d, (nq + nk) * d, seed, tid_layer(l, 2), s);
     init_tensor<T>((T*)w.wo, d * nq, d * nq, d * nq, 0, seed, tid_layer(l, 3), s);
     init_tensor<T>((T*)w.wr, E * d, E * d, E * d, 0, seed, tid_layer(l, 4), s);
-    init_tensor<T>((T*)w.gu, E * ff * d, ff * d, 2 * ff * d, 0, seed, tid_layer(l, 5), s);
-    init_tensor<T>((T*)w.gu, E * ff * d, ff * d, 2 * ff * d, ff * d, seed, tid_layer(l, 6), s);
+    // gate | up interleaved in blocks of 64 rows: rows [128 i, 128 i + 64) of
+    // an expert are gate rows 64 i.., the next 64 the matching up rows, so a
+    // 128-row GEMM tile holds both halves of 64 SwiGLU outputs
+    init_tensor<T>((T*)w.gu, E * ff * d, 64 * d, 128 * d, 0, seed, tid_layer(l, 5), s);
+    init_tensor<T>((T*)w.gu, E * ff * d, 64 * d, 128 * d, 64 * d, seed, tid_layer(l, 6), s);
     init_tensor<T>((T*)w.wd, E * d * ff, E * d * ff, E * d * ff, 0, seed, tid_layer(l, 7), s);
   }
   CU_TRY(cudaGetLastError());
@@ -637,6 +644,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     plan.mt[1] = cdiv(d, 128); plan.kb[1] = cdiv(m->ff, 64);
     plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
     plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
+    plan.fused0 = m->bf ? 1 : 0;
     plan.out = m->moe_splits;
     { LaunchScope ls(m, s, PH_PERMUTE);
       launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
@@ -652,11 +660,13 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     gu.split_stride = gu_stride; gu.k_splits_dev = m->bf ? m->moe_splits : nullptr;
     gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     gu.splits = m->bf ? 8 : 1;
+    // bf16: an unsplit gate|up GEMM applies SwiGLU in its epilogue
+    if (m->bf) { gu.act = m->act; gu.act_ld = m->ff; }
     DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
     { LaunchScope ls(m, s, PH_SWIGLU);
       const long long n = (long long)n_pairs * m->ff;
       launch_pdl(k_swiglu<T>, std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s, m->ws, m->ff, n, (T*)m->act,
-                                                                        m->moe_splits, gu_stride); }
+                                                                        m->moe_splits, gu_stride, m->bf ? 1 : 0); }
     GemmCall dn;
     dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
     dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;

@@ -30,6 +30,10 @@ struct GemmArgs {
   const int* work_count;
   const int* k_splits_dev; // persistent kernel: split-K factor chosen on the device (overrides k_splits)
   const int* max_rows_dev; // persistent kernel: rows of the largest work item (sizes the ring stages)
+  void* act;               // persistent gate|up: when non-null and the split factor is 1, the
+                           // epilogue writes round(silu(g) u) (bf16, row stride act_ld) instead
+                           // of the fp32 output; A rows interleave gate / up in blocks of 64
+  int act_ld;
   int* err;
 };
 
@@ -224,6 +228,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 // ---------------------------------------------------------------------------
 constexpr int kWorkSmem = 512;   // work items staged in shared memory (more are read from global)
 
+// Barrier among the four epilogue warps (threads 64..191) of the persistent kernel.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -242,6 +249,8 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ int4 s_work[kWorkSmem];
+  __shared__ float s_xfer[64 * 17];   // fused SwiGLU: up values of one 16-column chunk
+  __shared__ int s_epi_fail;          // fused SwiGLU: an epilogue wait ran out
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
@@ -249,6 +258,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    s_epi_fail = 0;
   }
   if (warp == 0) tmem_alloc(&tmem_base, kAllocCols);
   // the split factor and the work list are written by the permute kernel
@@ -365,6 +375,47 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const bool ok =
           __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, DGDEV_TIMEOUT_EPI));
       tc_fence_after();
+      if (p.act && p.k_splits == 1) {
+        // fused SwiGLU: accumulator rows 0..63 are gate rows of SwiGLU outputs
+        // f = 64 m_t .. 64 m_t + 63, rows 64..127 the matching up rows.  The up
+        // quads hand their values to the gate quads through shared memory.
+        // The four warps first agree on the wait outcome (they share barriers).
+        if (lane == 0 && !ok) s_epi_fail = 1;
+        epi_sync();
+        const bool ok_all = s_epi_fail == 0;
+        bf16* act = reinterpret_cast<bf16*>(p.act);
+        const int f = m_t * 64 + (quad & 1) * 32 + lane;
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t v[16];
+          if (ok_all && kb1 > kb0) {
+            tmem_ld16_nw(tmem + buf * kAccCols + ((uint32_t)(quad * 32) << 16) + c0, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0u;
+          }
+          if (quad >= 2) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) s_xfer[((quad - 2) * 32 + lane) * 17 + j] = __uint_as_float(v[j]);
+          }
+          epi_sync();
+          if (quad < 2) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (c0 + j < n_valid) {
+                const float g = __uint_as_float(v[j]);
+                const float u = s_xfer[(quad * 32 + lane) * 17 + j];
+                act[(long long)(out_row0 + c0 + j) * p.act_ld + f] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+              }
+            }
+          }
+          epi_sync();
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+        if (!ok_all) break;
+        continue;
+      }
       const int m0 = m_t * 128;
       const bool m_ok = (m0 + row) < p.M;
       float* outp = p.out + (long long)split * p.split_stride + (long long)out_row0 * p.ldo + m0 + row;

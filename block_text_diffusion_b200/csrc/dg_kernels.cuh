@@ -435,6 +435,7 @@ __global__ void k_router_bias_f32(float* bias, int E, float s) {
 // k blocks, cap); out[2] = rows of the largest work item.
 struct SplitPlan {
   int mt[2], kb[2], cap[2];
+  int fused0;   // the gate|up GEMM writes the SwiGLU output itself when it runs unsplit
   int* out;
 };
 
@@ -546,7 +547,8 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
         float best_cost = 3.4e38f;
         for (int s = 1; s <= s_max; ++s) {
           const int waves = (plan.mt[g] * nw * s + kSMs - 1) / kSMs;
-          const float cost = (float)waves / (float)s + (float)s * r;
+          // an unsplit fused gate|up GEMM writes no fp32 partials at all
+          const float cost = (float)waves / (float)s + ((g == 0 && plan.fused0 && s == 1) ? 0.0f : (float)s * r);
           if (cost < best_cost) { best_cost = cost; best = s; }
         }
         plan.out[g] = best;
@@ -589,23 +591,28 @@ __global__ void k_gather(const T* __restrict__ x, const int* __restrict__ perm, 
   for (int i = threadIdx.x; i < nv; i += blockDim.x) o[i] = s[i];
 }
 
-// SwiGLU: a = round(silu(g) * u), g/u the gate and up halves of each row,
-// each summed over the split-K partials (count read from the device).
+// SwiGLU: a = round(silu(g) * u) with g / u the gate and up columns of each
+// row of the gate|up GEMM output, interleaved in blocks of 64 (columns
+// [128 i, 128 i + 64) gate, the next 64 up), each summed over the split-K
+// partials (count read from the device).  When `fused` is set and the GEMM ran
+// with one split, its epilogue already wrote `a` and this kernel does nothing.
 template <typename T>
 __global__ void k_swiglu(const float* __restrict__ gu, int ff, long long n, T* __restrict__ a,
-                         const int* __restrict__ splits_dev, long long split_stride) {
+                         const int* __restrict__ splits_dev, long long split_stride, int fused) {
   pdl_enter();
   const int ns = splits_dev ? *splits_dev : 1;
+  if (fused && ns == 1) return;
   const long long n4 = n / 4;   // ff is a multiple of 64
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {
-    const long long e = i * 4, r = e / ff, c = e % ff;
-    const float* gp = gu + r * 2 * ff + c;
+    const long long e = i * 4, r = e / ff;
+    const int c = (int)(e % ff);
+    const float* gp = gu + r * 2 * ff + (c / 64) * 128 + c % 64;
     float4 g = *reinterpret_cast<const float4*>(gp);
-    float4 u = *reinterpret_cast<const float4*>(gp + ff);
+    float4 u = *reinterpret_cast<const float4*>(gp + 64);
     for (int s = 1; s < ns; ++s) {
       const float4 g2 = *reinterpret_cast<const float4*>(gp + s * split_stride);
-      const float4 u2 = *reinterpret_cast<const float4*>(gp + s * split_stride + ff);
+      const float4 u2 = *reinterpret_cast<const float4*>(gp + s * split_stride + 64);
       g.x += g2.x; g.y += g2.y; g.z += g2.z; g.w += g2.w;
       u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
     }

@@ -281,6 +281,34 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
         r0 += c
 
 
+@pytest.mark.parametrize("M,K,counts", [(1408, 2816, [17, 3, 0, 200, 12, 1, 256, 20]), (2048, 1024, [64, 65, 0, 9])])
+def test_grouped_gemm_fused_swiglu(M, K, counts):
+    # the unsplit gate|up GEMM writes round(silu(g) u) itself; A rows interleave
+    # gate / up in blocks of 64
+    g = np.random.default_rng(M + K + sum(counts))
+    G, rows, ff = len(counts), sum(counts), M // 2
+    A = I._bf16_grid((0.05 * g.standard_normal((G * M, K))).astype(F32))
+    B = I._bf16_grid(g.standard_normal((rows, K)).astype(F32))
+    out = torch.zeros((rows, M), dtype=torch.float32, device="cuda")
+    dg.test_grouped_gemm(bf16_tensor(A), bf16_tensor(B), counts, G, M, out, bn=256, persistent=True,
+                         sized_ring=True, swiglu=True)
+    act = out.view(torch.bfloat16).reshape(-1)[:rows * ff].reshape(rows, ff)
+    got = act.float().cpu().numpy().astype(np.float64)
+    f = np.arange(ff)
+    grow, urow = (f // 64) * 128 + f % 64, (f // 64) * 128 + 64 + f % 64
+    r0 = 0
+    for e, c in enumerate(counts):
+        if c:
+            Ae = A[e * M:(e + 1) * M].astype(np.float64)
+            x = B[r0:r0 + c].astype(np.float64)
+            gv, uv = x @ Ae[grow].T, x @ Ae[urow].T
+            ref = gv / (1.0 + np.exp(-gv)) * uv
+            sg, su = np.abs(x) @ np.abs(Ae[grow]).T, np.abs(x) @ np.abs(Ae[urow]).T
+            tol = 2.0 ** -8 * np.abs(ref) + 1e-5 * (sg * (np.abs(uv) + 1.0) + su * (np.abs(gv) + 1.0))
+            assert np.all(np.abs(got[r0:r0 + c] - ref) <= tol), e
+        r0 += c
+
+
 # --- router -----------------------------------------------------------------------------
 @pytest.mark.parametrize("T,d,E,k,zipf", [(256, 2816, 128, 8, 0.0), (77, 1024, 32, 4, 0.0),
                                           (1024, 1024, 32, 4, 1.1), (40, 512, 100, 5, 0.0)])
