@@ -14,6 +14,15 @@
 #pragma once
 #include "dg_device.cuh"
 
+// Timeline probes of the persistent GEMM's CTA 0 (global-timer stamps), only
+// in builds with -DDG_PROBE (performance diagnosis); no-ops otherwise.
+#ifdef DG_PROBE
+__device__ long long g_probe[1024];
+#define DG_PROBE_STAMP(i) do { if (blockIdx.x == 0 && (i) < 1024) g_probe[(i)] = (long long)global_ns(); } while (0)
+#else
+#define DG_PROBE_STAMP(i) do { } while (0)
+#endif
+
 struct GemmArgs {
   int M;                   // valid A rows per work item
   int m_tiles;             // ceil(M / tile M)
@@ -243,6 +252,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   // holds more of them (more weight bytes in flight per SM).
   constexpr int kMaxStages = 3 * STAGES;
   pdl_launch();
+  if (threadIdx.x == 0) DG_PROBE_STAMP(1000);
   GemmArgs p = p_in;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -306,6 +316,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
           const int s = it % n_stages;
           const uint32_t ph = (it / n_stages) & 1;
           if (it >= n_stages && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) { ok = false; break; }
+          if (it < 256) DG_PROBE_STAMP(it);                   // slot free, loads issued
           uint8_t* a_s = smem + s * stage_bytes;
           uint8_t* b_s = a_s + C::kABytes;
           mbar_expect_tx(&full_bar[s], tx);
@@ -337,12 +348,14 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
           ok = false;
           break;
         }
+        if (local < 64) DG_PROBE_STAMP(512 + local);          // accumulator free
         tc_fence_after();
         const uint32_t d_tmem = tmem + buf * kAccCols;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % n_stages;
           const uint32_t ph = (it / n_stages) & 1;
           if (!mbar_wait(&full_bar[s], ph, p.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
+          if (it < 256) DG_PROBE_STAMP(256 + it);             // data landed
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
           const uint64_t ad = sdesc_sw128(a_addr), bd = sdesc_sw128(a_addr + C::kABytes);
@@ -374,6 +387,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const int buf = local & 1;
       const bool ok =
           __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, DGDEV_TIMEOUT_EPI));
+      if (threadIdx.x == 64 && local < 64) DG_PROBE_STAMP(576 + local);   // accumulator complete
       tc_fence_after();
       if (p.act && p.k_splits == 1) {
         // fused SwiGLU: accumulator rows 0..63 are gate rows of SwiGLU outputs
@@ -433,6 +447,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         for (int n = 0; n < n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
       }
       tc_fence_before();
+      if (threadIdx.x == 64 && local < 64) DG_PROBE_STAMP(640 + local);   // epilogue done
       mbar_arrive(&acc_empty[buf]);
       if (!ok) break;
     }
