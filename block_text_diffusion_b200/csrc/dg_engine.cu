@@ -57,6 +57,13 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint3
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The four B-operand maps (boxes of 32, 64, 128, 256 rows) of a bf16 [rows][cols] matrix.
+bool bmaps(BMaps* b, const void* base, uint64_t rows, uint64_t cols) {
+  bool ok = true;
+  for (int i = 0; i < 4; ++i) ok &= map2d(&b->m[i], base, rows, cols, 32u << i);
+  return ok;
+}
+
 // 3D bf16 map; strides in bytes of dims 1 and 2.
 bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
            uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
@@ -144,7 +151,7 @@ struct dg_model {
 
   void *h = nullptr, *x = nullptr, *q = nullptr, *o = nullptr, *xp = nullptr, *act = nullptr;
   void *probs = nullptr, *u = nullptr, *sc = nullptr;
-  CUtensorMap tm_x, tm_o, tm_xp, tm_act, tm_probs, tm_u;
+  BMaps tm_x, tm_o, tm_xp, tm_act, tm_probs, tm_u;   // activation (B) operands
   float* ws = nullptr;
   float *o_part = nullptr, *lse_part = nullptr;
   int *ids = nullptr, *perm = nullptr, *inv = nullptr, *work_count = nullptr, *counts = nullptr;
@@ -261,7 +268,7 @@ struct LaunchScope {
 // ---------------------------------------------------------------------------
 struct GemmCall {
   const CUtensorMap* tA = nullptr;   // bf16 path
-  const CUtensorMap* tB = nullptr;
+  const BMaps* tB = nullptr;
   const float* A32 = nullptr;        // fp32 path
   const float* B32 = nullptr;
   long long lda = 0, ldb = 0;
@@ -475,12 +482,12 @@ dg_status build_maps(dg_model* m) {
     ok &= map2d(&w.tm_wr, w.wr, (uint64_t)m->E, d, 128);
   }
   const uint64_t Tw = m->Tw, Tk = (uint64_t)m->Tw * m->k;
-  ok &= map2d(&m->tm_x, m->x, Tw, d, kBoxRowsB);
-  ok &= map2d(&m->tm_o, m->o, Tw, (uint64_t)m->hq * m->hd, kBoxRowsB);
-  ok &= map2d(&m->tm_xp, m->xp, Tk, d, kBoxRowsB);
-  ok &= map2d(&m->tm_act, m->act, Tk, m->ff, kBoxRowsB);
-  ok &= map2d(&m->tm_probs, m->probs, m->T_cap, V, kBoxRowsB);
-  ok &= map2d(&m->tm_u, m->u, m->T_cap, d, kBoxRowsB);
+  ok &= bmaps(&m->tm_x, m->x, Tw, d);
+  ok &= bmaps(&m->tm_o, m->o, Tw, (uint64_t)m->hq * m->hd);
+  ok &= bmaps(&m->tm_xp, m->xp, Tk, d);
+  ok &= bmaps(&m->tm_act, m->act, Tk, m->ff);
+  ok &= bmaps(&m->tm_probs, m->probs, m->T_cap, V);
+  ok &= bmaps(&m->tm_u, m->u, m->T_cap, d);
   return ok ? DG_OK : DG_ERR_CUDA;
 }
 
@@ -617,7 +624,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
         attr = true;
       }
       RouterArgs ra{m->E, m->k, Tn, cdiv(d, 64), m->rbias, m->ids, m->gate, &m->st->err};
-      launch_pdl(k_router_tc, cdiv(Tn, kRouterBN) * kRouterSplits, 128, kRouterSmem, s, w.tm_wr, m->tm_x, ra);
+      launch_pdl(k_router_tc, cdiv(Tn, kRouterBN) * kRouterSplits, 128, kRouterSmem, s, w.tm_wr, m->tm_x.m[0], ra);
       CU_TRY(cudaGetLastError());
     } else {
     GemmCall rc;

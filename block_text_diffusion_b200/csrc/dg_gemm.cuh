@@ -82,7 +82,59 @@ __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& k
 // 128-row accumulators that share every B tile (M tile 256): for the big
 // vocabulary GEMMs this halves how often the activations stream from L2.
 // ---------------------------------------------------------------------------
-constexpr int kBoxRowsB = 32;
+constexpr int kBoxRowsB = 32;   // B rows are loaded in multiples of 32
+
+// Epilogue of one accumulator row (this thread's TMEM lane) of n_mma columns:
+// out[c * ldo] = alpha * acc[c] for c < n_valid.  TMEM loads are issued four
+// at a time (64 columns) before one wait.  Warp-collective: n_mma uniform.
+__device__ __forceinline__ void epilogue_store(uint32_t taddr, int n_mma, int n_valid, bool m_ok, float* outp,
+                                               long long ldo, float alpha) {
+  for (int c0 = 0; c0 < n_mma; c0 += 64) {
+    uint32_t v[4][16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (c0 + q * 16 < n_mma) tmem_ld16_nw(taddr + c0 + q * 16, v[q]);
+    tmem_wait_ld();
+    if (m_ok) {
+      float* o = outp + (long long)c0 * ldo;
+      if (c0 + 64 <= n_valid) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[(long long)(q * 16 + j) * ldo] = __uint_as_float(v[q][j]) * alpha;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + q * 16 + j < n_valid) o[(long long)(q * 16 + j) * ldo] = __uint_as_float(v[q][j]) * alpha;
+      }
+    }
+  }
+}
+
+// Tensor maps of one B operand with boxes of 32, 64, 128 and 256 rows: a tile
+// of n rows is fetched with the fewest boxes (greedy, largest first), since
+// every TMA box costs a fixed issue overhead (measured: 8 boxes of 32 rows per
+// k-block made a 256-row tile 50% slower than one box of 256).
+struct BMaps {
+  CUtensorMap m[4];   // box rows 32 << i
+};
+
+// Loads rows [row0, row0 + n_load) (n_load a multiple of 32, <= 256) of K
+// block x into dst (rows contiguous, 128 B each) on barrier bar.
+__device__ __forceinline__ void tma_load_b_rows(uint8_t* dst, const BMaps* bm, int x, int row0, int n_load,
+                                                uint64_t* bar) {
+  int r = 0;
+#pragma unroll 1
+  for (int i = 3; i >= 0; --i) {
+    const int box = 32 << i;
+    while (n_load - r >= box) {
+      tma_load_2d(dst + r * 128, &bm->m[i], x, row0 + r, bar);
+      r += box;
+    }
+  }
+}
 
 template <int BN, int STAGES, int MT = 1>
 struct GemmTcCfg {
@@ -95,7 +147,7 @@ struct GemmTcCfg {
 
 template <int BN, int STAGES, int MT = 1>
 __global__ void __launch_bounds__(128, 1)
-k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
           GemmArgs p) {
   using C = GemmTcCfg<BN, STAGES, MT>;
   static_assert(MT * C::kTmemCols <= 512, "tensor memory holds 512 columns");
@@ -128,7 +180,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
+    for (int i = 0; i < 4; ++i) prefetch_tmap(&tmB.m[i]);
   }
   if (warp == 0) tmem_alloc(&tmem_base, MT * C::kTmemCols);
   tc_fence_before();
@@ -169,8 +221,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           for (int mt = 0; mt < MT; ++mt)
             tma_load_2d(a_s + mt * 16384, &tmA, kx, t.a_row0 + m0 + mt * 128, &full_bar[s]);
         }
-        for (int j = 0; j < n_boxes; ++j)
-          tma_load_2d(b_s + j * kBoxRowsB * 128, &tmB, kx, t.b_row0 + j * kBoxRowsB, &full_bar[s]);
+        tma_load_b_rows(b_s, &tmB, kx, t.b_row0, n_boxes * kBoxRowsB, &full_bar[s]);
       }
     }
     __syncwarp();
@@ -209,15 +260,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const bool m_ok = (m0 + row) < p.M;
     float* outp = p.out + (long long)t.split * p.split_stride + (long long)t.out_row0 * p.ldo + m0 + row;
     if (ok && nkb > 0) {
-      for (int c0 = 0; c0 < n_mma; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + mt * C::kTmemCols + ((uint32_t)(warp * 32) << 16) + c0, v);
-        if (m_ok) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < t.n_valid) outp[(long long)(c0 + j) * p.ldo] = v[j] * p.alpha;
-        }
-      }
+      epilogue_store(tmem + mt * C::kTmemCols + ((uint32_t)(warp * 32) << 16), n_mma, t.n_valid, m_ok, outp,
+                     p.ldo, p.alpha);
     } else if (nkb == 0 && ok && m_ok) {
       for (int n = 0; n < t.n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
     }
@@ -242,7 +286,7 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
-k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                      GemmArgs p_in, int items_dense) {
   using C = GemmTcCfg<BN, STAGES>;
   constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
@@ -267,7 +311,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     fence_mbar_init();
     prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
+    for (int i = 0; i < 4; ++i) prefetch_tmap(&tmB.m[i]);
     s_epi_fail = 0;
   }
   if (warp == 0) tmem_alloc(&tmem_base, kAllocCols);
@@ -321,8 +365,7 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
           uint8_t* b_s = a_s + C::kABytes;
           mbar_expect_tx(&full_bar[s], tx);
           tma_load_2d(a_s, &tmA, kb * 64, t.a_row0 + t.m_tile * 128, &full_bar[s]);
-          for (int j = 0; j < n_boxes; ++j)
-            tma_load_2d(b_s + j * kBoxRowsB * 128, &tmB, kb * 64, t.b_row0 + j * kBoxRowsB, &full_bar[s]);
+          tma_load_b_rows(b_s, &tmB, kb * 64, t.b_row0, n_boxes * kBoxRowsB, &full_bar[s]);
         }
       }
     }
@@ -434,15 +477,8 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const bool m_ok = (m0 + row) < p.M;
       float* outp = p.out + (long long)split * p.split_stride + (long long)out_row0 * p.ldo + m0 + row;
       if (ok && kb1 > kb0) {
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
-          float v[16];
-          tmem_ld16(tmem + buf * kAccCols + ((uint32_t)(quad * 32) << 16) + c0, v);
-          if (m_ok) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (c0 + j < n_valid) outp[(long long)(c0 + j) * p.ldo] = v[j] * p.alpha;
-          }
-        }
+        epilogue_store(tmem + buf * kAccCols + ((uint32_t)(quad * 32) << 16), n_mma, n_valid, m_ok, outp, p.ldo,
+                       p.alpha);
       } else if (ok && m_ok) {
         for (int n = 0; n < n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
       }

@@ -92,9 +92,11 @@ extern "C" dg_status dg_gemm_splitk_noalloc(const void* A, const void* B, float*
   dg_status st = device_arrays(&scratch, &err);
   if (st != DG_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  CUtensorMap ta, tb;
-  if (!tensor_map(&ta, A, (uint64_t)M, (uint64_t)K, 128) || !tensor_map(&tb, B, (uint64_t)N, (uint64_t)K, kBoxRowsB))
-    return DG_ERR_CUDA;
+  CUtensorMap ta;
+  BMaps tb;
+  bool maps_ok = tensor_map(&ta, A, (uint64_t)M, (uint64_t)K, 128);
+  for (int i = 0; i < 4; ++i) maps_ok = maps_ok && tensor_map(&tb.m[i], B, (uint64_t)N, (uint64_t)K, 32u << i);
+  if (!maps_ok) return DG_ERR_CUDA;
   using C = GemmTcCfg<kBN, kStages>;
   if (cudaFuncSetAttribute(k_gemm_tc<kBN, kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
       cudaSuccess)
