@@ -253,11 +253,11 @@ def test_router(x, wr, ids, gate, bias=None, stream=None):
 
 
 def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, sized_ring=False, swiglu=False,
-                      stream=None):
+                      m256=False, stream=None):
     import torch
     K = A.shape[-1]
     c = (ctypes.c_int32 * groups)(*[int(x) for x in counts])
-    flags = int(persistent) | (2 if sized_ring else 0) | (4 if swiglu else 0)
+    flags = int(persistent) | (2 if sized_ring else 0) | (4 if swiglu else 0) | (8 if m256 else 0)
     _check(lib().dg_test_grouped_gemm(_ptr(A), _ptr(B), c, groups, M, K, 1 if A.dtype == torch.bfloat16 else 0,
                                       bn, flags, _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
 

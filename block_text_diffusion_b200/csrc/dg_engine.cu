@@ -307,12 +307,12 @@ dg_status launch_tc(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   return DG_OK;
 }
 
-template <int BN, int ST>
+template <int BN, int ST, int MT = 1>
 dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
-  using C = GemmTcCfg<BN, ST>;
+  using C = GemmTcCfg<BN, ST, MT>;
   static bool attr = false;
   if (!attr) {
-    CU_TRY(cudaFuncSetAttribute(k_gemm_tc_persistent<BN, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CU_TRY(cudaFuncSetAttribute(k_gemm_tc_persistent<BN, ST, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::kSmem));
     attr = true;
   }
@@ -322,7 +322,7 @@ dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   // CTAs per SM allowed by shared memory (228 KB per SM)
   const int per_sm = std::max(1, (228 * 1024) / (C::kSmem + 2048));
   const int grid = (int)std::min<long long>(max_tiles, (long long)kSMs * std::min(per_sm, 2));
-  launch_pdl(k_gemm_tc_persistent<BN, ST>, grid, 192, C::kSmem, s, *g.tA, *g.tB, a, items_dense);
+  launch_pdl(k_gemm_tc_persistent<BN, ST, MT>, grid, 192, C::kSmem, s, *g.tA, *g.tB, a, items_dense);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -359,6 +359,10 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   a.m_tiles = cdiv(g.M, 128);
   a.n_tile = g.bn;
   if (g.persistent) {
+    if (g.m256 && g.bn == 256) {   // 256-row tiles: two accumulators share each B tile
+      a.m_tiles = cdiv(g.M, 256);
+      return launch_tc_persistent<256, 3, 2>(g, a, s);
+    }
     switch (g.bn) {
       case 256: return launch_tc_persistent<256, 4>(g, a, s);
       case 128: return launch_tc_persistent<128, 6>(g, a, s);
@@ -647,8 +651,10 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     // (bf16 persistent path only; the fp32 path keeps one split)
     const long long gu_stride = (long long)n_pairs * 2 * m->ff, dn_stride = (long long)n_pairs * d;
     SplitPlan plan{};
-    plan.mt[0] = cdiv(2 * m->ff, 128); plan.kb[0] = cdiv(d, 64);
-    plan.mt[1] = cdiv(d, 128); plan.kb[1] = cdiv(m->ff, 64);
+    // bf16 expert GEMMs run 256-row tiles (two accumulators per CTA share each B tile)
+    const int m_rows = m->bf ? 256 : 128;
+    plan.mt[0] = cdiv(2 * m->ff, m_rows); plan.kb[0] = cdiv(d, 64);
+    plan.mt[1] = cdiv(d, m_rows); plan.kb[1] = cdiv(m->ff, 64);
     plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
     plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
     plan.fused0 = m->bf ? 1 : 0;
@@ -668,7 +674,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     gu.splits = m->bf ? 8 : 1;
     // bf16: an unsplit gate|up GEMM applies SwiGLU in its epilogue
-    if (m->bf) { gu.act = m->act; gu.act_ld = m->ff; }
+    if (m->bf) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = true; }
     DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
     { LaunchScope ls(m, s, PH_SWIGLU);
       const long long n = (long long)n_pairs * m->ff;
@@ -681,6 +687,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.max_items = max_items; dn.bn = bn_g; dn.persistent = m->bf;
     dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
     dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
+    dn.m256 = m->bf;
     dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);

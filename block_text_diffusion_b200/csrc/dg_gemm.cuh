@@ -284,13 +284,19 @@ constexpr int kWorkSmem = 512;   // work items staged in shared memory (more are
 // Barrier among the four epilogue warps (threads 64..191) of the persistent kernel.
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MT = 1>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                      GemmArgs p_in, int items_dense) {
-  using C = GemmTcCfg<BN, STAGES>;
-  constexpr int kAccCols = C::kTmemCols;               // one accumulator buffer
-  constexpr int kAllocCols = 2 * kAccCols;             // two buffers (<= 512)
+  using C = GemmTcCfg<BN, STAGES, MT>;
+  constexpr int kAccCols = C::kTmemCols;               // one 128-row accumulator
+  // MT = 1: two accumulator buffers (the epilogue of one tile overlaps the
+  // next tile's mainloop).  MT = 2: one buffer of two accumulators (a 256-row
+  // tile: every B tile feeds twice the MMA work).
+  constexpr int kNBuf = MT == 1 ? 2 : 1;
+  constexpr int kAllocCols = kNBuf * MT * kAccCols;
+  static_assert(kAllocCols <= 512, "tensor memory holds 512 columns");
+  constexpr int kTileRows = 128 * MT;
   // The ring holds STAGES full-size stages; when every work item has fewer
   // rows than BN, stages shrink to A + the rows actually loaded and the ring
   // holds more of them (more weight bytes in flight per SM).
@@ -334,6 +340,9 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  // 128-row halves of tile m_t that hold rows below M (the last tile of an
+  // odd number of halves loads and multiplies only its first half)
+  auto halves = [&](int m_t) { return MT == 1 ? 1 : min(MT, (p.M - m_t * kTileRows + 127) / 128); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -354,8 +363,9 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
         int kb0, kb1;
         split_range(p, t.split, kb0, kb1);
+        const int nh = halves(t.m_tile);
         const int n_boxes = (min(BN, (t.n_valid + 15) & ~15) + kBoxRowsB - 1) / kBoxRowsB;
-        const uint32_t tx = C::kABytes + n_boxes * kBoxRowsB * 128;
+        const uint32_t tx = nh * 16384 + n_boxes * kBoxRowsB * 128;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % n_stages;
           const uint32_t ph = (it / n_stages) & 1;
@@ -364,7 +374,8 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
           uint8_t* a_s = smem + s * stage_bytes;
           uint8_t* b_s = a_s + C::kABytes;
           mbar_expect_tx(&full_bar[s], tx);
-          tma_load_2d(a_s, &tmA, kb * 64, t.a_row0 + t.m_tile * 128, &full_bar[s]);
+          for (int h = 0; h < nh; ++h)
+            tma_load_2d(a_s + h * 16384, &tmA, kb * 64, t.a_row0 + t.m_tile * kTileRows + h * 128, &full_bar[s]);
           tma_load_b_rows(b_s, &tmB, kb * 64, t.b_row0, n_boxes * kBoxRowsB, &full_bar[s]);
         }
       }
@@ -380,20 +391,21 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int split = r % p.k_splits;
         const int item = r / p.k_splits;
         const int n_valid = p.work ? work[item].z : min(p.n_tile, p.N - item * p.n_tile);
-        (void)m_t;
+        const int nh = halves(m_t);
         int kb0, kb1;
         split_range(p, split, kb0, kb1);
         const int n_mma = min(BN, (n_valid + 15) & ~15);
         const uint32_t idesc = idesc_bf16(128, n_mma);
-        const int buf = local & 1;
-        // wait until the epilogue drained this buffer (use 2 tiles ago)
-        if (local >= 2 && !mbar_wait(&acc_empty[buf], ((local >> 1) & 1) ^ 1, p.err, DGDEV_TIMEOUT_MMA)) {
+        const int buf = local % kNBuf;
+        // wait until the epilogue drained this buffer (kNBuf tiles ago)
+        if (local >= kNBuf &&
+            !mbar_wait(&acc_empty[buf], ((local / kNBuf) & 1) ^ 1, p.err, DGDEV_TIMEOUT_MMA)) {
           ok = false;
           break;
         }
         if (local < 64) DG_PROBE_STAMP(512 + local);          // accumulator free
         tc_fence_after();
-        const uint32_t d_tmem = tmem + buf * kAccCols;
+        const uint32_t d_tmem = tmem + buf * MT * kAccCols;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % n_stages;
           const uint32_t ph = (it / n_stages) & 1;
@@ -401,10 +413,14 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
           if (it < 256) DG_PROBE_STAMP(256 + it);             // data landed
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
-          const uint64_t ad = sdesc_sw128(a_addr), bd = sdesc_sw128(a_addr + C::kABytes);
+          const uint64_t bd = sdesc_sw128(a_addr + C::kABytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < MT; ++h)
+              if (h < nh)
+                tc_mma_bf16(d_tmem + h * kAccCols, sdesc_sw128(a_addr + h * 16384) + 2 * kk, bd + 2 * kk, idesc,
+                            (kb > kb0 || kk > 0) ? 1u : 0u);
           tc_commit(&empty_bar[s]);
         }
         tc_commit(&acc_full[buf]);
@@ -427,60 +443,68 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int kb0, kb1;
       split_range(p, split, kb0, kb1);
       const int n_mma = min(BN, (n_valid + 15) & ~15);
-      const int buf = local & 1;
+      const int nh = halves(m_t);
+      const int buf = local % kNBuf;
       const bool ok =
-          __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, DGDEV_TIMEOUT_EPI));
+          __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local / kNBuf) & 1, p.err, DGDEV_TIMEOUT_EPI));
       if (threadIdx.x == 64 && local < 64) DG_PROBE_STAMP(576 + local);   // accumulator complete
       tc_fence_after();
       if (p.act && p.k_splits == 1) {
-        // fused SwiGLU: accumulator rows 0..63 are gate rows of SwiGLU outputs
-        // f = 64 m_t .. 64 m_t + 63, rows 64..127 the matching up rows.  The up
-        // quads hand their values to the gate quads through shared memory.
-        // The four warps first agree on the wait outcome (they share barriers).
+        // fused SwiGLU: in each 128-row half, rows 0..63 are gate rows of SwiGLU
+        // outputs f = 64 (half index) .. + 63 and rows 64..127 the matching up
+        // rows.  The up quads hand their values to the gate quads through shared
+        // memory.  The four warps first agree on the wait outcome (they share
+        // barriers).
         if (lane == 0 && !ok) s_epi_fail = 1;
         epi_sync();
         const bool ok_all = s_epi_fail == 0;
         bf16* act = reinterpret_cast<bf16*>(p.act);
-        const int f = m_t * 64 + (quad & 1) * 32 + lane;
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
-          uint32_t v[16];
-          if (ok_all && kb1 > kb0) {
-            tmem_ld16_nw(tmem + buf * kAccCols + ((uint32_t)(quad * 32) << 16) + c0, v);
-            tmem_wait_ld();
-          } else {
+        for (int h = 0; h < nh; ++h) {
+          const int f = (m_t * MT + h) * 64 + (quad & 1) * 32 + lane;
+          const uint32_t tbase = tmem + (buf * MT + h) * kAccCols + ((uint32_t)(quad * 32) << 16);
+          for (int c0 = 0; c0 < n_mma; c0 += 16) {
+            uint32_t v[16];
+            if (ok_all && kb1 > kb0) {
+              tmem_ld16_nw(tbase + c0, v);
+              tmem_wait_ld();
+            } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0u;
-          }
-          if (quad >= 2) {
+              for (int j = 0; j < 16; ++j) v[j] = 0u;
+            }
+            if (quad >= 2) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) s_xfer[((quad - 2) * 32 + lane) * 17 + j] = __uint_as_float(v[j]);
-          }
-          epi_sync();
-          if (quad < 2) {
+              for (int j = 0; j < 16; ++j) s_xfer[((quad - 2) * 32 + lane) * 17 + j] = __uint_as_float(v[j]);
+            }
+            epi_sync();
+            if (quad < 2) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (c0 + j < n_valid) {
-                const float g = __uint_as_float(v[j]);
-                const float u = s_xfer[(quad * 32 + lane) * 17 + j];
-                act[(long long)(out_row0 + c0 + j) * p.act_ld + f] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+              for (int j = 0; j < 16; ++j) {
+                if (c0 + j < n_valid) {
+                  const float g = __uint_as_float(v[j]);
+                  const float u = s_xfer[(quad * 32 + lane) * 17 + j];
+                  act[(long long)(out_row0 + c0 + j) * p.act_ld + f] =
+                      __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+                }
               }
             }
+            epi_sync();
           }
-          epi_sync();
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);
         if (!ok_all) break;
         continue;
       }
-      const int m0 = m_t * 128;
-      const bool m_ok = (m0 + row) < p.M;
-      float* outp = p.out + (long long)split * p.split_stride + (long long)out_row0 * p.ldo + m0 + row;
-      if (ok && kb1 > kb0) {
-        epilogue_store(tmem + buf * kAccCols + ((uint32_t)(quad * 32) << 16), n_mma, n_valid, m_ok, outp, p.ldo,
-                       p.alpha);
-      } else if (ok && m_ok) {
-        for (int n = 0; n < n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
+      for (int h = 0; h < nh; ++h) {
+        const int m0 = m_t * kTileRows + h * 128;
+        const bool m_ok = (m0 + row) < p.M;
+        float* outp = p.out + (long long)split * p.split_stride + (long long)out_row0 * p.ldo + m0 + row;
+        if (ok && kb1 > kb0) {
+          epilogue_store(tmem + (buf * MT + h) * kAccCols + ((uint32_t)(quad * 32) << 16), n_mma, n_valid, m_ok,
+                         outp, p.ldo, p.alpha);
+        } else if (ok && m_ok) {
+          for (int n = 0; n < n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
+        }
       }
       tc_fence_before();
       if (threadIdx.x == 64 && local < 64) DG_PROBE_STAMP(640 + local);   // epilogue done

@@ -541,7 +541,8 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
       //   cost(s) = ceil(mt * nw * s / SMs) / s + s * r,
       //   r = partial bytes / weight bytes = (n_pairs * 4) / (nw * K * 2) * 2.
       for (int g = 0; g < 2; ++g) {
-        const float r = 4.0f * (float)n_pairs / ((float)max(1, nw) * (float)(plan.kb[g] * 64));
+        // partial slabs mostly stay in L2: charged at half the weight-stream rate
+        const float r = 2.0f * (float)n_pairs / ((float)max(1, nw) * (float)(plan.kb[g] * 64));
         const int s_max = max(1, min(plan.cap[g], plan.kb[g] / 4));
         int best = 1;
         float best_cost = 3.4e38f;

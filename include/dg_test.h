@@ -71,7 +71,8 @@ dg_status dg_test_router(const void* x, const void* wr, const float* bias, int32
  * bit 1 (persistent only) sizes the ring stages from the largest item, bit 2
  * (persistent, bf16, M % 128 == 0) applies SwiGLU in the epilogue: A rows
  * interleave gate / up in blocks of 64 and out receives bf16 [rows][M/2],
- * out[r][f] = round(silu(g) u) with g, u the rows 128 (f/64) + f%64 (+64).
+ * out[r][f] = round(silu(g) u) with g, u the rows 128 (f/64) + f%64 (+64);
+ * bit 3 (persistent, bn 256) uses 256-row tiles (two accumulators per CTA).
  * Allocates. */
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
                                int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);

@@ -255,7 +255,7 @@ def test_gemm_f32():
     (1024, 256, [0, 9, 64, 65, 1], 64, False),
     (1408, 2816, [17, 3, 0, 31, 12, 1, 9, 20], 256, True),
 ])
-@pytest.mark.parametrize("persistent", [False, True, "sized_ring"])
+@pytest.mark.parametrize("persistent", [False, True, "sized_ring", "m256"])
 def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     g = np.random.default_rng(sum(counts) + M)
     G = len(counts)
@@ -269,8 +269,11 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     out = torch.full((rows, M), float("nan"), dtype=torch.float32, device="cuda")
     # "sized_ring": the persistent kernel's ring stages shrink to the largest
     # item (more stages in flight), as the expert GEMMs run in the step
+    # "m256": 256-row tiles (two accumulators), as the expert GEMMs run, with the
+    # ring sized from the largest item
     dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn, persistent=bool(persistent) and bf,
-                         sized_ring=persistent == "sized_ring" and bf)
+                         sized_ring=persistent in ("sized_ring", "m256") and bf,
+                         m256=persistent == "m256" and bf and bn == 256)
     got = host(out).astype(np.float64)
     r0 = 0
     for e, c in enumerate(counts):
@@ -282,7 +285,8 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
 
 
 @pytest.mark.parametrize("M,K,counts", [(1408, 2816, [17, 3, 0, 200, 12, 1, 256, 20]), (2048, 1024, [64, 65, 0, 9])])
-def test_grouped_gemm_fused_swiglu(M, K, counts):
+@pytest.mark.parametrize("m256", [False, True])
+def test_grouped_gemm_fused_swiglu(M, K, counts, m256):
     # the unsplit gate|up GEMM writes round(silu(g) u) itself; A rows interleave
     # gate / up in blocks of 64
     g = np.random.default_rng(M + K + sum(counts))
@@ -291,7 +295,7 @@ def test_grouped_gemm_fused_swiglu(M, K, counts):
     B = I._bf16_grid(g.standard_normal((rows, K)).astype(F32))
     out = torch.zeros((rows, M), dtype=torch.float32, device="cuda")
     dg.test_grouped_gemm(bf16_tensor(A), bf16_tensor(B), counts, G, M, out, bn=256, persistent=True,
-                         sized_ring=True, swiglu=True)
+                         sized_ring=True, swiglu=True, m256=m256)
     act = out.view(torch.bfloat16).reshape(-1)[:rows * ff].reshape(rows, ff)
     got = act.float().cpu().numpy().astype(np.float64)
     f = np.arange(ff)
