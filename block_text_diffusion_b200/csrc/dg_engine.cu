@@ -651,10 +651,11 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     // (bf16 persistent path only; the fp32 path keeps one split)
     const long long gu_stride = (long long)n_pairs * 2 * m->ff, dn_stride = (long long)n_pairs * d;
     SplitPlan plan{};
-    // bf16 expert GEMMs run 256-row tiles (two accumulators per CTA share each B tile)
-    const int m_rows = m->bf ? 256 : 128;
-    plan.mt[0] = cdiv(2 * m->ff, m_rows); plan.kb[0] = cdiv(d, 64);
-    plan.mt[1] = cdiv(d, m_rows); plan.kb[1] = cdiv(m->ff, 64);
+    // bf16 gate|up runs 256-row tiles (two accumulators per CTA share each B
+    // tile; its long K amortises the unoverlapped epilogue); down keeps
+    // 128-row tiles with double-buffered accumulators (K = ff is short)
+    plan.mt[0] = cdiv(2 * m->ff, m->bf ? 256 : 128); plan.kb[0] = cdiv(d, 64);
+    plan.mt[1] = cdiv(d, 128); plan.kb[1] = cdiv(m->ff, 64);
     plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
     plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
     plan.fused0 = m->bf ? 1 : 0;
@@ -687,7 +688,6 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.max_items = max_items; dn.bn = bn_g; dn.persistent = m->bf;
     dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
     dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
-    dn.m256 = m->bf;
     dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);

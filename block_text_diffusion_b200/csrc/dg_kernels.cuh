@@ -539,10 +539,10 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
       // adds one fp32 partial slab (written, then read by the consumer).  In
       // units of the time to stream the group's weights once:
       //   cost(s) = ceil(mt * nw * s / SMs) / s + s * r,
-      //   r = partial bytes / weight bytes = (n_pairs * 4) / (nw * K * 2) * 2.
+      //   r = partial bytes (written and read) / weight bytes / 4.
       for (int g = 0; g < 2; ++g) {
-        // partial slabs mostly stay in L2: charged at half the weight-stream rate
-        const float r = 2.0f * (float)n_pairs / ((float)max(1, nw) * (float)(plan.kb[g] * 64));
+        // partial slabs mostly stay in L2: charged at a quarter of the weight-stream rate
+        const float r = (float)n_pairs / ((float)max(1, nw) * (float)(plan.kb[g] * 64));
         const int s_max = max(1, min(plan.cap[g], plan.kb[g] / 4));
         int best = 1;
         float best_cost = 3.4e38f;
