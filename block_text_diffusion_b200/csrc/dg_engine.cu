@@ -288,6 +288,8 @@ struct GemmCall {
   void* act = nullptr;               // persistent gate|up: SwiGLU output (bf16) when the GEMM runs unsplit
   int act_ld = 0;
   bool m256 = false;                 // dense, bn 256: 256-row M tiles (two accumulators share B)
+  int qkv_on = 0;                    // dense bf16, one split: fused QKV post-process
+  QkvEpi qkv{};
 };
 
 template <int BN, int ST, int MT = 1>
@@ -344,6 +346,8 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   a.k_splits_dev = g.persistent ? g.k_splits_dev : nullptr;
   a.max_rows_dev = g.persistent ? g.max_rows_dev : nullptr;
   a.act = g.persistent ? g.act : nullptr;
+  a.qkv_on = g.qkv_on;
+  a.qkv = g.qkv;
   a.act_ld = g.act_ld;
   a.err = &m->st->err;
   if (!m->bf) {
@@ -391,6 +395,11 @@ int pick_splits(int m_tiles, int n_items, int kb_total, int cap) {
   s = std::min(s, std::max(1, kb_total / 4));
   return std::min(s, cap);
 }
+
+// Threads of a one-row-per-CTA kernel over d values in float4 groups: one
+// group per thread (whole warps, at most 1024), so every load of the row is in
+// flight at once.
+int row_threads(int d) { return std::min(1024, std::max(32, ((d / 4 + 31) / 32) * 32)); }
 
 // A tuned token tile (32, 64, 128 or 256) in place of the default one.
 int tuned_bn(int def, int want) {
@@ -560,8 +569,15 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       while (qc.splits > 1 && (size_t)qc.splits * Tn * m->nqkv > m->ws_elems) --qc.splits;
       qc.split_stride = (long long)Tn * m->nqkv;
     }
+    // bf16: one split and the RoPE / cache scatter in the GEMM epilogue
+    const bool fuse_qkv = m->bf && m->hd == 128 && m->tune.dense_splits == 0;
+    if (fuse_qkv) {
+      qc.splits = 1;
+      qc.qkv_on = 1;
+      qc.qkv = QkvEpi{(bf16*)m->q, (bf16*)g.K, (bf16*)g.Vt, m->rope, m->hq, m->hkv, n_per, pos0, b0, g.B, l, g.S};
+    }
     DG_TRY(gemm(m, qc, PH_QKV_GEMM, s));
-    {
+    if (!fuse_qkv) {
       LaunchScope ls(m, s, PH_QKV_POST);
       QkvPostArgs qa;
       qa.ws = m->ws; qa.split_stride = qc.split_stride; qa.splits = std::min(qc.splits, cdiv(d, 64));
@@ -613,7 +629,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     }
     DG_TRY(gemm(m, oc, PH_O_GEMM, s));
     { LaunchScope ls(m, s, PH_RESIDUAL);
-      launch_pdl(k_residual_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, oc.split_stride,
+      launch_pdl(k_residual_norm<T>, Tn, row_threads(d), 0, s, (T*)m->h, (T*)m->x, m->ws, oc.split_stride,
                                             std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
     if (m->dbg_h)
       launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
@@ -691,7 +707,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
-      launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
+      launch_pdl(k_moe_combine_norm<T>, Tn, row_threads(d), 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
                                                m->c.rms_eps, m->moe_splits + 1, dn_stride); }
     if (m->dbg_h) {
       launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l + 1) * Tn * d,
@@ -1034,11 +1050,13 @@ size_t dg_kv_bytes(const dg_model* m, int32_t B, int32_t P) {
 int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   if (!m) return 0;
   (void)B; (void)P;
-  // per layer: qkv gemm, qkv post, attention, attention combine, o gemm,
-  // residual+norm, router gemm, router top-k, permute, gather, gate/up gemm,
-  // swiglu, down gemm, combine+norm; then embed+norm, lm head, sampler,
-  // commit, 4 self-cond.
-  return 14 * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
+  // per layer: qkv gemm (bf16: with the RoPE / cache scatter; fp32: + qkv
+  // post), attention, attention combine, o gemm, residual+norm, router (bf16:
+  // one kernel; fp32: gemm + top-k), permute, gather, gate/up gemm, swiglu,
+  // down gemm, combine+norm; then embed+norm, lm head, sampler, commit,
+  // 4 self-cond.
+  const int per_layer = m->bf ? 12 : 14;
+  return per_layer * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          4 /*self-conditioning*/;
 }
 

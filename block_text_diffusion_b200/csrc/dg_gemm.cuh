@@ -23,6 +23,21 @@ __device__ long long g_probe[1024];
 #define DG_PROBE_STAMP(i) do { } while (0)
 #endif
 
+// Fused QKV post-process for the dense bf16 GEMM (head_dim 128, one split):
+// each 128-row tile of the fused QKV weight is one head; q and k heads get
+// rotate-half RoPE at their positions, q goes to Q [t][Hq][128], k into the
+// K cache [lbh][pos][128], v transposed into the V^T cache [lbh][128][pos].
+struct QkvEpi {
+  bf16* q;
+  bf16* kc;
+  bf16* vt;
+  const float2* rope;   // [pos][64] (cos, sin)
+  int Hq, Hkv;
+  int n_per;            // tokens per canvas in the launch
+  int pos0;             // position of a canvas's first token
+  int b0, B, layer, S;  // first canvas, canvases in the cache, layer, key slot stride
+};
+
 struct GemmArgs {
   int M;                   // valid A rows per work item
   int m_tiles;             // ceil(M / tile M)
@@ -39,6 +54,8 @@ struct GemmArgs {
   const int* work_count;
   const int* k_splits_dev; // persistent kernel: split-K factor chosen on the device (overrides k_splits)
   const int* max_rows_dev; // persistent kernel: rows of the largest work item (sizes the ring stages)
+  int qkv_on;              // dense, one split, MT 1: fused QKV post-process (see QkvEpi)
+  QkvEpi qkv;
   void* act;               // persistent gate|up: when non-null and the split factor is 1, the
                            // epilogue writes round(silu(g) u) (bf16, row stride act_ld) instead
                            // of the fp32 output; A rows interleave gate / up in blocks of 64
@@ -109,6 +126,79 @@ __device__ __forceinline__ void epilogue_store(uint32_t taddr, int n_mma, int n_
           for (int j = 0; j < 16; ++j)
             if (c0 + q * 16 + j < n_valid) o[(long long)(q * 16 + j) * ldo] = __uint_as_float(v[q][j]) * alpha;
       }
+    }
+  }
+}
+
+// Fused QKV epilogue of one 128-row tile (head `head`) of the dense GEMM,
+// 128 threads (thread = channel c = TMEM lane).  RoPE pairs channels c and
+// c + 64: the upper-half threads pass their values to the lower half through
+// shared memory `xch` (64 x 65 floats; the pipeline ring, free after the
+// mainloop), and the lower half writes both outputs.  Tokens tok0 + j.
+__device__ __forceinline__ void qkv_epilogue(const QkvEpi& e, uint32_t taddr, int head, int tok0, int n_valid,
+                                             int n_mma, bool have, float* xch) {
+  const int c = threadIdx.x;   // 0..127
+  for (int c0 = 0; c0 < n_mma; c0 += 64) {
+    uint32_t v[4][16];
+    if (have) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (c0 + q * 16 < n_mma) tmem_ld16_nw(taddr + c0 + q * 16, v[q]);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[q][j] = 0u;
+    }
+    if (head < e.Hq + e.Hkv) {
+      if (c >= 64) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) xch[(c - 64) * 65 + q * 16 + j] = __uint_as_float(v[q][j]);
+      }
+      __syncthreads();
+      if (c < 64) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + q * 16 + j;
+            if (n < n_valid) {
+              const int t = tok0 + n;
+              const int b = e.b0 + t / e.n_per, pos = e.pos0 + t % e.n_per;
+              const float2 cs = e.rope[(long long)pos * 64 + c];
+              const float x0 = __uint_as_float(v[q][j]), x1 = xch[c * 65 + q * 16 + j];
+              const float y0 = x0 * cs.x - x1 * cs.y;
+              const float y1 = x0 * cs.y + x1 * cs.x;
+              bf16* dst;
+              if (head < e.Hq) {
+                dst = e.q + ((long long)t * e.Hq + head) * 128;
+              } else {
+                const long long lbh = ((long long)e.layer * e.B + b) * e.Hkv + (head - e.Hq);
+                dst = e.kc + (lbh * e.S + pos) * 128;
+              }
+              dst[c] = __float2bfloat16_rn(y0);
+              dst[c + 64] = __float2bfloat16_rn(y1);
+            }
+          }
+      }
+      __syncthreads();
+    } else {
+      const int g = head - e.Hq - e.Hkv;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c0 + q * 16 + j;
+          if (n < n_valid) {
+            const int t = tok0 + n;
+            const int b = e.b0 + t / e.n_per, pos = e.pos0 + t % e.n_per;
+            const long long lbh = ((long long)e.layer * e.B + b) * e.Hkv + g;
+            e.vt[(lbh * 128 + c) * e.S + pos] = __float2bfloat16_rn(__uint_as_float(v[q][j]));
+          }
+        }
     }
   }
 }
@@ -255,6 +345,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps
   // tcgen05.ld is warp-collective: agree on the wait outcome across the warp.
   const bool ok = __all_sync(0xffffffffu, mbar_wait(&done_bar, 0, p.err, DGDEV_TIMEOUT_EPI));
   tc_fence_after();
+  if (MT == 1 && p.qkv_on) {
+    qkv_epilogue(p.qkv, tmem + ((uint32_t)(warp * 32) << 16), t.m_tile, t.out_row0, t.n_valid, n_mma,
+                 ok && nkb > 0, reinterpret_cast<float*>(smem));
+  } else
   for (int mt = 0; mt < MT; ++mt) {
     const int row = mt * 128 + warp * 32 + lane;
     const bool m_ok = (m0 + row) < p.M;
