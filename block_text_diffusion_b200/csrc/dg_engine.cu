@@ -396,11 +396,6 @@ int pick_splits(int m_tiles, int n_items, int kb_total, int cap) {
   return std::min(s, cap);
 }
 
-// Threads of a one-row-per-CTA kernel over d values in float4 groups: one
-// group per thread (whole warps, at most 1024), so every load of the row is in
-// flight at once.
-int row_threads(int d) { return std::min(1024, std::max(32, ((d / 4 + 31) / 32) * 32)); }
-
 // A tuned token tile (32, 64, 128 or 256) in place of the default one.
 int tuned_bn(int def, int want) {
   if (want != 32 && want != 64 && want != 128 && want != 256) return def;
@@ -629,7 +624,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     }
     DG_TRY(gemm(m, oc, PH_O_GEMM, s));
     { LaunchScope ls(m, s, PH_RESIDUAL);
-      launch_pdl(k_residual_norm<T>, Tn, row_threads(d), 0, s, (T*)m->h, (T*)m->x, m->ws, oc.split_stride,
+      launch_pdl(k_residual_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, oc.split_stride,
                                             std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
     if (m->dbg_h)
       launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
@@ -707,7 +702,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.splits = m->bf ? 8 : 1;
     DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
-      launch_pdl(k_moe_combine_norm<T>, Tn, row_threads(d), 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
+      launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
                                                m->c.rms_eps, m->moe_splits + 1, dn_stride); }
     if (m->dbg_h) {
       launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l + 1) * Tn * d,

@@ -131,12 +131,20 @@ __device__ __forceinline__ void epilogue_store(uint32_t taddr, int n_mma, int n_
 }
 
 // Fused QKV epilogue of one 128-row tile (head `head`) of the dense GEMM,
-// 128 threads (thread = channel c = TMEM lane).  RoPE pairs channels c and
-// c + 64: the upper-half threads pass their values to the lower half through
-// shared memory `xch` (64 x 65 floats; the pipeline ring, free after the
-// mainloop), and the lower half writes both outputs.  Tokens tok0 + j.
+// 128 threads (thread = channel c = TMEM lane), up to 64 tokens per pass.
+// q / k heads: RoPE pairs channels c and c + 64; the upper-half threads pass
+// their values to the lower half through shared memory, the lower half
+// rotates and writes the bf16 head rows of the pass into a [token][channel]
+// staging tile, and all threads then copy whole 256-byte rows (16-byte
+// stores) to Q or the K cache.  v heads: each thread owns one V^T row and
+// writes its run of positions with 16-byte stores when the tokens are
+// consecutive positions of one canvas (scalar stores otherwise).
+// `xch` is the pipeline ring (free after the mainloop).
 __device__ __forceinline__ void qkv_epilogue(const QkvEpi& e, uint32_t taddr, int head, int tok0, int n_valid,
-                                             int n_mma, bool have, float* xch) {
+                                             int n_mma, bool have, uint8_t* xch_raw) {
+  float* xch = reinterpret_cast<float*>(xch_raw);                      // [64][65] fp32
+  bf16* st = reinterpret_cast<bf16*>(xch_raw + 64 * 65 * 4 + 256);     // [64][136] bf16
+  constexpr int kStPitch = 136;
   const int c = threadIdx.x;   // 0..127
   for (int c0 = 0; c0 < n_mma; c0 += 64) {
     uint32_t v[4][16];
@@ -151,6 +159,7 @@ __device__ __forceinline__ void qkv_epilogue(const QkvEpi& e, uint32_t taddr, in
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[q][j] = 0u;
     }
+    const int nt = min(64, n_valid - c0);   // tokens of this pass
     if (head < e.Hq + e.Hkv) {
       if (c >= 64) {
 #pragma unroll
@@ -160,45 +169,70 @@ __device__ __forceinline__ void qkv_epilogue(const QkvEpi& e, uint32_t taddr, in
       }
       __syncthreads();
       if (c < 64) {
+        const int t = tok0 + c0;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = c0 + q * 16 + j;
-            if (n < n_valid) {
-              const int t = tok0 + n;
-              const int b = e.b0 + t / e.n_per, pos = e.pos0 + t % e.n_per;
-              const float2 cs = e.rope[(long long)pos * 64 + c];
-              const float x0 = __uint_as_float(v[q][j]), x1 = xch[c * 65 + q * 16 + j];
-              const float y0 = x0 * cs.x - x1 * cs.y;
-              const float y1 = x0 * cs.y + x1 * cs.x;
-              bf16* dst;
-              if (head < e.Hq) {
-                dst = e.q + ((long long)t * e.Hq + head) * 128;
-              } else {
-                const long long lbh = ((long long)e.layer * e.B + b) * e.Hkv + (head - e.Hq);
-                dst = e.kc + (lbh * e.S + pos) * 128;
-              }
-              dst[c] = __float2bfloat16_rn(y0);
-              dst[c + 64] = __float2bfloat16_rn(y1);
+            const int n = q * 16 + j;
+            if (n < nt) {
+              const int pn = e.pos0 + (t + n) % e.n_per;
+              const float2 cs = e.rope[(long long)pn * 64 + c];
+              const float x0 = __uint_as_float(v[q][j]), x1 = xch[c * 65 + n];
+              st[n * kStPitch + c] = __float2bfloat16_rn(x0 * cs.x - x1 * cs.y);
+              st[n * kStPitch + c + 64] = __float2bfloat16_rn(x0 * cs.y + x1 * cs.x);
             }
           }
       }
       __syncthreads();
+      // copy: 16 threads per token row (16 x 16 B = 256 B)
+      for (int id = threadIdx.x; id < nt * 16; id += 128) {
+        const int n = id >> 4, part = id & 15;
+        const int t = tok0 + c0 + n;
+        const int b = e.b0 + t / e.n_per, pn = e.pos0 + t % e.n_per;
+        bf16* dst;
+        if (head < e.Hq) {
+          dst = e.q + ((long long)t * e.Hq + head) * 128;
+        } else {
+          const long long lbh = ((long long)e.layer * e.B + b) * e.Hkv + (head - e.Hq);
+          dst = e.kc + (lbh * e.S + pn) * 128;
+        }
+        *reinterpret_cast<uint4*>(dst + part * 8) = *reinterpret_cast<const uint4*>(st + n * kStPitch + part * 8);
+      }
+      __syncthreads();
     } else {
       const int g = head - e.Hq - e.Hkv;
+      const int t0 = tok0 + c0;
+      const int b = e.b0 + t0 / e.n_per, p0 = e.pos0 + t0 % e.n_per;
+      const long long lbh = ((long long)e.layer * e.B + b) * e.Hkv + g;
+      bf16* row = e.vt + (lbh * 128 + c) * e.S + p0;
+      const bool vec = nt == 64 && (t0 % e.n_per) + 64 <= e.n_per && (p0 % 8) == 0 && (e.S % 8) == 0;
+      if (vec) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = c0 + q * 16 + j;
-          if (n < n_valid) {
-            const int t = tok0 + n;
-            const int b = e.b0 + t / e.n_per, pos = e.pos0 + t % e.n_per;
-            const long long lbh = ((long long)e.layer * e.B + b) * e.Hkv + g;
-            e.vt[(lbh * 128 + c) * e.S + pos] = __float2bfloat16_rn(__uint_as_float(v[q][j]));
+          for (int j = 0; j < 16; j += 2) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(v[q][j]), __uint_as_float(v[q][j + 1]));
+            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&pr);
           }
+          *reinterpret_cast<uint4*>(row + q * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(row + q * 16 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = q * 16 + j;
+            if (n < nt) {
+              const int t = t0 + n;
+              const int bb = e.b0 + t / e.n_per, pn = e.pos0 + t % e.n_per;
+              const long long lb = ((long long)e.layer * e.B + bb) * e.Hkv + g;
+              e.vt[(lb * 128 + c) * e.S + pn] = __float2bfloat16_rn(__uint_as_float(v[q][j]));
+            }
+          }
+      }
     }
   }
 }
@@ -347,7 +381,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps
   tc_fence_after();
   if (MT == 1 && p.qkv_on) {
     qkv_epilogue(p.qkv, tmem + ((uint32_t)(warp * 32) << 16), t.m_tile, t.out_row0, t.n_valid, n_mma,
-                 ok && nkb > 0, reinterpret_cast<float*>(smem));
+                 ok && nkb > 0, smem);
   } else
   for (int mt = 0; mt < MT; ++mt) {
     const int row = mt * 128 + warp * 32 + lane;
