@@ -103,9 +103,10 @@ struct LayerW {
 };
 
 // Tile-shape overrides for sweeps, read once from DG_TUNE="key=value,..."
-// (dense_bn, dense_splits, router_bn, router_splits; 0 keeps the default).
+// (dense_bn, dense_splits, router_bn, router_splits, qkv_fused; 0 keeps the
+// default).
 struct Tune {
-  int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0;
+  int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0, qkv_fused = 0;
 };
 inline Tune read_tune() {
   Tune t;
@@ -125,6 +126,7 @@ inline Tune read_tune() {
       else if (k == "dense_splits") t.dense_splits = v;
       else if (k == "router_bn") t.router_bn = v;
       else if (k == "router_splits") t.router_splits = v;
+      else if (k == "qkv_fused") t.qkv_fused = v;
     }
     pos = end + 1;
   }
@@ -565,7 +567,9 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       qc.split_stride = (long long)Tn * m->nqkv;
     }
     // bf16: one split and the RoPE / cache scatter in the GEMM epilogue
-    const bool fuse_qkv = m->bf && m->hd == 128 && m->tune.dense_splits == 0;
+    // (off by default: the unsplit 64-token-tile GEMM measured slower than the
+    // split GEMM plus the separate post-process; DG_TUNE qkv_fused=1 enables it)
+    const bool fuse_qkv = m->bf && m->hd == 128 && m->tune.qkv_fused == 1;
     if (fuse_qkv) {
       qc.splits = 1;
       qc.qkv_on = 1;
@@ -1050,7 +1054,7 @@ int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   // one kernel; fp32: gemm + top-k), permute, gather, gate/up gemm, swiglu,
   // down gemm, combine+norm; then embed+norm, lm head, sampler, commit,
   // 4 self-cond.
-  const int per_layer = m->bf ? 12 : 14;
+  const int per_layer = (m->bf ? 12 : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
   return per_layer * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          4 /*self-conditioning*/;
 }
