@@ -364,9 +364,7 @@ __global__ void k_attn_f32(const float* __restrict__ Q, const float* __restrict_
 }
 
 // Merge split partials: o = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),
-// splits in index order.  One warp per (token, head) row; hd <= 128 (one
-// float4 per lane per split, lanes past hd idle).  Loads of up to 8 splits
-// are issued before they are combined.
+// splits in index order.  One warp per (token, head) row; hd % 32 == 0.
 template <typename T>
 __global__ void k_attn_combine(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                                int n_splits, long long rows, int hd, T* __restrict__ out) {
@@ -377,26 +375,20 @@ __global__ void k_attn_combine(const float* __restrict__ o_part, const float* __
   float M = -INFINITY;
   for (int s = 0; s < n_splits; ++s) M = fmaxf(M, lse_part[s * rows + row]);
   float den = 0.0f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int c0 = lane * 4;
-  if (c0 >= hd) return;
-  for (int s0 = 0; s0 < n_splits; s0 += 8) {
-    float l[8];
-    float4 o[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (s0 + j < n_splits) {
-        l[j] = lse_part[(s0 + j) * rows + row];
-        o[j] = *reinterpret_cast<const float4*>(o_part + ((s0 + j) * rows + row) * hd + c0);
-      }
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (s0 + j < n_splits && l[j] != -INFINITY) {
-        const float wgt = exp2f(l[j] - M);
-        den += wgt;
-        acc.x += wgt * o[j].x; acc.y += wgt * o[j].y; acc.z += wgt * o[j].z; acc.w += wgt * o[j].w;
-      }
+  for (int s = 0; s < n_splits; ++s) {
+    const float l = lse_part[s * rows + row];
+    den += (l == -INFINITY) ? 0.0f : exp2f(l - M);
   }
   const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-  store4<T>(out + row * hd + c0, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  for (int c0 = lane * 4; c0 < hd; c0 += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_splits; ++s) {
+      const float l = lse_part[s * rows + row];
+      if (l == -INFINITY) continue;
+      const float wgt = exp2f(l - M);
+      const float4 o = *reinterpret_cast<const float4*>(o_part + (s * rows + row) * hd + c0);
+      acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
+    }
+    store4<T>(out + row * hd + c0, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
 }
