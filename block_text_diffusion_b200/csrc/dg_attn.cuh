@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, AttnArgs a) {
   pdl_launch();
+  if (threadIdx.x == 0) DG_PROBE_STAMP(2000);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                                   // tile t at t * 32 KB
@@ -118,6 +119,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
+  if (threadIdx.x == 0) DG_PROBE_STAMP(2001);
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
@@ -146,6 +148,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     // ---------------- MMA issuer ----------------
     if (lane == 0 && nblk > 0) {
       bool ok = mbar_wait(&q_full, 0, a.err, DGDEV_TIMEOUT_MMA);
+      DG_PROBE_STAMP(2002);
       const uint32_t idesc_s = idesc_bf16(128, kAttnBK), idesc_o = idesc_bf16(128, 128);
       for (int j = 0; j <= nblk && ok; ++j) {
         if (j < nblk && !mbar_wait(&kv_full[j % kAttnStages], (j / kAttnStages) & 1, a.err, DGDEV_TIMEOUT_MMA)) {
@@ -176,6 +179,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
               tc_mma_bf16(tmem + t * kAttnBK, sdesc_sw128(q_addr + (kk >> 2) * 16384) + 2 * (kk & 3),
                           sdesc_sw128(k_addr + (kk >> 2) * 8192) + 2 * (kk & 3), idesc_s, kk > 0 ? 1u : 0u);
             tc_commit(&s_full[t]);
+            if (t == 0 && j < 32) DG_PROBE_STAMP(2010 + j);
           }
         }
       }
@@ -197,6 +201,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     // uniform across the warp (wait outcomes are agreed with __all_sync).
     for (int j = 0; j < nblk && ok; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, a.err, DGDEV_TIMEOUT_EPI))) { ok = false; break; }
+      if (threadIdx.x == 0 && j < 32) DG_PROBE_STAMP(2050 + j);
       tc_fence_after();
       const int key0 = (kb_begin + j) * kAttnBK;
       float v[kAttnBK];
@@ -284,7 +289,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
+      if (threadIdx.x == 0 && j < 32) DG_PROBE_STAMP(2090 + j);
     }
+    if (threadIdx.x == 0) DG_PROBE_STAMP(2130);
     // epilogue: normalised partial O and log2-sum-exp of this split
     if (ok && nblk > 0) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], (nblk - 1) & 1, a.err, DGDEV_TIMEOUT_EPI));
     tc_fence_after();
@@ -318,10 +325,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       }
     }
     if (row_valid) a.lse_part[(long long)split * rows_total + row] = have ? m_run + log2f(l_run) : -INFINITY;
+    if (threadIdx.x == 0) DG_PROBE_STAMP(2131);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+  if (threadIdx.x == 0) DG_PROBE_STAMP(2140);
 }
 
 // ---------------------------------------------------------------------------

@@ -14,14 +14,6 @@
 #pragma once
 #include "dg_device.cuh"
 
-// Timeline probes of the persistent GEMM's CTA 0 (global-timer stamps), only
-// in builds with -DDG_PROBE (performance diagnosis); no-ops otherwise.
-#ifdef DG_PROBE
-__device__ long long g_probe[1024];
-#define DG_PROBE_STAMP(i) do { if (blockIdx.x == 0 && (i) < 1024) g_probe[(i)] = (long long)global_ns(); } while (0)
-#else
-#define DG_PROBE_STAMP(i) do { } while (0)
-#endif
 
 // Fused QKV post-process for the dense bf16 GEMM (head_dim 128, one split):
 // each 128-row tile of the fused QKV weight is one head; q and k heads get
