@@ -30,7 +30,7 @@ def run(name, M, K, counts, swiglu, m256=False):
     for _ in range(3):
         dg.test_grouped_gemm(A, B, counts, G, M, out, bn=256, persistent=True, sized_ring=True, swiglu=swiglu,
                              m256=m256)
-    buf = (ctypes.c_longlong * 1024)()
+    buf = (ctypes.c_longlong * 4096)()
     L.dg_probe_read(buf)
     a = np.array(buf[:], dtype=np.int64)
     t0 = a[1000]

@@ -192,6 +192,10 @@ def test_long_context_block_loop_matches_oracle(layers):
     print(f"  noise envelope: rounds {rn['steps_used']}; committed {rn['n_committed']}; "
           f"committed-token agreement {agree_n:.4f}")
     assert abs(steps - ref["steps_used"]) <= 2 * abs(rn["steps_used"] - ref["steps_used"]) + 1
-    assert abs(ncom - ref["n_committed"]) <= 2 * abs(rn["n_committed"] - ref["n_committed"]) + \
-        max(2, ref["n_committed"] // 20)
+    # once the trajectories have diverged, each position's final commit is an
+    # independent draw: the committed count of another correct run scatters
+    # binomially around the oracle's (three standard deviations allowed)
+    p = ref["n_committed"] / 256.0
+    sd = np.sqrt(256.0 * p * (1.0 - p))
+    assert abs(ncom - ref["n_committed"]) <= max(2 * abs(rn["n_committed"] - ref["n_committed"]), 3.0 * sd) + 2
     assert agree >= agree_n - 0.05
