@@ -215,16 +215,14 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
           for (int u = 0; u < 16; ++u) v[q * 16 + u] = __uint_as_float(w[q][u]);
       }
-      // scale to log2 units; keys past the end (or after the query, causal) get -inf
-      if (!a.causal && key0 + kAttnBK <= a.n_keys) {
-#pragma unroll
-        for (int c = 0; c < kAttnBK; ++c) v[c] *= a.scale_log2;
-      } else {
+      // keys past the end (or after the query, causal) get -inf; the max is
+      // taken on raw scores (scale_log2 > 0) and scaled once
+      if (a.causal || key0 + kAttnBK > a.n_keys) {
 #pragma unroll
         for (int c = 0; c < kAttnBK; ++c) {
           const int key = key0 + c;
           const bool vis = key < a.n_keys && (!a.causal || key <= qpos);
-          v[c] = vis ? v[c] * a.scale_log2 : -INFINITY;
+          if (!vis) v[c] = -INFINITY;
         }
       }
       float mt[kAttnBK / 2];
@@ -234,7 +232,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       for (int w2 = kAttnBK / 4; w2 >= 1; w2 >>= 1)
 #pragma unroll
         for (int c = 0; c < w2; ++c) mt[c] = fmaxf(mt[c], mt[c + w2]);
-      const float mx = mt[0];
+      const float mx = mt[0] * a.scale_log2;
       // The running reference max moves only when the block max exceeds it by
       // more than 8 (a factor 256 in P), so O is rarely rescaled; the final
       // normalisation uses the same reference, so the result is unchanged.
@@ -245,7 +243,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         break;
       }
       tc_fence_after();
-      const float alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
+      const float alpha = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_new);
+      // p = 2^(s * scale - m) with one FFMA and one MUFU.EX2 (exp2(-inf) = 0);
+      // the row sum adds the fp32 values
+      const float nm = m_new == -INFINITY ? 0.0f : -m_new;
       float ls[kAttnBK / 8];
 #pragma unroll
       for (int ch = 0; ch < kAttnBK / 8; ++ch) {
@@ -253,10 +254,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         float acc = 0.0f;
 #pragma unroll
         for (int q = 0; q < 8; q += 2) {
-          const float p0 = m_new != -INFINITY ? exp2f(v[ch * 8 + q] - m_new) : 0.0f;
-          const float p1 = m_new != -INFINITY ? exp2f(v[ch * 8 + q + 1] - m_new) : 0.0f;
+          const float p0 = ex2_approx(fmaf(v[ch * 8 + q], a.scale_log2, nm));
+          const float p1 = ex2_approx(fmaf(v[ch * 8 + q + 1], a.scale_log2, nm));
+          acc += p0 + p1;
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-          acc += __low2float(pr) + __high2float(pr);
           pk[q / 2] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         ls[ch] = acc;

@@ -158,6 +158,14 @@ __device__ __forceinline__ float dg_expf(float x) {
   return __fmul_rn(p, __uint_as_float((uint32_t)(ki + 127) << 23));
 }
 
+// 2^x by the hardware approximation (flushes denormals; 2^-inf = 0); used
+// where a few ulps do not matter (attention probabilities).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // trunc(x * 2^40) as int64 for |x| < 2^23, by exponent and mantissa shifts
 // (bit-identical to converting the exact product x * 2^40 toward zero).
 __device__ __forceinline__ long long q40_trunc(float x) {
