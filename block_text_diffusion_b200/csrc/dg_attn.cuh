@@ -300,10 +300,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const bool row_valid = tok < a.n_q;
     const long long row = ((long long)(bc * a.n_q + min(tok, a.n_q - 1))) * a.Hq + head;
     const long long rows_total = (long long)a.n_canvas * a.n_q * a.Hq;
-    float* op = a.o_part + ((long long)split * rows_total + row) * 128;
     const bool loaded = ok && nblk > 0;
     const bool have = loaded && l_run > 0.0f;
     const float inv_l = have ? 1.0f / l_run : 0.0f;
+    // Staged through this tile's Q buffer (free after its last QK^T): each
+    // thread writes its row's 64 columns of a half into shared memory, then
+    // the tile's four warps copy whole 256-byte row segments with coalesced
+    // 16-byte stores (two rows per warp instruction).
+    // [128 rows][16 float4], float4 index XOR (row & 15): conflict-free both ways
+    float4* stage = reinterpret_cast<float4*>(sQ + t * kAttnQBytes);
+    const int wt = warp & 3;   // warp within the tile's group
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       uint32_t o[4][16];
@@ -312,18 +318,28 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         for (int q = 0; q < 4; ++q) tmem_ld16_nw(tO + half * 64 + q * 16, o[q]);
         tmem_wait_ld();
       }
-      if (row_valid) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int u = 0; u < 16; u += 4) {
-            const float4 o4 = have ? make_float4(__uint_as_float(o[q][u]) * inv_l, __uint_as_float(o[q][u + 1]) * inv_l,
-                                                 __uint_as_float(o[q][u + 2]) * inv_l,
-                                                 __uint_as_float(o[q][u + 3]) * inv_l)
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4*>(op + half * 64 + q * 16 + u) = o4;
-          }
+        for (int u = 0; u < 16; u += 4) {
+          const float4 o4 = have ? make_float4(__uint_as_float(o[q][u]) * inv_l, __uint_as_float(o[q][u + 1]) * inv_l,
+                                               __uint_as_float(o[q][u + 2]) * inv_l,
+                                               __uint_as_float(o[q][u + 3]) * inv_l)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          stage[r * 16 + (((q * 16 + u) >> 2) ^ (r & 15))] = o4;
+        }
+      asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
+      // rows 2i, 2i+1 of the tile per warp instruction; lane l copies float4 l % 16
+      for (int rr = wt * 2; rr < 128; rr += 8) {
+        const int rl = rr + (lane >> 4);
+        const int tok_r = tok0 + t * tok_per_tile + rl / a.G;
+        if (tok_r < a.n_q) {
+          const long long grow = ((long long)(bc * a.n_q + tok_r)) * a.Hq + g * a.G + rl % a.G;
+          float* dst = a.o_part + ((long long)split * rows_total + grow) * 128 + half * 64;
+          *reinterpret_cast<float4*>(dst + (lane & 15) * 4) = stage[rl * 16 + ((lane & 15) ^ (rl & 15))];
+        }
       }
+      asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
     }
     if (row_valid) a.lse_part[(long long)split * rows_total + row] = have ? m_run + log2f(l_run) : -INFINITY;
     if (threadIdx.x == 0) DG_PROBE_STAMP(2131);
