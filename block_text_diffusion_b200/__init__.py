@@ -62,6 +62,7 @@ def lib():
             "dg_encode_prompt": ([P, P, I32, I32, P, P], I32),
             "dg_denoise_step": ([P, P, I32, I32, P, P, I32, F, ctypes.POINTER(StepOut), P], I32),
             "dg_generate_block": ([P, P, I32, I32, P, P, P, P], I32),
+            "dg_generate": ([P, P, I32, I32, I32, P, P, P, P, P], I32),
             "dg_sync_status": ([P, P], I32),
             "dg_status_string": ([I32], ctypes.c_char_p),
             "dg_kernels_per_step": ([P, I32, I32], I32),
@@ -162,6 +163,11 @@ class Model:
     def generate_block(self, kv, B, P, canvas_out, steps_used, n_committed, stream=None):
         _check(lib().dg_generate_block(self.h, _ptr(kv), B, P, _ptr(canvas_out), _ptr(steps_used),
                                        _ptr(n_committed), _stream(stream)), "dg_generate_block")
+
+    def generate(self, prompt, B, P, n_blocks, kv, tokens_out, steps_used, n_committed, stream=None):
+        """Block-autoregressive generation of n_blocks canvases (see dg_generate)."""
+        _check(lib().dg_generate(self.h, _ptr(prompt), B, P, n_blocks, _ptr(kv), _ptr(tokens_out),
+                                 _ptr(steps_used), _ptr(n_committed), _stream(stream)), "dg_generate")
 
     def sync_status(self, stream=None):
         _check(lib().dg_sync_status(self.h, _stream(stream)), "device status")

@@ -170,7 +170,8 @@ struct dg_model {
   cudaGraphExec_t gexec = nullptr;
   cudaGraph_t graph = nullptr;
   void* g_kv = nullptr;
-  int g_B = -1, g_P = -1;
+  int g_B = -1, g_P = -1, g_S = -1;
+  uint64_t g_seed = 0;
   int launches_per_round = 0;
 
   Prof prof;
@@ -510,15 +511,19 @@ struct KvGeom {
   void* Vt;
 };
 
-KvGeom kv_geom(const dg_model* m, void* kv, int B, int P) {
+// Cache geometry for a context of P positions in a buffer laid out for a
+// context of up to P_cap positions (slot stride S from P_cap).
+KvGeom kv_geom_cap(const dg_model* m, void* kv, int B, int P, int P_cap) {
   KvGeom g;
   g.B = B;
   g.P = P;
-  g.S = ((P + kCanvas + 63) / 64) * 64;
+  g.S = ((P_cap + kCanvas + 63) / 64) * 64;
   g.K = kv;
   g.Vt = (uint8_t*)kv + (size_t)m->L * B * m->hkv * g.S * m->hd * m->esz;
   return g;
 }
+
+KvGeom kv_geom(const dg_model* m, void* kv, int B, int P) { return kv_geom_cap(m, kv, B, P, P); }
 
 struct AttnMaps {
   CUtensorMap q, k, v;
@@ -824,6 +829,32 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
   return DG_OK;
 }
 
+// Causal encode of tokens [B][n] (row stride ld) at positions P0 .. P0+n-1
+// of every canvas into the cache geometry g: each chunk attends to keys
+// [0, its last position], so a continuation sees the cache written before it.
+dg_status encode_tokens(dg_model* m, const KvGeom& g, const int32_t* tok, long long ld, int P0, int n,
+                        cudaStream_t s) {
+  const int chunk = std::min(n, m->Tw);
+  for (int b = 0; b < g.B; ++b) {
+    for (int c0 = 0; c0 < n; c0 += chunk) {
+      const int nc = std::min(chunk, n - c0);
+      {
+        LaunchScope ls(m, s, PH_EMBED);
+        if (m->bf)
+          launch_pdl(k_embed_norm<bf16>, nc, 256, 0, s, tok + (size_t)b * ld + c0, (const bf16*)m->emb, nullptr,
+                     nullptr, (bf16*)m->h, (bf16*)m->x, m->d, m->V, m->c.rms_eps, &m->st->err);
+        else
+          launch_pdl(k_embed_norm<float>, nc, 256, 0, s, tok + (size_t)b * ld + c0, (const float*)m->emb, nullptr,
+                     nullptr, (float*)m->h, (float*)m->x, m->d, m->V, m->c.rms_eps, &m->st->err);
+      }
+      dg_status st = m->bf ? run_layers<bf16>(m, g, b, 1, nc, P0 + c0, P0 + c0 + nc, true, s)
+                           : run_layers<float>(m, g, b, 1, nc, P0 + c0, P0 + c0 + nc, true, s);
+      if (st != DG_OK) return st;
+    }
+  }
+  return DG_OK;
+}
+
 dg_status check_shape(const dg_model* m, int B, int P) {
   if (B < 1 || B > m->c.max_canvases || P < 1 || P > m->c.max_prompt) return DG_ERR_INVALID_ARG;
   return DG_OK;
@@ -835,7 +866,7 @@ void release_graph(dg_model* m) {
   m->gexec = nullptr;
   m->graph = nullptr;
   m->g_kv = nullptr;
-  m->g_B = m->g_P = -1;
+  m->g_B = m->g_P = m->g_S = -1;
 }
 
 template <typename T>
@@ -912,6 +943,30 @@ dg_status latched(dg_model* m, cudaStream_t s) {
 // ===========================================================================
 // C ABI
 // ===========================================================================
+// One block on the device loop for the cache geometry g: (re)captures the
+// loop graph when the geometry or the sampling seed changed, then launches it.
+// Results stay in m->canvas_out / steps_used / ncom_out.
+dg_status run_block(dg_model* m, const KvGeom& g, cudaStream_t s) {
+  if (!m->gexec || m->g_kv != g.K || m->g_B != g.B || m->g_P != g.P || m->g_S != g.S ||
+      m->g_seed != m->c.sample_seed) {
+    dg_status st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
+    if (st != DG_OK && g_use_pdl) {
+      // a driver that cannot capture programmatic edges into the loop body:
+      // capture the same launches without the attribute
+      cudaGetLastError();
+      g_use_pdl = false;
+      st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
+    }
+    if (st != DG_OK) return st;
+    m->g_kv = g.K; m->g_B = g.B; m->g_P = g.P; m->g_S = g.S; m->g_seed = m->c.sample_seed;
+  }
+  { LaunchScope ls(m, s, PH_CONTROL);
+    k_loop_init<<<g.B, 256, 0, s>>>(m->st, m->c.max_steps, g.B, m->canvas_cur, m->done, m->steps_used, m->ncom_out,
+                                    m->prev_amax, m->c.sample_seed, m->V); }
+  CU_TRY(cudaGraphLaunch(m->gexec, s));
+  return DG_OK;
+}
+
 extern "C" {
 
 const char* dg_status_string(dg_status s) {
@@ -1065,26 +1120,7 @@ dg_status dg_encode_prompt(dg_model* m, const int32_t* prompt, int32_t B, int32_
   cudaStream_t s = (cudaStream_t)stream;
   const KvGeom g = kv_geom(m, kv, B, P);
   CU_TRY(cudaMemsetAsync(kv, 0, dg_kv_bytes(m, B, P), s));
-  const int chunk = std::min(P, m->Tw);
-  for (int b = 0; b < B; ++b) {
-    for (int c0 = 0; c0 < P; c0 += chunk) {
-      const int n = std::min(chunk, P - c0);
-      {
-        LaunchScope ls(m, s, PH_EMBED);
-        if (m->bf)
-          launch_pdl(k_embed_norm<bf16>, n, 256, 0, s, prompt + (size_t)b * P + c0, (const bf16*)m->emb, nullptr, nullptr,
-                                              (bf16*)m->h, (bf16*)m->x, m->d, m->V, m->c.rms_eps, &m->st->err);
-        else
-          launch_pdl(k_embed_norm<float>, n, 256, 0, s, prompt + (size_t)b * P + c0, (const float*)m->emb, nullptr,
-                                               nullptr, (float*)m->h, (float*)m->x, m->d, m->V, m->c.rms_eps,
-                                               &m->st->err);
-      }
-      dg_status st = m->bf ? run_layers<bf16>(m, g, b, 1, n, c0, c0 + n, true, s)
-                           : run_layers<float>(m, g, b, 1, n, c0, c0 + n, true, s);
-      if (st != DG_OK) return st;
-    }
-  }
-  return DG_OK;
+  return encode_tokens(m, g, prompt, P, 0, P, s);
 }
 
 dg_status dg_denoise_step(dg_model* m, void* kv, int32_t B, int32_t P, const int32_t* canvas,
@@ -1120,27 +1156,47 @@ dg_status dg_generate_block(dg_model* m, void* kv, int32_t B, int32_t P, int32_t
   if (!m || !kv || !canvas_out || !steps_used || !n_committed) return DG_ERR_INVALID_ARG;
   DG_TRY(check_shape(m, B, P));
   cudaStream_t s = (cudaStream_t)stream;
-  const KvGeom g = kv_geom(m, kv, B, P);
-  if (!m->gexec || m->g_kv != kv || m->g_B != B || m->g_P != P) {
-    dg_status st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
-    if (st != DG_OK && g_use_pdl) {
-      // a driver that cannot capture programmatic edges into the loop body:
-      // capture the same launches without the attribute
-      cudaGetLastError();
-      g_use_pdl = false;
-      st = m->bf ? capture_block_graph<bf16>(m, g) : capture_block_graph<float>(m, g);
-    }
-    if (st != DG_OK) return st;
-    m->g_kv = kv; m->g_B = B; m->g_P = P;
-  }
-  { LaunchScope ls(m, s, PH_CONTROL);
-    k_loop_init<<<B, 256, 0, s>>>(m->st, m->c.max_steps, B, m->canvas_cur, m->done, m->steps_used, m->ncom_out,
-                                  m->prev_amax, m->c.sample_seed, m->V); }
-  CU_TRY(cudaGraphLaunch(m->gexec, s));
+  DG_TRY(run_block(m, kv_geom(m, kv, B, P), s));
   CU_TRY(cudaMemcpyAsync(canvas_out, m->canvas_out, (size_t)B * kCanvas * sizeof(int), cudaMemcpyDeviceToDevice, s));
   CU_TRY(cudaMemcpyAsync(steps_used, m->steps_used, (size_t)B * sizeof(int), cudaMemcpyDeviceToDevice, s));
   CU_TRY(cudaMemcpyAsync(n_committed, m->ncom_out, (size_t)B * sizeof(int), cudaMemcpyDeviceToDevice, s));
   return DG_OK;
+}
+
+dg_status dg_generate(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, int32_t n_blocks, void* kv,
+                      int32_t* tokens_out, int32_t* steps_used, int32_t* n_committed, void* stream) {
+  if (!m || !prompt || !kv || !tokens_out || !steps_used || !n_committed || n_blocks < 1)
+    return DG_ERR_INVALID_ARG;
+  const long long P_cap = (long long)P + (long long)kCanvas * (n_blocks - 1);
+  if (P_cap > m->c.max_prompt) return DG_ERR_INVALID_ARG;
+  DG_TRY(check_shape(m, B, (int)P_cap));
+  DG_TRY(check_shape(m, B, P));
+  cudaStream_t s = (cudaStream_t)stream;
+  CU_TRY(cudaMemsetAsync(kv, 0, dg_kv_bytes(m, B, (int)P_cap), s));
+  DG_TRY(encode_tokens(m, kv_geom_cap(m, kv, B, P, (int)P_cap), prompt, P, 0, P, s));
+  const uint64_t seed0 = m->c.sample_seed;
+  dg_status st = DG_OK;
+  for (int i = 0; i < n_blocks && st == DG_OK; ++i) {
+    const int Pi = P + kCanvas * i;
+    const KvGeom g = kv_geom_cap(m, kv, B, Pi, (int)P_cap);
+    m->c.sample_seed = seed0 + (uint64_t)i;   // block i samples with seed + i
+    st = run_block(m, g, s);
+    if (st != DG_OK) break;
+    const size_t row = (size_t)n_blocks * kCanvas * sizeof(int);
+    if (cudaMemcpy2DAsync(tokens_out + (size_t)i * kCanvas, row, m->canvas_out, kCanvas * sizeof(int),
+                          kCanvas * sizeof(int), B, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpy2DAsync(steps_used + i, n_blocks * sizeof(int), m->steps_used, sizeof(int), sizeof(int), B,
+                          cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpy2DAsync(n_committed + i, n_blocks * sizeof(int), m->ncom_out, sizeof(int), sizeof(int), B,
+                          cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+      st = DG_ERR_CUDA;
+      break;
+    }
+    // the finished canvas joins the context: causal encode of its tokens
+    if (i + 1 < n_blocks) st = encode_tokens(m, g, m->canvas_out, kCanvas, Pi, kCanvas, s);
+  }
+  m->c.sample_seed = seed0;
+  return st;
 }
 
 dg_status dg_sync_status(dg_model* m, void* stream) {

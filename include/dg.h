@@ -140,6 +140,22 @@ dg_status dg_denoise_step(dg_model* model, void* kv, int32_t B, int32_t P, const
 dg_status dg_generate_block(dg_model* model, void* kv, int32_t B, int32_t P, int32_t* canvas_out,
                             int32_t* steps_used, int32_t* n_committed, void* stream);
 
+/* Block-autoregressive generation (release news "不是逐词写，而是整块去噪";
+ * "谷歌都下场了：扩散语言模型的四倍速与六倍错", section 一): the prompt is encoded
+ * causally, then n_blocks canvases are generated one after another, each as
+ * dg_generate_block does; a finished canvas joins the context by a causal
+ * encode of its 256 tokens at positions P + 256 i, so block i attends to
+ * [prompt ; blocks 0 .. i-1 ; its own canvas].  Block i samples with seed
+ * sample_seed + i.
+ *   prompt      device int32 [B, P].
+ *   kv          caller buffer of dg_kv_bytes(model, B, P + 256 (n_blocks - 1))
+ *               bytes; holds the whole context on return.
+ *   tokens_out  device int32 [B, n_blocks, 256]: each block's sampled tokens.
+ *   steps_used, n_committed  device int32 [B, n_blocks].
+ * P + 256 (n_blocks - 1) must not exceed max_prompt (DG_ERR_INVALID_ARG). */
+dg_status dg_generate(dg_model* model, const int32_t* prompt, int32_t B, int32_t P, int32_t n_blocks, void* kv,
+                      int32_t* tokens_out, int32_t* steps_used, int32_t* n_committed, void* stream);
+
 /* Wait for the model's stream and return the first latched device error
  * (DG_ERR_TIMEOUT, DG_ERR_STATE) or DG_OK; clears the latch. */
 dg_status dg_sync_status(dg_model* model, void* stream);

@@ -402,3 +402,23 @@ def generate_block(model, K, V, canvas_id=0, max_steps=None):
             return dict(canvas=r["tokens"], steps_used=s + 1, n_committed=r["n_committed"], trace=trace)
         canvas, selfcond, prev_amax = r["canvas_next"], r["selfcond_next"], r["amax"]
     raise AssertionError("unreachable")
+
+
+def generate(model, prompt, n_blocks, canvas_id=0):
+    """Block-autoregressive generation: canvases are produced one after another
+    (release news "不是逐词写，而是整块去噪"; "谷歌都下场了：扩散语言模型的四倍速与六倍错"
+    section 一: a finished canvas joins the context, then the next canvas
+    starts).  Block i is generated against the causal KV of [prompt ; blocks
+    0..i-1] (its canvas at positions P + 256 i) and samples with seed
+    sample_seed + i.  Returns the list of generate_block results."""
+    import copy
+    context = [int(x) for x in prompt]
+    blocks = []
+    for i in range(n_blocks):
+        K, V = encode_prompt(model, context)
+        mi = copy.copy(model)
+        mi.cfg = model.cfg.replace(sample_seed=model.cfg.sample_seed + i)
+        ref = generate_block(mi, K, V, canvas_id)
+        blocks.append(ref)
+        context += [int(x) for x in ref["canvas"]]
+    return blocks

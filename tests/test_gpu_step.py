@@ -159,6 +159,35 @@ def test_tiny_round_and_block_match_oracle(tiny):
     assert abs(int(host(nc)[0]) - ref["n_committed"]) <= 2
 
 
+def test_tiny_block_autoregressive_generation():
+    # dg_generate: two blocks, the first joining the context before the second
+    # (causal encode of its tokens after the prompt); against the oracle's chain
+    w = I.TINY_FP32
+    P, n_blocks = w.prompt_len, 2
+    P_cap = P + 256 * (n_blocks - 1)
+    gm = dg.Model(w, max_prompt=P_cap)
+    prompt = I.prompt_ids(w.sample_seed, 1, P, w.vocab)
+    kv = gm.new_kv(1, P_cap)
+    toks = torch.zeros((1, n_blocks, 256), dtype=torch.int32, device="cuda")
+    su = torch.zeros((1, n_blocks), dtype=torch.int32, device="cuda")
+    nc = torch.zeros((1, n_blocks), dtype=torch.int32, device="cuda")
+    gm.generate(cu(prompt), 1, P, n_blocks, kv, toks, su, nc)
+    gm.sync_status()
+    gt, gs, gn = host(toks)[0], host(su)[0], host(nc)[0]
+    om_ = om.Model(w)
+    refs = om.generate(om_, prompt[0], n_blocks)
+    for i, ref in enumerate(refs):
+        assert int(gs[i]) == ref["steps_used"], i
+        assert (gt[i] == ref["canvas"]).mean() >= 0.99, i
+        assert abs(int(gn[i]) - ref["n_committed"]) <= 2, i
+    # the cache holds [prompt ; block 0] encoded causally (block 1's canvas after it)
+    K, V = read_kv(gm, kv, 1, P_cap)
+    Ko, Vo = om.encode_prompt(om_, np.concatenate([prompt[0], gt[0]]))
+    assert np.allclose(K[:, 0, :, :P_cap], Ko, rtol=1e-4, atol=1e-5)
+    assert np.allclose(V[:, 0, :, :P_cap], Vo, rtol=1e-4, atol=1e-5)
+    gm.close()
+
+
 # --- mid bf16 workload with a synthetic prompt cache -------------------------------------
 @pytest.fixture(scope="module")
 def mid():

@@ -346,3 +346,38 @@ def test_token_logits_with_routing_reproduces_forward(micro):
         row = om.token_logits_with_routing(one, one.layers[0], trace[0]["h_attn"][t], ids, w)
         assert np.allclose(row, logits[t], rtol=1e-12, atol=1e-12)
         assert list(ids) == list(trace[0]["ids"][t])
+
+
+# --- block-autoregressive continuation ------------------------------------------------------
+def test_causal_encode_is_prefix_consistent():
+    # a finished canvas joins the context by a causal encode: the cache of the
+    # prompt part must not change when tokens are appended after it
+    w = I.TINY_FP32.replace(n_layers=1, max_steps=2)
+    m = om.Model(w)
+    prompt = I.prompt_ids(w.sample_seed, 1, 24, w.vocab)[0]
+    extra = I.prompt_ids(w.sample_seed + 1, 1, 40, w.vocab)[0]
+    K0, V0 = om.encode_prompt(m, prompt)
+    K1, V1 = om.encode_prompt(m, np.concatenate([prompt, extra]))
+    assert np.array_equal(K1[:, :, :24], K0) and np.array_equal(V1[:, :, :24], V0)
+
+
+def test_generate_chains_blocks_on_the_growing_context():
+    w = I.TINY_FP32.replace(n_layers=1, max_steps=2)
+    m = om.Model(w)
+    prompt = I.prompt_ids(w.sample_seed, 1, 16, w.vocab)[0]
+    blocks = om.generate(m, prompt, 2)
+    # block 0 is exactly the single-block generation on the prompt
+    K, V = om.encode_prompt(m, prompt)
+    b0 = om.generate_block(m, K, V)
+    assert np.array_equal(blocks[0]["canvas"], b0["canvas"]) and blocks[0]["steps_used"] == b0["steps_used"]
+    # block 1 runs on [prompt ; block 0] with seed + 1
+    K1, V1 = om.encode_prompt(m, np.concatenate([prompt, b0["canvas"]]))
+    assert K1.shape[2] == 16 + 256
+    import copy
+    m1 = copy.copy(m)
+    m1.cfg = w.replace(sample_seed=w.sample_seed + 1)
+    b1 = om.generate_block(m1, K1, V1)
+    assert np.array_equal(blocks[1]["canvas"], b1["canvas"])
+    # the two blocks start from different noise
+    assert not np.array_equal(sp.initial_canvas(w.sample_seed, 0, 256, w.vocab),
+                              sp.initial_canvas(w.sample_seed + 1, 0, 256, w.vocab))
