@@ -42,6 +42,8 @@ def parse():
                     help="override the round budget (short runs for profiler launch lists)")
     ap.add_argument("--no-fast-converging", action="store_true",
                     help="skip the committed-tokens measurement on the fast-converging workload")
+    ap.add_argument("--routing-study", action="store_true",
+                    help="also sweep a structured router bias over expert-pool sizes (routing locality)")
     return ap.parse_args()
 
 
@@ -258,6 +260,10 @@ def run_ours(a):
     # distinct experts each layer streamed in the profiled round (measured routing)
     touched = model.touched_experts()
 
+    study = None
+    if a.routing_study:
+        study = routing_study(dg, I, torch, model, w, kv, B, P, block, steps)
+
     # committed tokens on the fast-converging workload (logit scale 16), where
     # random-init weights still commit: single-GPU runs only
     fast = None
@@ -316,6 +322,7 @@ def run_ours(a):
                 "h2d_bytes_per_step": B * P * 4 * world, "d2h_bytes_per_step": (B * 256 + 2 * B) * 4 * world,
                 "includes": "prompt H2D, causal prompt encode, block loop, result D2H"},
         "fast_converging": fast,
+        "routing_study": study,
         "gpu_launches": int(n_rounds / world * (kper + 1) + a.steps * (1 + 3)) * world,
         "clocks": clk.summary(),
     }
@@ -353,6 +360,49 @@ def fast_converging(dg, I, torch, blocks=3):
     n_r, n_c = int(rounds.item()), int(committed.item())
     return {"workload": w.name, "prompt_len": P, "blocks": blocks, "committed_tokens_per_s": n_c / (ms * 1e-3),
             "committed_per_block": n_c / blocks, "rounds_per_block": n_r / blocks, "ms_per_block": ms / blocks}
+
+
+def routing_study(dg, I, torch, model, w, kv, B, P, block, steps, pools=(8, 16, 32, 64, 84, 128), beta=8.0,
+                  reps=2):
+    """Routing locality: a structured per-token router bias confines each
+    layer's canvas tokens to a pool of experts (each token prefers top_k of
+    them, bias `beta`).  Per pool size: the distinct experts the layers
+    touched, ms per round, the step roofline and its fraction, and the expert
+    gate|up GEMM's achieved bandwidth."""
+    stream = torch.cuda.current_stream()
+    hbm, _, tf_sus, _ = peaks()
+    out = []
+    for pool in pools:
+        if not w.top_k <= pool <= w.n_experts:
+            continue
+        bias = torch.from_numpy(I.routing_bias(7, w.n_layers, B * 256, w.n_experts, w.top_k, pool, beta)).cuda()
+        model.set_routing_bias(bias)
+        try:
+            block()                                   # recapture + warm-up
+            torch.cuda.synchronize()
+            rounds = torch.zeros((), dtype=torch.int64, device="cuda")
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                block()
+                rounds += steps.sum()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_round = e0.elapsed_time(e1) / max(1, int(rounds.item()))
+            prof = model.profile_step(kv, B, P, reps=2)
+            touched = model.touched_experts()
+        finally:
+            model.set_routing_bias(None)
+        model.sync_status()
+        b_round, f_round = round_work(w, B, P, touched)
+        roof = max(b_round / (hbm * 1e9), f_round / (tf_sus * 1e12)) * 1e3
+        gu_ms, gu_n = prof["expert_gate_up_gemm"]
+        dn_ms = prof["expert_down_gemm"][0]
+        gu_gbs = gate_up_bytes(w, B, touched) / (gu_ms / max(1, gu_n) * 1e-3) / 1e9
+        out.append({"pool": pool, "touched_mean": sum(touched) / len(touched), "ms_per_round": ms_round,
+                    "roof_ms": roof, "frac": roof / ms_round, "expert_ms_per_round": (gu_ms + dn_ms) / 2,
+                    "gate_up_gbs": gu_gbs, "gate_up_frac": gu_gbs / hbm})
+    return out
 
 
 def block_autoregressive(dg, I, torch, blocks=3):

@@ -72,7 +72,8 @@ def lib():
             "dg_test_commit": ([P, P, P, P, I32, I32, U64, I32, I32, I32, F, I32, F, P, P, P, P, P], I32),
             "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, I32, P], I32),
             "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
-            "dg_test_router": ([P, P, P, I32, I32, I32, I32, P, P, P], I32),
+            "dg_test_router": ([P, P, P, P, I32, I32, I32, I32, P, P, P], I32),
+            "dg_set_routing_bias": ([P, P, I32], I32),
             "dg_test_attention": ([P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P], I32),
             "dg_read_weight": ([P, I32, P, P], I32),
             "dg_load_kv": ([P, P, I32, I32, P, P, P], I32),
@@ -194,6 +195,17 @@ class Model:
         _check(lib().dg_expert_counts(self.h, _ptr(counts), _stream(stream)), "dg_expert_counts")
         return counts
 
+    def set_routing_bias(self, bias, n_tok=None):
+        """Per-token router bias of the canvas passes, device fp32 [L, n_tok, E]
+        (None removes it); the caller keeps the tensor alive while in use."""
+        if bias is None:
+            _check(lib().dg_set_routing_bias(self.h, None, 0), "dg_set_routing_bias")
+            self._routing_bias = None
+            return
+        n = bias.shape[1] if n_tok is None else n_tok
+        _check(lib().dg_set_routing_bias(self.h, _ptr(bias), n), "dg_set_routing_bias")
+        self._routing_bias = bias
+
     def touched_experts(self, stream=None):
         """Distinct experts each layer of the most recent call routed to (list)."""
         import torch
@@ -250,11 +262,12 @@ def test_gemm(A, B, out, alpha=1.0, k_splits=1, bn=256, persistent=False, m256=F
                               float(alpha), k_splits, bn, flags, _stream(stream)), "dg_test_gemm")
 
 
-def test_router(x, wr, ids, gate, bias=None, stream=None):
+def test_router(x, wr, ids, gate, bias=None, tok_bias=None, stream=None):
     T, d = x.shape
     E = wr.shape[0]
     k = ids.shape[1]
-    _check(lib().dg_test_router(_ptr(x), _ptr(wr), _ptr(bias) if bias is not None else None, T, d, E, k,
+    _check(lib().dg_test_router(_ptr(x), _ptr(wr), _ptr(bias) if bias is not None else None,
+                                _ptr(tok_bias) if tok_bias is not None else None, T, d, E, k,
                                 _ptr(ids), _ptr(gate), _stream(stream)), "dg_test_router")
 
 

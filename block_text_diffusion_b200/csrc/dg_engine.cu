@@ -149,6 +149,10 @@ struct dg_model {
   std::vector<LayerW> layers;
   float2* rope = nullptr;
   float* rbias = nullptr;
+  // optional per-token router bias of the canvas pass (caller-owned, fp32
+  // [L][tok_bias_n][E]; a workload input that structures routing)
+  const float* tok_bias = nullptr;
+  int tok_bias_n = 0;
   CUtensorMap tm_E, tm_ET, tm_Wsc;
 
   void *h = nullptr, *x = nullptr, *q = nullptr, *o = nullptr, *xp = nullptr, *act = nullptr;
@@ -638,6 +642,10 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     if (m->dbg_h)
       launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
     // MoE
+    // per-token router bias: canvas passes only, rows of canvases b0 ..
+    const float* tb = (!causal && m->tok_bias)
+                          ? m->tok_bias + ((size_t)l * m->tok_bias_n + (size_t)b0 * n_per) * m->E : nullptr;
+    if (tb && (b0 + n_canvas) * n_per > m->tok_bias_n) return DG_ERR_INVALID_ARG;
     // router: logits r = x Wr^T (fp32 accumulation) and top-k.  Up to 128
     // experts (bf16): one clustered kernel; otherwise a GEMM then a top-k kernel.
     if (m->bf && m->E <= 128 && m->k <= 32) {
@@ -647,7 +655,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
         CU_TRY(cudaFuncSetAttribute(k_router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterSmem));
         attr = true;
       }
-      RouterArgs ra{m->E, m->k, Tn, cdiv(d, 64), m->rbias, m->ids, m->gate, &m->st->err};
+      RouterArgs ra{m->E, m->k, Tn, cdiv(d, 64), m->rbias, tb, m->ids, m->gate, &m->st->err};
       launch_pdl(k_router_tc, cdiv(Tn, kRouterBN) * kRouterSplits, 128, kRouterSmem, s, w.tm_wr, m->tm_x.m[0], ra);
       CU_TRY(cudaGetLastError());
     } else {
@@ -665,7 +673,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     DG_TRY(gemm(m, rc, PH_ROUTER, s));
     { LaunchScope ls(m, s, PH_ROUTER);
       launch_pdl(k_router_topk, cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s, 
-          m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, m->E, m->k, Tn, m->ids, m->gate); }
+          m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, tb, m->E, m->k, Tn, m->ids, m->gate); }
     }
     // expert GEMM split-K factors are picked on the device from the routing
     // (bf16 persistent path only; the fp32 path keeps one split)

@@ -374,8 +374,8 @@ __global__ void k_sum_round(T* __restrict__ out, const float* __restrict__ ws, l
 // over the k selected logits.  One warp per token.
 // ---------------------------------------------------------------------------
 __global__ void k_router_topk(const float* __restrict__ r, int splits, long long split_stride,
-                              const float* __restrict__ bias, int E, int k, int n_tok, int* __restrict__ ids,
-                              float* __restrict__ gate) {
+                              const float* __restrict__ bias, const float* __restrict__ tok_bias, int E, int k,
+                              int n_tok, int* __restrict__ ids, float* __restrict__ gate) {
   pdl_enter();
   extern __shared__ float rt[];   // [warps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -385,7 +385,7 @@ __global__ void k_router_topk(const float* __restrict__ r, int splits, long long
   for (int e = lane; e < E; e += 32) {
     float v = r[t * E + e];
     for (int s = 1; s < splits; ++s) v += r[s * split_stride + t * E + e];
-    lg[e] = v + (bias ? bias[e] : 0.0f);
+    lg[e] = v + (bias ? bias[e] : 0.0f) + (tok_bias ? tok_bias[t * E + e] : 0.0f);
   }
   __syncwarp();
   float sel = 0.0f, top = 0.0f;

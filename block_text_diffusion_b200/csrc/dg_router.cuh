@@ -1,7 +1,8 @@
 // MoE router as one kernel: router logits on the tensor cores, split-K
 // partials reduced through distributed shared memory, top-k and gate softmax.
 //
-// r[t][e] = sum_k x[t][k] Wr[e][k] (+ b_e), fp32 accumulation; the k largest
+// r[t][e] = sum_k x[t][k] Wr[e][k] (+ b_e) (+ c[t][e], an optional per-token
+// bias given as input), fp32 accumulation; the k largest
 // (ties to the lower expert id) in descending order; gates = softmax over the
 // k selected logits.  (Mixture-of-Experts FFN of the DiffusionGemma
 // technical-report explainer, section 二: each token goes to top_k experts.)
@@ -24,6 +25,7 @@ constexpr int kRouterSmem = kRouterStages * kRouterStage + kRouterBN * 128 * 4 +
 struct RouterArgs {
   int E, k, n_tok, kb_total;
   const float* bias;   // [E] or null
+  const float* tok_bias;   // [n_tok][E] or null
   int* ids;            // [n_tok][k]
   float* gate;         // [n_tok][k]
   int* err;
@@ -133,7 +135,8 @@ k_router_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       const int e = lane + 32 * q;
       float acc = 0.0f;
       for (int r = 0; r < kRouterSplits; ++r) acc += cluster_peer(part, r)[tl * 128 + e];
-      lg[q] = (e < p.E) ? acc + (p.bias ? p.bias[e] : 0.0f) : -INFINITY;
+      lg[q] = (e < p.E) ? acc + (p.bias ? p.bias[e] : 0.0f) + (p.tok_bias ? p.tok_bias[t * p.E + e] : 0.0f)
+                        : -INFINITY;
     }
     float sel = 0.0f, top = 0.0f;
     int sid = 0;

@@ -193,3 +193,23 @@ def prompt_kv(seed: int, n_layers: int, batch: int, n_kv_heads: int, prompt_len:
     k = normal(seed, 108, shape, std=1.0, bf16=bf16)
     v = normal(seed, 109, shape, std=1.0, bf16=bf16)
     return k, v
+
+
+def routing_bias(seed: int, n_layers: int, tokens: int, n_experts: int, top_k: int, pool: int,
+                 beta: float = 8.0) -> np.ndarray:
+    """Structured per-token router bias [n_layers, tokens, n_experts] float32
+    standing in for the expert locality of a trained router (the pages report
+    about 84 of 128 experts touched per round).  In each layer a random pool
+    of `pool` experts serves the canvas tokens and each token prefers top_k
+    distinct experts of that pool: +beta on those, 0 elsewhere.  With beta
+    well above the spread of the router logits every token picks its preferred
+    experts, so a layer touches about `pool` distinct experts."""
+    if not top_k <= pool <= n_experts:
+        raise ValueError("pool must lie in [top_k, n_experts]")
+    g = _rng(seed, 110)
+    out = np.zeros((n_layers, tokens, n_experts), dtype=np.float32)
+    for l in range(n_layers):
+        members = g.permutation(n_experts)[:pool]
+        for t in range(tokens):
+            out[l, t, members[g.choice(pool, size=top_k, replace=False)]] = beta
+    return out

@@ -62,8 +62,20 @@ dg_status dg_test_gemm(const void* A, const void* B, float* out, int32_t M, int3
  * order -> ids int32 [T, k], and their softmax -> gate fp32 [T, k]
  * (Mixture-of-Experts FFN, DiffusionGemma technical-report explainer,
  * section 二).  Allocates (a 32-byte error word); synchronises. */
-dg_status dg_test_router(const void* x, const void* wr, const float* bias, int32_t T, int32_t d, int32_t E,
-                         int32_t k, int32_t* ids, float* gate, void* stream);
+dg_status dg_test_router(const void* x, const void* wr, const float* bias, const float* tok_bias, int32_t T,
+                         int32_t d, int32_t E, int32_t k, int32_t* ids, float* gate, void* stream);
+
+/* Structured per-token router bias for the canvas passes (routing-locality
+ * workloads: a stand-in for the expert locality of a trained router, which
+ * the DiffusionGemma technical-report explainer, section 五, puts at about
+ * 84 of 128 experts per round).  bias: device fp32 [L][n_tok][E], owned by
+ * the caller and read by every later canvas round until replaced; row
+ * b*256 + i biases canvas b, position i; the router adds it to the logits
+ * (selection and gates).  n_tok = 0 (bias may be NULL) removes it.  n_tok
+ * must be a multiple of 256 and at most max_canvases*256, and a later round
+ * over more canvases than n_tok/256 fails with DG_ERR_INVALID_ARG.  Drops
+ * the captured block loop (the next block recaptures it).  Host-only. */
+dg_status dg_set_routing_bias(dg_model* m, const float* bias, int32_t n_tok);
 
 /* Grouped GEMM as used by the experts: A [groups*M, K], B [rows, K] with
  * rows ordered by group (counts host int32 [groups]); out [rows, M] fp32,

@@ -116,6 +116,9 @@ class Model:
         s = cfg.weight_seed
         self.embed = weight_values(s, T_EMBED, (V, d), bf)
         self.wsc = weight_values(s, T_WSC, (d, d), bf)
+        # optional per-token router bias of the canvas pass, [L, 256 * canvases, E]
+        # (a workload input that structures routing; None = no such term)
+        self.route_bias = None
         self.layers = []
         for l in range(cfg.n_layers if layers is None else layers):
             t = lambda w: layer_tensor_id(l, w)
@@ -176,14 +179,12 @@ def attention(q, k, v, causal_offset=None):
     return out
 
 
-def router(x, wr, top_k, zipf_s=0.0):
-    """Top-k gating.  r = x Wr^T (+ b_e = -s ln(e+1)); the k largest logits
-    (ties to the lower expert id) in descending order; gate weights are the
-    softmax over those k logits, so they sum to 1.  Returns (ids [n,k] int32,
-    weights [n,k] float64)."""
-    r = np.asarray(x, dtype=np.float64) @ np.asarray(wr, dtype=np.float64).T
-    if zipf_s:
-        r = r + (-zipf_s * np.log(np.arange(wr.shape[0], dtype=np.float64) + 1.0))[None, :]
+def router(x, wr, top_k, zipf_s=0.0, extra=None):
+    """Top-k gating.  r = x Wr^T (+ b_e = -s ln(e+1)) (+ extra[t, e], a per-token
+    bias given as input); the k largest logits (ties to the lower expert id) in
+    descending order; gate weights are the softmax over those k logits, so they
+    sum to 1.  Returns (ids [n,k] int32, weights [n,k] float64)."""
+    r = router_logits(x, wr, zipf_s, extra)
     n, E = r.shape
     ids = np.empty((n, top_k), dtype=np.int32)
     w = np.empty((n, top_k))
@@ -200,12 +201,12 @@ def silu(z):
     return z / (1.0 + np.exp(-z))
 
 
-def moe(model, layer, x):
+def moe(model, layer, x, extra=None):
     """sum over the k slots (in slot order) of gate_weight * expert FFN, with
     expert FFN(x) = (silu(x Wg^T) * (x Wu^T)) Wd^T and the SwiGLU activation
-    rounded to the storage dtype."""
+    rounded to the storage dtype.  `extra`: per-token router bias or None."""
     cfg = model.cfg
-    ids, w = router(x, layer.wr, cfg.top_k, cfg.zipf_s)
+    ids, w = router(x, layer.wr, cfg.top_k, cfg.zipf_s, extra)
     y = np.zeros_like(x)
     for j in range(cfg.top_k):
         for e in np.unique(ids[:, j]):
@@ -220,12 +221,10 @@ def _proj(x, w):
     return x @ np.asarray(w, dtype=np.float64).T
 
 
-def router_margin(x, wr, top_k, zipf_s=0.0):
+def router_margin(x, wr, top_k, zipf_s=0.0, extra=None):
     """Gap between the k-th and (k+1)-th largest router logit per token (how
     close the top-k decision is to a tie; +inf when k = E).  Diagnostic only."""
-    r = np.asarray(x, dtype=np.float64) @ np.asarray(wr, dtype=np.float64).T
-    if zipf_s:
-        r = r + (-zipf_s * np.log(np.arange(wr.shape[0], dtype=np.float64) + 1.0))[None, :]
+    r = router_logits(x, wr, zipf_s, extra)
     if top_k >= r.shape[1]:
         return np.full(r.shape[0], np.inf)
     s = -np.sort(-r, axis=1)
@@ -280,19 +279,22 @@ def token_logits_with_routing(model, layer, h_attn_row, ids, gates):
     return (cfg.logit_scale * _proj(xf, model.embed))[0]
 
 
-def router_logits(x, wr, zipf_s=0.0):
-    """Router logits x Wr^T (+ Zipf bias), float64."""
+def router_logits(x, wr, zipf_s=0.0, extra=None):
+    """Router logits x Wr^T (+ Zipf bias) (+ per-token bias `extra` [n, E]), float64."""
     r = np.asarray(x, dtype=np.float64) @ np.asarray(wr, dtype=np.float64).T
     if zipf_s:
         r = r + (-zipf_s * np.log(np.arange(wr.shape[0], dtype=np.float64) + 1.0))[None, :]
+    if extra is not None:
+        r = r + np.asarray(extra, dtype=np.float64)
     return r
 
 
-def block(model, layer, h, positions, k_prefix, v_prefix, causal, trace=None):
+def block(model, layer, h, positions, k_prefix, v_prefix, causal, trace=None, route_bias=None):
     """One pre-norm transformer block over n tokens.  k_prefix/v_prefix are
     cached keys/values [n_prefix, Hkv, hd] the tokens also attend to.  Returns
     (h_out, k_new, v_new) with k_new/v_new the stored keys/values of the tokens.
-    `trace` (a list) receives the intermediate states for diagnostics."""
+    `trace` (a list) receives the intermediate states for diagnostics;
+    `route_bias` [n, E] is added to the router logits (None: no term)."""
     cfg = model.cfg
     n = h.shape[0]
     hq, hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
@@ -305,10 +307,11 @@ def block(model, layer, h, positions, k_prefix, v_prefix, causal, trace=None):
     o = model.store(attention(q, kk, vv, causal_offset=k_prefix.shape[0] if causal else None))
     h = model.store(h + _proj(o.reshape(n, hq * hd), layer.wo))
     x2 = model.store(rmsnorm(h, cfg.rms_eps))
-    y, ids, w = moe(model, layer, x2)
+    y, ids, w = moe(model, layer, x2, route_bias)
     if trace is not None:
-        trace.append(dict(h_attn=h.copy(), ids=ids, margin=router_margin(x2, layer.wr, cfg.top_k, cfg.zipf_s),
-                          router=router_logits(x2, layer.wr, cfg.zipf_s)))
+        trace.append(dict(h_attn=h.copy(), ids=ids,
+                          margin=router_margin(x2, layer.wr, cfg.top_k, cfg.zipf_s, route_bias),
+                          router=router_logits(x2, layer.wr, cfg.zipf_s, route_bias)))
     h = model.store(h + y)
     if trace is not None:
         trace[-1]["h_out"] = h.copy()
@@ -332,10 +335,11 @@ def encode_prompt(model, prompt):
 
 
 # --- one denoising step ----------------------------------------------------------
-def forward_canvas(model, K, V, canvas, selfcond, trace=None):
+def forward_canvas(model, K, V, canvas, selfcond, trace=None, canvas_id=0):
     """Bidirectional canvas pass.  K, V: prompt cache [L, Hkv, P, hd];
     canvas [256] ids; selfcond [256, d] or None.  Returns float64 logits
-    [256, vocab] and the canvas keys/values written per layer."""
+    [256, vocab] and the canvas keys/values written per layer.  A per-token
+    router bias (model.route_bias) applies its rows of canvas `canvas_id`."""
     cfg = model.cfg
     P = K.shape[2]
     h = model.embed[np.asarray(canvas)].astype(np.float64)
@@ -346,7 +350,10 @@ def forward_canvas(model, K, V, canvas, selfcond, trace=None):
     for l, layer in enumerate(model.layers):
         kp = K[l].transpose(1, 0, 2).astype(np.float64)
         vp = V[l].transpose(1, 0, 2).astype(np.float64)
-        h, k, v = block(model, layer, h, pos, kp, vp, causal=False, trace=trace)
+        rb = getattr(model, "route_bias", None)
+        if rb is not None:
+            rb = rb[l, canvas_id * CANVAS:(canvas_id + 1) * CANVAS]
+        h, k, v = block(model, layer, h, pos, kp, vp, causal=False, trace=trace, route_bias=rb)
         kv_new.append((k, v))
     x = model.store(rmsnorm(h, cfg.rms_eps))
     if trace is not None:
@@ -369,7 +376,7 @@ def denoise_step(model, K, V, canvas, selfcond, step, t, canvas_id=0, prev_amax=
     binary32 values the sampler reads), entropy, sampled tokens, argmax,
     commit mask, next canvas, next self-conditioning, stop flag and count."""
     cfg = model.cfg
-    logits64, _ = forward_canvas(model, K, V, canvas, selfcond, trace=trace)
+    logits64, _ = forward_canvas(model, K, V, canvas, selfcond, trace=trace, canvas_id=canvas_id)
     l32 = logits64.astype(F32)
     T = sp.temperature(t, cfg.temp_start, cfg.temp_end)
     inv_t = F32(1.0) / T

@@ -314,27 +314,28 @@ def test_grouped_gemm_fused_swiglu(M, K, counts, m256):
 
 
 # --- router -----------------------------------------------------------------------------
-@pytest.mark.parametrize("T,d,E,k,zipf", [(256, 2816, 128, 8, 0.0), (77, 1024, 32, 4, 0.0),
-                                          (1024, 1024, 32, 4, 1.1), (40, 512, 100, 5, 0.0)])
-def test_router_kernel(T, d, E, k, zipf):
+@pytest.mark.parametrize("T,d,E,k,zipf,pool", [(256, 2816, 128, 8, 0.0, 0), (77, 1024, 32, 4, 0.0, 0),
+                                               (1024, 1024, 32, 4, 1.1, 0), (40, 512, 100, 5, 0.0, 0),
+                                               (256, 2816, 128, 8, 0.0, 84), (512, 1024, 32, 4, 1.1, 16)])
+def test_router_kernel(T, d, E, k, zipf, pool):
     # top-k ids identical to the oracle's wherever the decision is farther
     # from a tie than the fp32 accumulation error can move it; gates within
-    # 1e-4 of the fp64 softmax
+    # 1e-4 of the fp64 softmax.  pool > 0 adds a per-token bias (beta 2, of
+    # the order of the logit spread, so selection depends on both terms)
     g = np.random.default_rng(T + d + E)
     x = I._bf16_grid(g.standard_normal((T, d)).astype(F32))
     wr = I._bf16_grid((0.02 * g.standard_normal((E, d))).astype(F32))
     bias = None
     if zipf:
         bias = cu((-zipf * np.log(np.arange(E, dtype=np.float64) + 1.0)).astype(F32))
+    tb = I.routing_bias(T, 1, T, E, k, pool, beta=2.0)[0] if pool else None
     ids = torch.zeros((T, k), dtype=torch.int32, device="cuda")
     gate = torch.zeros((T, k), dtype=torch.float32, device="cuda")
-    dg.test_router(bf16_tensor(x), bf16_tensor(wr), ids, gate, bias=bias)
+    dg.test_router(bf16_tensor(x), bf16_tensor(wr), ids, gate, bias=bias, tok_bias=cu(tb) if pool else None)
     gi, gg = host(ids), host(gate)
-    oi, ow = om.router(x, wr, k, zipf_s=zipf)
-    r = x.astype(np.float64) @ wr.astype(np.float64).T
-    if zipf:
-        r += (-zipf * np.log(np.arange(E) + 1.0))[None, :]
-    # fp32 accumulation error bound, plus the binary32 rounding of the bias
+    oi, ow = om.router(x, wr, k, zipf_s=zipf, extra=tb)
+    r = om.router_logits(x, wr, zipf, tb)
+    # fp32 accumulation error bound, plus the binary32 rounding of the biases
     err = 4e-6 * (np.abs(x.astype(np.float64)) @ np.abs(wr.astype(np.float64)).T).max(axis=1) + 1e-6 + 1e-5 * zipf
     srt = -np.sort(-r, axis=1)
     gaps = srt[:, :k] - srt[:, 1:k + 1]                       # adjacent gaps through the (k+1)-th

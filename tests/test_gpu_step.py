@@ -9,6 +9,8 @@ stay within twice that of an oracle whose bf16 storage rounds one value in
 64 to the other neighbour (see storage_noise.py for why no fixed absolute
 bound can hold there); tokens identical wherever the Gumbel-max margin
 exceeds twice the row's logit error."""
+import copy
+
 import numpy as np
 import pytest
 
@@ -186,6 +188,33 @@ def test_tiny_block_autoregressive_generation():
     assert np.allclose(K[:, 0, :, :P_cap], Ko, rtol=1e-4, atol=1e-5)
     assert np.allclose(V[:, 0, :, :P_cap], Vo, rtol=1e-4, atol=1e-5)
     gm.close()
+
+
+def test_tiny_round_with_routing_bias(tiny):
+    # structured per-token router bias (routing-locality workloads): the round
+    # and the distinct experts each layer routed to match the oracle's
+    w, gm, om_ = tiny
+    P = w.prompt_len
+    prompt = I.prompt_ids(w.sample_seed, 1, P, w.vocab)
+    kv = gm.new_kv(1, P)
+    gm.encode_prompt(cu(prompt), kv)
+    Ko, Vo = om.encode_prompt(om_, prompt[0])
+    rb = I.routing_bias(11, w.n_layers, 256, w.n_experts, w.top_k, pool=4, beta=2.0)
+    gm.set_routing_bias(cu(rb))
+    try:
+        canvas = sp.initial_canvas(w.sample_seed, 0, 256, w.vocab)
+        out = step_buffers(w, 1)
+        gm.denoise_step(kv, P, cu(canvas[None]), None, 0, 1.0, out)
+        g = {k: host(v)[0] for k, v in out.items()}
+        touched = gm.touched_experts()
+    finally:
+        gm.set_routing_bias(None)
+    biased = copy.copy(om_)
+    biased.route_bias = rb
+    trace = []
+    r = om.denoise_step(biased, Ko, Vo, canvas, None, 0, F32(1.0), trace=trace)
+    compare_round(g, r, w, 0, 1.0, True)
+    assert touched == [len(np.unique(trace[l]["ids"])) for l in range(w.n_layers)]
 
 
 # --- mid bf16 workload with a synthetic prompt cache -------------------------------------

@@ -381,3 +381,46 @@ def test_generate_chains_blocks_on_the_growing_context():
     # the two blocks start from different noise
     assert not np.array_equal(sp.initial_canvas(w.sample_seed, 0, 256, w.vocab),
                               sp.initial_canvas(w.sample_seed + 1, 0, 256, w.vocab))
+
+
+def test_route_bias_steers_selection_and_keeps_gate_softmax():
+    # per-token router bias (routing-locality workloads): with a bias far above
+    # the logit spread each token selects exactly its preferred experts; the
+    # gates stay the softmax over the selected logits, which a constant shift
+    # of the selected set leaves unchanged; the rows used are the canvas's own
+    w = I.TINY_FP32.replace(n_layers=2)
+    model = om.Model(w)
+    E, k = w.n_experts, w.top_k
+    pool = 4
+    rb = I.routing_bias(5, w.n_layers, 2 * 256, E, k, pool, beta=1000.0)
+    model.route_bias = rb
+    K, V = om.encode_prompt(model, I.prompt_ids(w.sample_seed, 1, 16, w.vocab)[0])
+    canvas = I.canvas_ids(9, 1, w.vocab)[0]
+    for cid in (0, 1):
+        trace = []
+        om.forward_canvas(model, K, V, canvas, None, trace=trace, canvas_id=cid)
+        for l in range(w.n_layers):
+            ids = trace[l]["ids"]
+            pref = rb[l, cid * 256:(cid + 1) * 256] > 0
+            for t in range(256):
+                assert set(ids[t].tolist()) == set(np.nonzero(pref[t])[0].tolist()), (cid, l, t)
+            assert len(np.unique(ids)) == pool
+            # gates (router on the biased logits r, identity weights) equal the
+            # softmax of the unbiased logits over the selected experts
+            r = trace[l]["router"]
+            for t in (0, 100, 255):
+                sel_ids, gates = om.router(r[t:t + 1], np.eye(E), k)
+                base = r[t, sel_ids[0]] - rb[l, cid * 256 + t, sel_ids[0]]
+                ex = np.exp(base - base.max())
+                assert np.allclose(gates[0], ex / ex.sum(), rtol=1e-12)
+
+
+def test_zero_route_bias_is_no_bias():
+    w = I.TINY_FP32.replace(n_layers=1)
+    model = om.Model(w)
+    K, V = om.encode_prompt(model, I.prompt_ids(w.sample_seed, 1, 16, w.vocab)[0])
+    canvas = I.canvas_ids(9, 1, w.vocab)[0]
+    ref, _ = om.forward_canvas(model, K, V, canvas, None)
+    model.route_bias = np.zeros((1, 256, w.n_experts), dtype=np.float32)
+    got, _ = om.forward_canvas(model, K, V, canvas, None)
+    assert np.array_equal(ref, got)

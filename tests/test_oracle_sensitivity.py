@@ -71,7 +71,7 @@ def test_forward_mistakes_are_caught(micro, monkeypatch, name):
         monkeypatch.setattr(om, "block", _block_no_residual)
     elif name == "moe_slot_weights":
         orig = om.router
-        monkeypatch.setattr(om, "router", lambda x, wr, k, z=0.0: (orig(x, wr, k, z)[0], orig(x, wr, k, z)[1][:, ::-1]))
+        monkeypatch.setattr(om, "router", lambda x, wr, k, z=0.0, extra=None: (orig(x, wr, k, z, extra)[0], orig(x, wr, k, z, extra)[1][:, ::-1]))
     elif name == "rmsnorm_eps_inside":
         monkeypatch.setattr(om, "rmsnorm", lambda h, eps: h / (np.sqrt(np.mean(h * h, -1, keepdims=True)) + 1e-2))
     elif name == "logit_scale":
