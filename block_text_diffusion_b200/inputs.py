@@ -47,6 +47,7 @@ class Workload:
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
     zipf_s: float = 0.0          # 0 = no router bias
+    sample_topk: int = 0         # 0 = exact sampling; K = draw among the K largest logits
     temp_start: float = 0.8
     temp_end: float = 0.4
     max_steps: int = 48

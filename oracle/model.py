@@ -370,6 +370,19 @@ def self_condition(model, probs):
     return model.store(_proj(u, model.wsc))
 
 
+def self_condition_topk(model, ids, weights):
+    """self_condition for a top-k-truncated distribution: p is zero outside
+    the candidates ids [256, K] and holds the binary32 weights [256, K] on
+    them, so p E is the weighted sum of K embedding rows per position."""
+    p = model.store(np.asarray(weights, dtype=np.float64))
+    n, K = p.shape
+    u = np.zeros((n, model.cfg.d_model))
+    for j in range(K):
+        u += p[:, j:j + 1] * model.embed[np.asarray(ids)[:, j]].astype(np.float64)
+    u = model.store(u)
+    return model.store(_proj(u, model.wsc))
+
+
 def denoise_step(model, K, V, canvas, selfcond, step, t, canvas_id=0, prev_amax=None, max_steps=None,
                  trace=None):
     """One round for one canvas.  Returns a dict with logits (float64 and the
@@ -380,17 +393,22 @@ def denoise_step(model, K, V, canvas, selfcond, step, t, canvas_id=0, prev_amax=
     l32 = logits64.astype(F32)
     T = sp.temperature(t, cfg.temp_start, cfg.temp_end)
     inv_t = F32(1.0) / T
-    st = sp.sampler_rows(l32, inv_t, cfg.sample_seed, canvas_id, step)
+    K = getattr(cfg, "sample_topk", 0)
+    if K:
+        st = sp.sampler_rows_topk(l32, K, inv_t, cfg.sample_seed, canvas_id, step)
+    else:
+        st = sp.sampler_rows(l32, inv_t, cfg.sample_seed, canvas_id, step)
     tok = st["tokens"]
     mask = sp.commit_mask(st["H"], cfg.commit_mode, cfg.commit_bound)
     nxt = sp.next_canvas(tok, mask, cfg.sample_seed, canvas_id, step, cfg.vocab)
     n_steps = cfg.max_steps if max_steps is None else max_steps
     stop = sp.stop_decision(st["H"], mask, st["amax"], prev_amax, step, n_steps,
                             cfg.stop_mode, cfg.stop_bound)
-    s_next = self_condition(model, st["p"])
+    s_next = self_condition_topk(model, st["cand_ids"], st["cand_w"]) if K else self_condition(model, st["p"])
     return dict(logits64=logits64, logits=l32, H=st["H"], tokens=tok, amax=st["amax"],
                 commit=mask, canvas_next=nxt, selfcond_next=s_next, stop=stop,
-                n_committed=int(mask.sum()), probs=st["p"])
+                n_committed=int(mask.sum()), probs=st.get("p"), cand_ids=st.get("cand_ids"),
+                cand_w=st.get("cand_w"))
 
 
 def generate_block(model, K, V, canvas_id=0, max_steps=None):

@@ -161,6 +161,73 @@ def sampler_rows(logits, inv_t, seed, canvas_id, step):
     return st
 
 
+# --- top-k-truncated sampling (explainer section 九) ---------------------------
+# The explainer names top-k truncation as the sampler optimisation for large
+# batches that the release lacks.  Reading: with truncation K, the token is the
+# Gumbel-max draw restricted to the K largest logits (a draw from softmax(l/T)
+# renormalised over them), each candidate keeping the noise g_v it has in the
+# exact sampler; the self-conditioning input is the untempered distribution
+# renormalised over the same candidates; entropy, argmax and the commit / stop
+# decisions stay those of the full distribution.
+def topk_ids(logits_row, K: int) -> np.ndarray:
+    """Indices of the K largest binary32 logits of a row, by value descending,
+    ties to the lower index (every index when K >= V)."""
+    l = np.asarray(logits_row, dtype=F32)
+    order = np.lexsort((np.arange(l.size), -l.astype(np.float64)))
+    return order[:K].astype(np.int32)
+
+
+def gumbel_noise_at(ids, seed: int, canvas_id: int, position: int, step: int) -> np.ndarray:
+    """g_v of gumbel_noise at the given vocabulary ids only (same Philox
+    counter (v>>2, position, step, stream 0) and word v&3)."""
+    k0, k1 = nm.seed_key(seed, canvas_id)
+    ids = np.asarray(ids, dtype=np.uint32)
+    w = nm.philox4x32_10(ids >> np.uint32(2), np.uint32(position), np.uint32(step),
+                         np.uint32(nm.STREAM_GUMBEL), k0, k1)
+    words = np.stack(w, axis=1)[np.arange(ids.size), (ids & np.uint32(3)).astype(np.int64)]
+    u = nm.uniform_open(words)
+    return -nm.log_f32(-nm.log_f32(u))
+
+
+def topk_sample(logits_row, K: int, inv_t, seed: int, canvas_id: int, position: int, step: int):
+    """Top-k-truncated draw of one row.  Returns (token, ids, weights):
+    ids = topk_ids(l, K); token = the id of the largest key l_v (1/T) + g_v
+    among them (binary32, the lowest id on equal keys); weights = the
+    untempered probabilities renormalised over the candidates, binary32:
+    e_j = exp(l_j - m) (own exp, m the row maximum), s = e_0 + e_1 + ...
+    accumulated in candidate order, w_j = e_j (1/s)."""
+    l = np.asarray(logits_row, dtype=F32)
+    ids = topk_ids(l, K)
+    lc = l[ids]
+    key = lc * F32(inv_t) + gumbel_noise_at(ids, seed, canvas_id, position, step)
+    token = int(ids[key == key.max()].min())
+    e = nm.exp_f32(lc - lc[0])
+    s = F32(0.0)
+    for x in e:
+        s = F32(s + x)
+    w = (e * (F32(1.0) / s)).astype(F32)
+    return token, ids, w
+
+
+def sampler_rows_topk(logits, K: int, inv_t, seed, canvas_id, step):
+    """sampler_rows with top-k-truncated tokens: the full-distribution
+    statistics (H, amax, S, U) plus tokens, candidate ids [R, K] and
+    candidate weights [R, K] (no dense probabilities)."""
+    st = sampler_rows(logits, inv_t, seed, canvas_id, step)
+    st.pop("p", None)
+    R = logits.shape[0]
+    toks = np.empty(R, dtype=np.int32)
+    ids, ws = [], []
+    for i in range(R):
+        toks[i], c, w = topk_sample(logits[i], K, inv_t, seed, canvas_id, i, step)
+        ids.append(c)
+        ws.append(w)
+    st["tokens"] = toks
+    st["cand_ids"] = np.stack(ids)
+    st["cand_w"] = np.stack(ws)
+    return st
+
+
 # --- commit / re-noise / stop (explainer section 四) -----------------------------
 def fixed_entropy(H) -> np.ndarray:
     """Per-position entropy in Q32 fixed point: trunc(H * 2^32) (exact

@@ -424,3 +424,19 @@ def test_zero_route_bias_is_no_bias():
     model.route_bias = np.zeros((1, 256, w.n_experts), dtype=np.float32)
     got, _ = om.forward_canvas(model, K, V, canvas, None)
     assert np.array_equal(ref, got)
+
+
+def test_topk_self_condition_is_dense_self_condition_of_the_sparse_distribution():
+    # p E with p zero outside the candidates equals the weighted sum of the
+    # candidates' embedding rows
+    for w in (I.TINY_FP32.replace(n_layers=1), I.TINY_FP32.replace(n_layers=1, dtype=I.DTYPE_BF16)):
+        model = om.Model(w)
+        g = np.random.default_rng(3)
+        K = 7
+        ids = np.stack([g.choice(w.vocab, size=K, replace=False) for _ in range(256)]).astype(np.int32)
+        wt = g.dirichlet(np.ones(K), size=256).astype(F32)
+        dense = np.zeros((256, w.vocab), F32)
+        dense[np.arange(256)[:, None], ids] = wt
+        a = om.self_condition_topk(model, ids, wt)
+        b = om.self_condition(model, dense)
+        assert np.allclose(a, b, rtol=1e-6, atol=1e-9)

@@ -188,3 +188,68 @@ def test_next_canvas_keeps_committed_renoises_rest():
     fresh = sp.renoise_tokens(8, 1, 4, 256, 5000)
     assert np.array_equal(nxt[mask == 1], tok[mask == 1])
     assert np.array_equal(nxt[mask == 0], fresh[mask == 0])
+
+
+# --- top-k-truncated sampling ---------------------------------------------------------
+@pytest.mark.parametrize("kind", ["normal", "ties", "flat", "peaked"])
+def test_topk_ids_brute_force(kind):
+    l = I.logits(11, 6, 64, kind, 2.0)
+    for K in (1, 5, 17, 64, 100):
+        for r in range(l.shape[0]):
+            ref = sorted(range(64), key=lambda v: (-float(l[r, v]), v))[:K]
+            assert sp.topk_ids(l[r], K).tolist() == ref
+
+
+def test_topk_at_full_vocab_is_the_exact_sampler():
+    for kind in ("normal", "ties", "flat", "mixed"):
+        l = I.logits(12, 8, 512, kind, 3.0)
+        inv_t = F32(1.0) / F32(0.65)
+        for r in range(l.shape[0]):
+            tok, _, _ = sp.topk_sample(l[r], 512, inv_t, 5, 1, r, 7)
+            assert tok == sp.gumbel_argmax(l[r], inv_t, 5, 1, r, 7)
+
+
+def test_topk_token_equals_exact_when_exact_winner_is_a_candidate():
+    # Gumbel-max over a subset that holds the overall winner picks that winner;
+    # otherwise the draw is still one of the candidates
+    l = I.logits(13, 64, 2048, "normal", 1.0)
+    inv_t = F32(1.0) / F32(0.8)
+    hits = 0
+    for r in range(l.shape[0]):
+        exact = sp.gumbel_argmax(l[r], inv_t, 9, 0, r, 2)
+        for K in (4, 32):
+            tok, ids, _ = sp.topk_sample(l[r], K, inv_t, 9, 0, r, 2)
+            assert tok in ids.tolist()
+            if exact in ids.tolist():
+                assert tok == exact
+                hits += 1
+    assert hits > 0
+
+
+def test_topk_frequencies_match_truncated_softmax():
+    # the truncated draw is softmax(l/T) renormalised over the K largest logits
+    V, K = 8, 3
+    l = np.array([0.0, 1.0, -1.0, 0.5, 2.0, -3.0, 0.25, 1.5], F32)
+    T = F32(0.7)
+    inv_t = F32(1.0) / T
+    counts = np.zeros(V)
+    for s in range(40):
+        for pos in range(256):
+            counts[sp.topk_sample(l, K, inv_t, 42, 3, pos, s)[0]] += 1
+    ids = [4, 7, 1]
+    assert counts.sum() == counts[ids].sum()
+    lt = l[ids].astype(np.float64) / float(T)
+    p = np.exp(lt - lt.max())
+    p /= p.sum()
+    assert stats.chisquare(counts[ids], p * counts.sum()).pvalue > 1e-4
+
+
+def test_topk_weights_are_the_renormalised_untempered_softmax():
+    l = I.logits(14, 5, 4096, "mixed", 4.0)
+    for r in range(l.shape[0]):
+        _, ids, w = sp.topk_sample(l[r], 50, F32(2.0), 1, 0, r, 0)
+        x = l[r, ids].astype(np.float64)
+        ref = np.exp(x - x.max())
+        ref /= ref.sum()
+        assert np.allclose(w, ref, rtol=2e-6, atol=1e-12)
+        assert abs(float(w.astype(np.float64).sum()) - 1.0) < 50 * 2 ** -23
