@@ -42,6 +42,8 @@ def parse():
                     help="override the round budget (short runs for profiler launch lists)")
     ap.add_argument("--no-fast-converging", action="store_true",
                     help="skip the committed-tokens measurement on the fast-converging workload")
+    ap.add_argument("--topk-study", action="store_true",
+                    help="also compare exact and top-k-truncated sampling at batch 32 (mid workload)")
     ap.add_argument("--routing-study", action="store_true",
                     help="also sweep a structured router bias over expert-pool sizes (routing locality)")
     return ap.parse_args()
@@ -263,6 +265,9 @@ def run_ours(a):
     study = None
     if a.routing_study:
         study = routing_study(dg, I, torch, model, w, kv, B, P, block, steps)
+    topk = None
+    if a.topk_study and world == 1:
+        topk = topk_study(dg, I, torch)
 
     # committed tokens on the fast-converging workload (logit scale 16), where
     # random-init weights still commit: single-GPU runs only
@@ -323,6 +328,7 @@ def run_ours(a):
                 "includes": "prompt H2D, causal prompt encode, block loop, result D2H"},
         "fast_converging": fast,
         "routing_study": study,
+        "topk_study": topk,
         "gpu_launches": int(n_rounds / world * (kper + 1) + a.steps * (1 + 3)) * world,
         "clocks": clk.summary(),
     }
@@ -402,6 +408,46 @@ def routing_study(dg, I, torch, model, w, kv, B, P, block, steps, pools=(8, 16, 
         out.append({"pool": pool, "touched_mean": sum(touched) / len(touched), "ms_per_round": ms_round,
                     "roof_ms": roof, "frac": roof / ms_round, "expert_ms_per_round": (gu_ms + dn_ms) / 2,
                     "gate_up_gbs": gu_gbs, "gate_up_frac": gu_gbs / hbm})
+    return out
+
+
+def topk_study(dg, I, torch, K=64, B=32, reps=2):
+    """Exact vs top-k-truncated sampling on the Zipf-routed batch workload
+    (mid architecture, 2048-token prompts) at B canvases: ms per round of the
+    device block loop, and the sampler and self-conditioning phases of single
+    rounds (CUDA events around each launch)."""
+    base = I.BATCH_ZIPF
+    P = base.prompt_len
+    stream = torch.cuda.current_stream()
+    prompt = torch.from_numpy(I.prompt_ids(base.sample_seed, B, P, base.vocab)).cuda()
+    out = {"workload": base.name, "canvases": B, "K": K}
+    for name, w in (("exact", base), ("topk", base.replace(sample_topk=K))):
+        model = dg.Model(w, max_canvases=B, max_prompt=P)
+        kv = model.new_kv(B, P)
+        model.encode_prompt(prompt, kv)
+        z = lambda *shape: torch.zeros(shape, dtype=torch.int32, device="cuda")
+        canvas, steps, ncom = z(B, 256), z(B), z(B)
+        model.generate_block(kv, B, P, canvas, steps, ncom)
+        torch.cuda.synchronize()
+        rounds = torch.zeros((), dtype=torch.int64, device="cuda")
+        committed = torch.zeros((), dtype=torch.int64, device="cuda")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            model.generate_block(kv, B, P, canvas, steps, ncom)
+            rounds += steps.max()          # the loop runs until the last canvas stops
+            committed += ncom.sum()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        model.sync_status()
+        n_r = max(1, int(rounds.item()))
+        prof = model.profile_step(kv, B, P, reps=2)
+        ph = {k: v[0] / 2 for k, v in prof.items() if v[1]}
+        out[name] = {"ms_per_round": e0.elapsed_time(e1) / n_r,
+                     "committed_per_round": int(committed.item()) / n_r,
+                     "sampler_ms": ph.get("sampler", 0.0),
+                     "selfcond_ms": ph.get("selfcond_gemm", 0.0) + ph.get("selfcond_round", 0.0)}
+        model.close()
     return out
 
 

@@ -37,7 +37,7 @@ class Config(ctypes.Structure):
                 ("temp_end", ctypes.c_float), ("max_steps", ctypes.c_int32), ("commit_mode", ctypes.c_int32),
                 ("commit_bound", ctypes.c_float), ("stop_mode", ctypes.c_int32), ("stop_bound", ctypes.c_float),
                 ("canvas_len", ctypes.c_int32), ("max_canvases", ctypes.c_int32), ("max_prompt", ctypes.c_int32),
-                ("sample_seed", ctypes.c_uint64)]
+                ("sample_seed", ctypes.c_uint64), ("sample_topk", ctypes.c_int32)]
 
 
 class StepOut(ctypes.Structure):
@@ -69,6 +69,8 @@ def lib():
             "dg_test_math": ([I32, P, P, I64, U64, U32, P], I32),
             "dg_test_philox": ([P, P, I64, P], I32),
             "dg_test_sampler": ([P, I32, I32, I32, U64, I32, F, F, F, P, P, P, P, P, P, I32, P], I32),
+            "dg_test_sampler_topk": ([P, I32, I32, I32, U64, I32, F, F, F, I32, P, P, P, P, P, P, P, I32, P], I32),
+            "dg_test_sc_gather": ([P, P, I32, I32, P, I32, I32, P, P], I32),
             "dg_test_commit": ([P, P, P, P, I32, I32, U64, I32, I32, I32, F, I32, F, P, P, P, P, P], I32),
             "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, I32, P], I32),
             "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
@@ -112,7 +114,7 @@ def make_config(w, max_canvases=None, max_prompt=None) -> Config:
     return Config(w.n_layers, w.d_model, w.n_heads, w.n_kv_heads, w.head_dim, w.n_experts, w.top_k, w.d_ff,
                   w.vocab, w.dtype, w.logit_scale, w.rope_theta, w.rms_eps, w.zipf_s, w.temp_start, w.temp_end,
                   w.max_steps, w.commit_mode, w.commit_bound, w.stop_mode, w.stop_bound, 256,
-                  max_canvases or w.batch, max_prompt or w.prompt_len, w.sample_seed)
+                  max_canvases or w.batch, max_prompt or w.prompt_len, w.sample_seed, w.sample_topk)
 
 
 class Model:
@@ -243,6 +245,25 @@ def test_sampler(logits, positions, seed, step, t, temp_start, temp_end, H, tok,
     _check(lib().dg_test_sampler(_ptr(logits), rows, vocab, positions, seed, step, float(t), float(temp_start),
                                  float(temp_end), _ptr(H), _ptr(tok), _ptr(amax), _ptr(s_q), _ptr(u_q),
                                  _ptr(probs), bf, _stream(stream)), "dg_test_sampler")
+
+
+def test_sampler_topk(logits, positions, seed, step, t, temp_start, temp_end, K, H, tok, amax, cand_ids, cand_w,
+                      s_q=None, u_q=None, stream=None):
+    import torch
+    rows, vocab = logits.shape
+    bf = 1 if cand_w.dtype == torch.bfloat16 else 0
+    _check(lib().dg_test_sampler_topk(_ptr(logits), rows, vocab, positions, seed, step, float(t), float(temp_start),
+                                      float(temp_end), K, _ptr(H), _ptr(tok), _ptr(amax), _ptr(s_q), _ptr(u_q),
+                                      _ptr(cand_ids), _ptr(cand_w), bf, _stream(stream)), "dg_test_sampler_topk")
+
+
+def test_sc_gather(cand_ids, cand_w, emb, u, stream=None):
+    import torch
+    rows, K = cand_ids.shape
+    d = emb.shape[1]
+    _check(lib().dg_test_sc_gather(_ptr(cand_ids), _ptr(cand_w), rows, K, _ptr(emb), d,
+                                   1 if emb.dtype == torch.bfloat16 else 0, _ptr(u), _stream(stream)),
+           "dg_test_sc_gather")
 
 
 def test_commit(H, tok, amax, prev_amax, vocab, seed, step, max_steps, commit_mode, commit_bound, stop_mode,

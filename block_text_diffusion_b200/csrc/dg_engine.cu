@@ -157,6 +157,9 @@ struct dg_model {
 
   void *h = nullptr, *x = nullptr, *q = nullptr, *o = nullptr, *xp = nullptr, *act = nullptr;
   void *probs = nullptr, *u = nullptr, *sc = nullptr;
+  // top-k-truncated sampling: per position the K candidate ids and weights
+  int* cand_ids = nullptr;
+  void* cand_w = nullptr;
   BMaps tm_x, tm_o, tm_xp, tm_act, tm_probs, tm_u;   // activation (B) operands
   float* ws = nullptr;
   float *o_part = nullptr, *lse_part = nullptr;
@@ -437,6 +440,7 @@ bool config_ok(const dg_config& c) {
   if (c.commit_mode != DG_COMMIT_THRESH && c.commit_mode != DG_COMMIT_EB) return false;
   if (c.stop_mode != DG_STOP_MEAN && c.stop_mode != DG_STOP_EB) return false;
   if (!(c.logit_scale == c.logit_scale) || !(c.rope_theta > 0.0f) || !(c.rms_eps >= 0.0f)) return false;
+  if (c.sample_topk < 0 || c.sample_topk > kTopkMax || c.sample_topk > c.vocab) return false;
   return true;
 }
 
@@ -501,7 +505,7 @@ dg_status build_maps(dg_model* m) {
   ok &= bmaps(&m->tm_o, m->o, Tw, (uint64_t)m->hq * m->hd);
   ok &= bmaps(&m->tm_xp, m->xp, Tk, d);
   ok &= bmaps(&m->tm_act, m->act, Tk, m->ff);
-  ok &= bmaps(&m->tm_probs, m->probs, m->T_cap, V);
+  if (m->probs) ok &= bmaps(&m->tm_probs, m->probs, m->T_cap, V);
   ok &= bmaps(&m->tm_u, m->u, m->T_cap, d);
   return ok ? DG_OK : DG_ERR_CUDA;
 }
@@ -777,7 +781,10 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     sa.temp_start = m->c.temp_start; sa.temp_end = m->c.temp_end; sa.state = m->st;
     sa.step_override = io.step_override; sa.t_override = io.t_override;
     sa.H = io.entropy; sa.tok = io.tokens; sa.amax = io.argmax;
-    CU_TRY(launch_sampler<T>(sa, io.selfcond_next ? (T*)m->probs : nullptr, Tn, s, g_use_pdl));
+    if (m->c.sample_topk > 0)
+      CU_TRY(launch_sampler_topk<T>(sa, m->c.sample_topk, m->cand_ids, (T*)m->cand_w, Tn, s, g_use_pdl));
+    else
+      CU_TRY(launch_sampler<T>(sa, io.selfcond_next ? (T*)m->probs : nullptr, Tn, s, g_use_pdl));
   }
   // commit / re-noise / stop
   {
@@ -798,7 +805,13 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     launch_pdl(k_commit, B, 256, 0, s, ca);
   }
   // self-conditioning for the next round: s' = round(round(p E) W_sc^T)
-  if (io.selfcond_next) {
+  const long long n_sc = (long long)Tn * d;
+  if (io.selfcond_next && m->c.sample_topk > 0) {
+    // truncated distribution: p E is a weighted sum of K embedding rows
+    { LaunchScope ls(m, s, PH_SC_GEMM);
+      launch_pdl(k_sc_gather<T>, Tn, 256, 0, s, (const int*)m->cand_ids, (const T*)m->cand_w, m->c.sample_topk,
+                 (const T*)m->emb, d, (T*)m->u); }
+  } else if (io.selfcond_next) {
     GemmCall sc;
     sc.tA = &m->tm_ET; sc.tB = &m->tm_probs; sc.A32 = (const float*)m->embT; sc.B32 = (const float*)m->probs;
     sc.lda = V; sc.ldb = V; sc.M = d; sc.K = V; sc.N = Tn; sc.out = m->ws; sc.ldo = d; sc.bn = dense_bn(Tn);
@@ -814,10 +827,12 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
       sc.split_stride = (long long)Tn * d;
     }
     DG_TRY(gemm(m, sc, PH_SC_GEMM, s));
-    const long long n = (long long)Tn * d;
     { LaunchScope ls(m, s, PH_SC_ROUND);
-      launch_pdl(k_sum_round<T>, std::min(cdiv(n, 256), kSMs * 16), 256, 0, s, 
-          (T*)m->u, m->ws, sc.split_stride, std::min(sc.splits, cdiv(V, 64)), n); }
+      launch_pdl(k_sum_round<T>, std::min(cdiv(n_sc, 256), kSMs * 16), 256, 0, s,
+          (T*)m->u, m->ws, sc.split_stride, std::min(sc.splits, cdiv(V, 64)), n_sc); }
+  }
+  if (io.selfcond_next) {
+    const long long n = n_sc;
     GemmCall s2;
     s2.tA = &m->tm_Wsc; s2.tB = &m->tm_u; s2.A32 = (const float*)m->Wsc; s2.B32 = (const float*)m->u;
     s2.lda = d; s2.ldb = d; s2.M = d; s2.K = d; s2.N = Tn; s2.out = m->ws; s2.ldo = d; s2.bn = dense_bn(Tn);
@@ -1056,7 +1071,12 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   A(&m->o, Tw * nq * es);
   A(&m->xp, Tk * d * es);
   A(&m->act, Tk * m->ff * es);
-  A(&m->probs, (size_t)m->T_cap * V * es);
+  if (cfg->sample_topk > 0) {
+    A((void**)&m->cand_ids, (size_t)m->T_cap * cfg->sample_topk * sizeof(int));
+    A(&m->cand_w, (size_t)m->T_cap * cfg->sample_topk * es);
+  } else {
+    A(&m->probs, (size_t)m->T_cap * V * es);
+  }
   A(&m->u, (size_t)m->T_cap * d * es);
   A(&m->sc, (size_t)m->T_cap * d * es);
   A((void**)&m->ws, m->ws_elems * sizeof(float));
@@ -1119,7 +1139,7 @@ int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   // 4 self-cond.
   const int per_layer = (m->bf ? 12 : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
   return per_layer * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
-         4 /*self-conditioning*/;
+         (m->c.sample_topk > 0 ? 3 : 4) /*self-conditioning*/;
 }
 
 dg_status dg_encode_prompt(dg_model* m, const int32_t* prompt, int32_t B, int32_t P, void* kv, void* stream) {

@@ -838,6 +838,263 @@ cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cuda
 }
 
 // ---------------------------------------------------------------------------
+// Top-k-truncated sampler (the optimisation the DiffusionGemma technical-
+// report explainer, section 九, names for large batches).  Per row: the K
+// largest logits (value descending, ties to the lower index) are the
+// candidates; the token is the Gumbel-max draw among them with the exact
+// sampler's noise g_v (Philox counter (v>>2, position, round, stream 0));
+// the candidate weights w_j = e_j (1/s), e_j = exp(l_j - m), s = e_0 + e_1 +
+// ... in candidate order, feed self-conditioning.  Entropy, row argmax and
+// the Q40 sums are those of the full row, as in k_sampler.
+//
+// Same cluster layout as k_sampler (kSampCta CTAs per row).  Pass 1 keeps
+// the slice's K best in a shared candidate buffer: every value above the
+// current threshold (the K-th best so far) is appended; when the next
+// iteration could overflow the buffer it is sorted and cut back to K.
+// Iterations visit increasing indices, so a later value equal to the
+// threshold can never displace a kept one and a strict comparison suffices.
+// Rank 0 merges the kSampCta lists through distributed shared memory and
+// draws among the row's K candidates: Philox runs on K values per row, not V.
+// ---------------------------------------------------------------------------
+constexpr int kTopkMax = 256;      // largest supported truncation K
+constexpr int kCandCap = 2048;     // candidate buffer per CTA (>= kSampCta * kTopkMax)
+
+// Sort cv/ci[0, n) best first -- value descending, index ascending -- by a
+// bitonic network over the next power of two (padding with (-inf, INT_MAX),
+// which ranks after every real entry).  Block-wide; n <= kCandCap.
+__device__ __forceinline__ void cand_sort(float* cv, int* ci, int n) {
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  for (int i = n + (int)threadIdx.x; i < n2; i += blockDim.x) { cv[i] = -INFINITY; ci[i] = 0x7fffffff; }
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int p = i ^ j;
+        if (p > i) {
+          const float va = cv[i], vb = cv[p];
+          const int ia = ci[i], ib = ci[p];
+          const bool b_ahead = vb > va || (vb == va && ib < ia);
+          if (((i & k) == 0) == b_ahead) { cv[i] = vb; cv[p] = va; ci[i] = ib; ci[p] = ia; }
+        }
+      }
+      __syncthreads();
+    }
+}
+
+template <typename T>
+__global__ void __cluster_dims__(kSampCta, 1, 1) __launch_bounds__(kSampThreads)
+k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__ cand_w) {
+  pdl_enter();
+  __shared__ SampPart part;
+  __shared__ ArgBest red_m[32], red_g[32];
+  __shared__ long long red_s[32], red_u[32];
+  __shared__ float cv[kCandCap];
+  __shared__ int ci[kCandCap];
+  __shared__ float ew[kTopkMax];
+  __shared__ int s_cnt, s_have;
+  __shared__ float s_tau, s_inv;
+  uint32_t rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  const long long row = blockIdx.x / kSampCta;
+  const int canvas = (int)(row / a.positions), pos = (int)(row % a.positions);
+  const int step = a.step_override >= 0 ? a.step_override : a.state->step;
+  const float t = a.step_override >= 0 ? a.t_override : a.state->t;
+  const float temp = __fadd_rn(a.temp_end, __fmul_rn(__fsub_rn(a.temp_start, a.temp_end), t));
+  const float inv_t = __fdiv_rn(1.0f, temp);
+  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32) ^ (uint32_t)canvas;
+  const int n4 = a.vocab / (4 * kSampCta);
+  const int g0 = (int)rank * n4;
+  const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab) + g0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+
+  // pass 1: row max / argmax and the slice's K best
+  if (threadIdx.x == 0) { s_cnt = 0; s_have = 0; s_tau = -INFINITY; }
+  __syncthreads();
+  ArgBest bm{-INFINITY, -1};
+  for (int base = 0; base < n4; base += blockDim.x) {
+    const int cnt = s_cnt;
+    __syncthreads();                       // every thread has read cnt before any append
+    if (cnt + 4 * (int)blockDim.x > kCandCap) {
+      cand_sort(cv, ci, cnt);
+      if (threadIdx.x == 0) {
+        s_cnt = min(cnt, K);
+        s_have = cnt >= K;
+        s_tau = cnt >= K ? cv[K - 1] : -INFINITY;
+      }
+      __syncthreads();
+    }
+    const bool have = s_have != 0;
+    const float tau = s_tau;
+    const int i = base + (int)threadIdx.x;
+    if (i < n4) {
+      const float4 l = l4[i];
+      const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = (g0 + i) * 4 + j;
+        bm = arg_better(bm, ArgBest{lv[j], v});
+        if (!have || lv[j] > tau) {
+          const int slot = atomicAdd(&s_cnt, 1);
+          if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = v; }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  {
+    const int cnt = min(s_cnt, kCandCap);
+    __syncthreads();
+    cand_sort(cv, ci, cnt);
+    if (threadIdx.x == 0) s_cnt = min(cnt, K);
+  }
+  bm = warp_argmax(bm);
+  if (lane == 0) red_m[warp] = bm;
+  __syncthreads();
+  if (warp == 0) {
+    ArgBest x = lane < nw ? red_m[lane] : ArgBest{-INFINITY, -1};
+    x = warp_argmax(x);
+    if (lane == 0) part.m = x;
+  }
+  cluster_sync_all();
+  ArgBest M{-INFINITY, -1};
+  for (int r = 0; r < kSampCta; ++r) {
+    const SampPart* pr = cluster_peer(&part, r);
+    M = arg_better(M, ArgBest{pr->m.v, pr->m.i});
+  }
+  const float m = M.v;
+
+  if (rank == 0) {
+    // merge the clusters' lists: rank r's K best go to [r K, (r+1) K)
+    for (int r = 1; r < kSampCta; ++r) {
+      const float* pv = cluster_peer(cv, r);
+      const int* pi = cluster_peer(ci, r);
+      const int pc = *cluster_peer(&s_cnt, r);
+      for (int j = threadIdx.x; j < K; j += blockDim.x) {
+        cv[r * K + j] = j < pc ? pv[j] : -INFINITY;
+        ci[r * K + j] = j < pc ? pi[j] : 0x7fffffff;
+      }
+    }
+    for (int j = s_cnt + (int)threadIdx.x; j < K; j += blockDim.x) { cv[j] = -INFINITY; ci[j] = 0x7fffffff; }
+    __syncthreads();
+    cand_sort(cv, ci, kSampCta * K);
+    // Gumbel-max among the candidates; candidate weights
+    ArgBest bg{-INFINITY, -1};
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      const int v = ci[j];
+      const uint4 w = philox4x32_10(make_uint4((uint32_t)v >> 2, (uint32_t)pos, (uint32_t)step, STREAM_GUMBEL),
+                                    k0, k1);
+      const uint32_t word = (v & 3) == 0 ? w.x : (v & 3) == 1 ? w.y : (v & 3) == 2 ? w.z : w.w;
+      const float key = __fadd_rn(__fmul_rn(cv[j], inv_t), gumbel_of(word));
+      bg = arg_better(bg, ArgBest{key, v});
+      ew[j] = dg_expf(__fsub_rn(cv[j], m));
+    }
+    bg = warp_argmax(bg);
+    if (lane == 0) red_g[warp] = bg;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      ArgBest G{-INFINITY, -1};
+      for (int w = 0; w < nw; ++w) G = arg_better(G, red_g[w]);
+      a.tok[row] = G.i;
+      a.amax[row] = M.i;
+      float sum = 0.0f;
+      for (int j = 0; j < K; ++j) sum = __fadd_rn(sum, ew[j]);
+      s_inv = __fdiv_rn(1.0f, sum);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+      cand_ids[row * K + j] = ci[j];
+      cand_w[row * K + j] = from_f<T>(__fmul_rn(ew[j], s_inv));
+    }
+  }
+
+  // pass 2: S, U of the full row (as in k_sampler)
+  long long sq = 0, uq = 0;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 l = l4[i];
+    const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float dlt = __fsub_rn(lv[j], m);
+      const float e = dg_expf(dlt);
+      sq += q40_trunc(e);
+      uq += q40_trunc(__fmul_rn(e, dlt));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    uq += __shfl_xor_sync(0xffffffffu, uq, o);
+  }
+  if (lane == 0) { red_s[warp] = sq; red_u[warp] = uq; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long S = 0, U = 0;
+    for (int w = 0; w < nw; ++w) { S += red_s[w]; U += red_u[w]; }
+    part.s = S;
+    part.u = U;
+  }
+  cluster_sync_all();
+  long long S = 0, U = 0;
+  for (int r = 0; r < kSampCta; ++r) {
+    const SampPart* pr = cluster_peer(&part, r);
+    S += pr->s;
+    U += pr->u;
+  }
+  // no CTA may leave while another still reads its shared memory
+  cluster_sync_all();
+  if (rank == 0 && threadIdx.x == 0) {
+    const float sf = __ll2float_rn(S), uf = __ll2float_rn(U);
+    a.H[row] = __fsub_rn(dg_logf(__fmul_rn(sf, 9.094947017729282e-13f)), __fdiv_rn(uf, sf));
+    if (a.s_q) a.s_q[row] = S;
+    if (a.u_q) a.u_q[row] = U;
+  }
+}
+
+template <typename T>
+cudaError_t launch_sampler_topk(const SamplerArgs& sa, int K, int* cand_ids, T* cand_w, long long rows,
+                                cudaStream_t s, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * kSampCta));
+  cfg.blockDim = dim3(kSampThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_sampler_topk<T>, sa, K, cand_ids, cand_w);
+}
+
+// Self-conditioning input of a truncated distribution: u[t] = sum_j w[t][j]
+// E[id[t][j]] (fp32, candidate order), stored in T.  One CTA per position.
+template <typename T>
+__global__ void k_sc_gather(const int* __restrict__ ids, const T* __restrict__ w, int K,
+                            const T* __restrict__ emb, int d, T* __restrict__ u) {
+  pdl_enter();
+  __shared__ int s_id[kTopkMax];
+  __shared__ float s_w[kTopkMax];
+  const long long t = blockIdx.x;
+  for (int j = threadIdx.x; j < K; j += blockDim.x) {
+    s_id[j] = ids[t * K + j];
+    s_w[j] = to_f(w[t * K + j]);
+  }
+  __syncthreads();
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+    for (int j = 0; j < K; ++j) {
+      const float4 e = load4<T>(emb + (long long)s_id[j] * d + c);
+      a0 = fmaf(s_w[j], e.x, a0);
+      a1 = fmaf(s_w[j], e.y, a1);
+      a2 = fmaf(s_w[j], e.z, a2);
+      a3 = fmaf(s_w[j], e.w, a3);
+    }
+    store4<T>(u + t * d + c, a0, a1, a2, a3);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Commit / re-noise / stop, one CTA of 256 threads per canvas.
 // Default: commit where H < bound.  Entropy-bounded: sort (trunc(H 2^32), i)
 // ascending, commit the longest prefix with exact sum <= trunc(bound 2^32),

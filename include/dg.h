@@ -55,7 +55,8 @@ enum { DG_STOP_MEAN = 0, DG_STOP_EB = 1 };
  * canvas_len == 256; head_dim in {64, 128} (128 for DG_BF16); n_heads a
  * multiple of n_kv_heads with 128 % (n_heads / n_kv_heads) == 0;
  * d_model, d_ff multiples of 64; vocab a multiple of 64; top_k <= n_experts
- * <= 1024, top_k <= 64; 1 <= max_canvases; max_prompt >= 1. */
+ * <= 1024, top_k <= 64; 1 <= max_canvases; max_prompt >= 1;
+ * 0 <= sample_topk <= min(256, vocab). */
 typedef struct dg_config {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim;
   int32_t n_experts, top_k, d_ff, vocab;
@@ -75,6 +76,14 @@ typedef struct dg_config {
   int32_t max_canvases;   /* largest batch B passed to any call                  */
   int32_t max_prompt;     /* largest prompt length P passed to any call          */
   uint64_t sample_seed;   /* Philox key of all sampling draws                    */
+  int32_t sample_topk;    /* 0: exact sampling over the vocabulary.  K > 0: top-k
+                             truncation (DiffusionGemma technical-report
+                             explainer, section 九: the large-batch sampler
+                             optimisation) -- the token is the Gumbel-max draw
+                             among the K largest logits (same noise per token id
+                             as the exact draw), self-conditioning uses the
+                             untempered probabilities renormalised over those K;
+                             entropy, argmax, commit and stop are unchanged.    */
 } dg_config;
 
 typedef struct dg_model dg_model;

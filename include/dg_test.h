@@ -25,6 +25,26 @@ extern "C" {
 dg_status dg_test_math(int32_t which, const void* in, float* out, int64_t n, uint64_t aux0, uint32_t aux1,
                        void* stream);
 
+/* The top-k-truncated sampler kernel (DiffusionGemma technical-report
+ * explainer, section 九): as dg_test_sampler for H, argmax and S_q/U_q; the
+ * token is the Gumbel-max draw among the K largest logits of the row (value
+ * descending, ties to the lower index; noise as in the exact sampler);
+ * cand_ids int32 [rows, K] lists them best first and cand_w [rows, K] (bf16
+ * if w_bf16 else fp32) holds w_j = e_j (1/s), e_j = exp(l_j - max),
+ * s = e_0 + ... + e_{K-1} summed in that order.  vocab a multiple of 32,
+ * 1 <= K <= min(256, vocab) (DG_ERR_INVALID_ARG otherwise).  Asynchronous. */
+dg_status dg_test_sampler_topk(const float* logits, int32_t rows, int32_t vocab, int32_t positions, uint64_t seed,
+                               int32_t step, float t, float temp_start, float temp_end, int32_t K, float* H,
+                               int32_t* tok, int32_t* amax, int64_t* s_q, int64_t* u_q, int32_t* cand_ids,
+                               void* cand_w, int32_t w_bf16, void* stream);
+
+/* Self-conditioning gather of a truncated distribution: u [rows, d] =
+ * sum_j cand_w[r][j] emb[cand_ids[r][j]] (fp32 in candidate order, stored
+ * bf16 if bf16 else fp32; emb [*, d] in the same dtype).  d a multiple of
+ * 64, 1 <= K <= 256.  Asynchronous. */
+dg_status dg_test_sc_gather(const int32_t* cand_ids, const void* cand_w, int32_t rows, int32_t K, const void* emb,
+                            int32_t d, int32_t bf16, void* u, void* stream);
+
 /* Philox4x32-10 of n (counter[4], key[2]) records: in uint32 [n,6] ->
  * out uint32 [n,4] (Salmon et al., SC'11). */
 dg_status dg_test_philox(const uint32_t* in, uint32_t* out, int64_t n, void* stream);

@@ -163,6 +163,61 @@ def test_sampler_uniform_entropy_is_log_v():
     assert np.array_equal(host(am), [0, 0])
 
 
+# --- top-k-truncated sampler -----------------------------------------------------------
+@pytest.mark.parametrize("V,rows,positions,kind,scale,K,bf", [
+    (1024, 256, 256, "normal", 1.0, 256, False),
+    (1024, 300, 256, "mixed", 3.0, 64, False),     # ragged: a second canvas of 44 rows
+    (32768, 64, 32, "peaked", 1.0, 64, True),
+    (32768, 16, 16, "ties", 1.0, 200, True),       # many equal logits across the K-th place
+    (32768, 8, 8, "flat", 1.0, 32, True),          # every logit equal: the K lowest ids
+    (262144, 8, 8, "normal", 4.0, 64, True),
+    (262144, 4, 4, "mixed", 16.0, 256, True),
+    (4096, 16, 16, "normal", 1.0, 1, False),
+])
+def test_sampler_topk_bit_exact(V, rows, positions, kind, scale, K, bf):
+    l = I.logits(V + rows + K, rows, V, kind, scale)
+    step, t, seed = 3, 0.61, (7 << 32) + 5
+    inv_t = F32(1.0) / sp.temperature(F32(t))
+    ref = {k: [] for k in ("H", "amax", "tokens", "S_q", "U_q", "cand_ids", "cand_w")}
+    for c0 in range(0, rows, positions):
+        r = sp.sampler_rows_topk(l[c0:c0 + positions], K, inv_t, seed, c0 // positions, step)
+        for k in ref:
+            ref[k].append(r[k])
+    ref = {k: np.concatenate(v) for k, v in ref.items()}
+    z = lambda dt, *shape: torch.empty(shape, dtype=dt, device="cuda")
+    H, tok, am = z(torch.float32, rows), z(torch.int32, rows), z(torch.int32, rows)
+    sq, uq = z(torch.int64, rows), z(torch.int64, rows)
+    ids, wts = z(torch.int32, rows, K), z(torch.bfloat16 if bf else torch.float32, rows, K)
+    dg.test_sampler_topk(cu(l), positions, seed, step, t, 0.8, 0.4, K, H, tok, am, ids, wts, sq, uq)
+    assert np.array_equal(host(sq), ref["S_q"]) and np.array_equal(host(uq), ref["U_q"])
+    assert np.array_equal(host(H).view(np.uint32), ref["H"].view(np.uint32))
+    assert np.array_equal(host(am), ref["amax"])
+    assert np.array_equal(host(ids), ref["cand_ids"])
+    assert np.array_equal(host(tok), ref["tokens"])
+    wref = nm.round_bf16_from_f32(ref["cand_w"]) if bf else ref["cand_w"]
+    assert np.array_equal(host(wts.float()).view(np.uint32), wref.view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,K,d,bf", [(256, 64, 2816, True), (300, 16, 256, False), (8, 256, 1024, True)])
+def test_sc_gather(rows, K, d, bf):
+    g = np.random.default_rng(rows + K)
+    V = 4096
+    emb = g.standard_normal((V, d)).astype(F32) * F32(0.02)
+    ids = np.stack([g.choice(V, size=K, replace=False) for _ in range(rows)]).astype(np.int32)
+    w = g.dirichlet(np.ones(K), size=rows).astype(F32)
+    if bf:
+        emb, w = nm.round_bf16_from_f32(emb), nm.round_bf16_from_f32(w)
+    dt = torch.bfloat16 if bf else torch.float32
+    u = torch.empty((rows, d), dtype=dt, device="cuda")
+    dg.test_sc_gather(cu(ids), cu(w).to(dt), cu(emb).to(dt), u)
+    ref = np.einsum("rk,rkd->rd", w.astype(np.float64), emb[ids].astype(np.float64))
+    got = host(u.float())
+    # fp32 accumulation of K products, then the storage rounding
+    bound = (2.0 ** -8 if bf else 1e-6) * np.abs(ref) + K * 2e-7 * np.einsum(
+        "rk,rkd->rd", np.abs(w.astype(np.float64)), np.abs(emb[ids].astype(np.float64)))
+    assert np.all(np.abs(got - ref) <= bound + 1e-12)
+
+
 # --- commit / stop -------------------------------------------------------------------
 @pytest.mark.parametrize("mode,bound,stop_mode,stop_bound,step,ties,same", [
     (0, 0.5, 0, 0.1, 3, False, False),

@@ -72,6 +72,22 @@ def gumbel_margin(l32, inv_t, seed, canvas_id, step):
     return out
 
 
+def gumbel_margin_topk(l32, K, inv_t, seed, canvas_id, step):
+    """Top-k-truncated draws: gap between the best and second-best key among
+    the K candidates, capped by the gap between the K-th and (K+1)-th logit
+    (scaled to key units) since a candidate set that rounding can change may
+    change the draw."""
+    out = np.empty(l32.shape[0])
+    for i in range(l32.shape[0]):
+        ids = sp.topk_ids(l32[i], K + 1)
+        key = np.sort(l32[i, ids[:K]].astype(np.float64) * float(inv_t)
+                      + sp.gumbel_noise_at(ids[:K], seed, canvas_id, i, step))
+        gap = key[-1] - key[-2] if K > 1 else np.inf
+        edge = (float(l32[i, ids[K - 1]]) - float(l32[i, ids[K]])) * float(inv_t) if K < l32.shape[1] else np.inf
+        out[i] = min(gap, edge)
+    return out
+
+
 def check_logits(got, ref, fp32):
     if fp32:
         scale = np.maximum(np.abs(ref), np.sqrt((ref ** 2).mean(axis=-1, keepdims=True)))
@@ -80,12 +96,13 @@ def check_logits(got, ref, fp32):
         assert np.abs(got - ref).max() <= 2e-2, np.abs(got - ref).max()
 
 
-def compare_round(r_gpu, r_ora, w, step, t, fp32, canvas_id=0):
+def compare_round(r_gpu, r_ora, w, step, t, fp32, canvas_id=0, topk=0):
     check_logits(r_gpu["logits"], r_ora["logits64"], fp32)
     H_tol = 1e-4 * np.maximum(1.0, np.abs(r_ora["H"])) if fp32 else 2e-2
     assert np.all(np.abs(r_gpu["entropy"] - r_ora["H"]) <= H_tol)
     inv_t = F32(1.0) / sp.temperature(F32(t), w.temp_start, w.temp_end)
-    margin = gumbel_margin(r_ora["logits"], inv_t, w.sample_seed, canvas_id, step)
+    margin = (gumbel_margin_topk(r_ora["logits"], topk, inv_t, w.sample_seed, canvas_id, step) if topk
+              else gumbel_margin(r_ora["logits"], inv_t, w.sample_seed, canvas_id, step))
     err = np.abs(r_gpu["logits"] - r_ora["logits64"]).max(axis=1)
     safe = margin > 4 * err * float(inv_t) + 1e-6
     assert np.array_equal(r_gpu["tokens"][safe], r_ora["tokens"][safe])
@@ -215,6 +232,42 @@ def test_tiny_round_with_routing_bias(tiny):
     r = om.denoise_step(biased, Ko, Vo, canvas, None, 0, F32(1.0), trace=trace)
     compare_round(g, r, w, 0, 1.0, True)
     assert touched == [len(np.unique(trace[l]["ids"])) for l in range(w.n_layers)]
+
+
+def test_tiny_topk_sampler_round_and_block_match_oracle():
+    # sampling truncated to the 16 largest logits: rounds (tokens, entropy,
+    # commit, self-conditioning through the candidate gather) and a full block
+    K = 16
+    w = I.TINY_FP32.replace(sample_topk=K)
+    gm, om_ = dg.Model(w), om.Model(w)
+    P = w.prompt_len
+    prompt = I.prompt_ids(w.sample_seed, 1, P, w.vocab)
+    kv = gm.new_kv(1, P)
+    gm.encode_prompt(cu(prompt), kv)
+    Ko, Vo = om.encode_prompt(om_, prompt[0])
+    canvas = sp.initial_canvas(w.sample_seed, 0, 256, w.vocab)
+    out = step_buffers(w, 1)
+    gm.denoise_step(kv, P, cu(canvas[None]), None, 0, 1.0, out)
+    g = {k: host(v)[0] for k, v in out.items()}
+    r = om.denoise_step(om_, Ko, Vo, canvas, None, 0, F32(1.0))
+    compare_round(g, r, w, 0, 1.0, True, topk=K)
+    assert np.allclose(g["selfcond_next"], r["selfcond_next"], rtol=1e-4, atol=1e-6)
+    t1 = float(sp.schedule_t(1, w.max_steps))
+    gm.denoise_step(kv, P, cu(r["canvas_next"][None]), cu(r["selfcond_next"][None].astype(F32)), 1, t1, out)
+    g2 = {k: host(v)[0] for k, v in out.items()}
+    r2 = om.denoise_step(om_, Ko, Vo, r["canvas_next"], r["selfcond_next"], 1, sp.schedule_t(1, w.max_steps),
+                         prev_amax=r["amax"])
+    compare_round(g2, r2, w, 1, t1, True, topk=K)
+    cout = torch.zeros((1, 256), dtype=torch.int32, device="cuda")
+    su = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nc = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gm.generate_block(kv, 1, P, cout, su, nc)
+    gm.sync_status()
+    ref = om.generate_block(om_, Ko, Vo)
+    assert int(host(su)[0]) == ref["steps_used"]
+    assert (host(cout)[0] == ref["canvas"]).mean() >= 0.99
+    assert abs(int(host(nc)[0]) - ref["n_committed"]) <= 2
+    gm.close()
 
 
 # --- mid bf16 workload with a synthetic prompt cache -------------------------------------
