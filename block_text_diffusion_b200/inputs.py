@@ -48,6 +48,7 @@ class Workload:
     rms_eps: float = 1e-6
     zipf_s: float = 0.0          # 0 = no router bias
     sample_topk: int = 0         # 0 = exact sampling; K = draw among the K largest logits
+    expert_fp8: bool = False     # expert weights as E4M3 codes with power-of-two block scales
     temp_start: float = 0.8
     temp_end: float = 0.4
     max_steps: int = 48

@@ -42,6 +42,7 @@ import dataclasses
 import numpy as np
 
 from . import _native
+from . import fp8 as f8
 from . import numerics as nm
 from . import sampler as sp
 
@@ -127,6 +128,11 @@ class Model:
                 wv=weight_values(s, t("wv"), (hkv, d), bf), wo=weight_values(s, t("wo"), (d, hq), bf),
                 wr=weight_values(s, t("wr"), (E, d), bf), wg=weight_values(s, t("wg"), (E, ff, d), bf),
                 wu=weight_values(s, t("wu"), (E, ff, d), bf), wd=weight_values(s, t("wd"), (E, d, ff), bf)))
+            if getattr(cfg, "expert_fp8", False):
+                # FP8 expert weights: the GEMMs use the dequantised values q s
+                # (exact in bf16), every other weight stays as generated
+                L = self.layers[-1]
+                L.wg, L.wu, L.wd = (f8.quantize(L.wg)[2], f8.quantize(L.wu)[2], f8.quantize(L.wd)[2])
 
     def store(self, x):
         """Round float64 values to the storage dtype (returned as float64)."""
