@@ -71,6 +71,8 @@ def lib():
             "dg_test_sampler": ([P, I32, I32, I32, U64, I32, F, F, F, P, P, P, P, P, P, I32, P], I32),
             "dg_test_sampler_topk": ([P, I32, I32, I32, U64, I32, F, F, F, I32, P, P, P, P, P, P, P, I32, P], I32),
             "dg_test_sc_gather": ([P, P, I32, I32, P, I32, I32, P, P], I32),
+            "dg_test_quant_fp8": ([P, I64, I32, P, P, P], I32),
+            "dg_test_grouped_gemm_fp8": ([P, P, P, P, I32, I32, I32, I32, I32, P, P], I32),
             "dg_test_commit": ([P, P, P, P, I32, I32, U64, I32, I32, I32, F, I32, F, P, P, P, P, P], I32),
             "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, I32, P], I32),
             "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
@@ -264,6 +266,18 @@ def test_sc_gather(cand_ids, cand_w, emb, u, stream=None):
     _check(lib().dg_test_sc_gather(_ptr(cand_ids), _ptr(cand_w), rows, K, _ptr(emb), d,
                                    1 if emb.dtype == torch.bfloat16 else 0, _ptr(u), _stream(stream)),
            "dg_test_sc_gather")
+
+
+def test_quant_fp8(w, codes, scales, stream=None):
+    rows, K = w.shape
+    _check(lib().dg_test_quant_fp8(_ptr(w), rows, K, _ptr(codes), _ptr(scales), _stream(stream)), "dg_test_quant_fp8")
+
+
+def test_grouped_gemm_fp8(codes, scales, B, counts, groups, M, out, bn=64, k_splits=1, stream=None):
+    K = codes.shape[-1]
+    c = (ctypes.c_int32 * groups)(*[int(x) for x in counts])
+    _check(lib().dg_test_grouped_gemm_fp8(_ptr(codes), _ptr(scales), _ptr(B), c, groups, M, K, bn, k_splits,
+                                          _ptr(out), _stream(stream)), "dg_test_grouped_gemm_fp8")
 
 
 def test_commit(H, tok, amax, prev_amax, vocab, seed, step, max_steps, commit_mode, commit_bound, stop_mode,

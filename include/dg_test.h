@@ -109,6 +109,23 @@ dg_status dg_set_routing_bias(dg_model* m, const float* bias, int32_t n_tok);
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
                                int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);
 
+/* FP8 expert-weight quantisation (OCP E4M3, one power-of-two scale per 128
+ * inputs of each row: s = 2^ceil(log2(amax / 448)), q = RNE(w / s); a
+ * reading of the FP8 deployment in the DiffusionGemma release news, section
+ * "速度数据"): w bf16 [rows, K] -> codes uint8 [rows, K], scales fp32
+ * [rows, ceil(K / 128)].  Asynchronous. */
+dg_status dg_test_quant_fp8(const void* w, int64_t rows, int32_t K, uint8_t* codes, float* scales, void* stream);
+
+/* Grouped GEMM over FP8 weights: A8 codes [groups*M, K] with scales
+ * [groups*M, ceil(K/128)], B bf16 [rows, K] ordered by group (counts host
+ * int32 [groups]); out fp32 [k_splits][rows][M], the split-K partials
+ * (K chunks of 128 divided evenly, the last split taking the rest):
+ * out[s][r][m] = sum over the split's inputs of (q s)[g(r)*M + m][k] B[r][k].
+ * K a multiple of 16; bn in {32, 64, 128, 256}.  Allocates; synchronises. */
+dg_status dg_test_grouped_gemm_fp8(const uint8_t* A8, const float* scales, const void* B, const int32_t* counts,
+                                   int32_t groups, int32_t M, int32_t K, int32_t bn, int32_t k_splits, float* out,
+                                   void* stream);
+
 /* Attention kernels (tcgen05 for bf16, SIMT for fp32) plus the split
  * combine, on plain layouts: q [n_canvas*n_q, Hq, hd], k and v
  * [n_canvas, Hkv, n_keys, hd] -> out fp32 [n_canvas*n_q, Hq*hd].  Query i of
