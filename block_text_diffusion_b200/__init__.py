@@ -37,7 +37,7 @@ class Config(ctypes.Structure):
                 ("temp_end", ctypes.c_float), ("max_steps", ctypes.c_int32), ("commit_mode", ctypes.c_int32),
                 ("commit_bound", ctypes.c_float), ("stop_mode", ctypes.c_int32), ("stop_bound", ctypes.c_float),
                 ("canvas_len", ctypes.c_int32), ("max_canvases", ctypes.c_int32), ("max_prompt", ctypes.c_int32),
-                ("sample_seed", ctypes.c_uint64), ("sample_topk", ctypes.c_int32)]
+                ("sample_seed", ctypes.c_uint64), ("sample_topk", ctypes.c_int32), ("expert_fp8", ctypes.c_int32)]
 
 
 class StepOut(ctypes.Structure):
@@ -116,7 +116,8 @@ def make_config(w, max_canvases=None, max_prompt=None) -> Config:
     return Config(w.n_layers, w.d_model, w.n_heads, w.n_kv_heads, w.head_dim, w.n_experts, w.top_k, w.d_ff,
                   w.vocab, w.dtype, w.logit_scale, w.rope_theta, w.rms_eps, w.zipf_s, w.temp_start, w.temp_end,
                   w.max_steps, w.commit_mode, w.commit_bound, w.stop_mode, w.stop_bound, 256,
-                  max_canvases or w.batch, max_prompt or w.prompt_len, w.sample_seed, w.sample_topk)
+                  max_canvases or w.batch, max_prompt or w.prompt_len, w.sample_seed, w.sample_topk,
+                  int(w.expert_fp8))
 
 
 class Model:

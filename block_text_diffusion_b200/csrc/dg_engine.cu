@@ -115,6 +115,10 @@ struct Prof {
 struct LayerW {
   void *qkv = nullptr, *wo = nullptr, *wr = nullptr, *gu = nullptr, *wd = nullptr;
   CUtensorMap tm_qkv, tm_wo, tm_gu, tm_wd, tm_wr;
+  // FP8 expert weights (expert_fp8): E4M3 codes and per-128-input scales
+  uint8_t *gu8 = nullptr, *wd8 = nullptr;
+  float *gu_s = nullptr, *wd_s = nullptr;
+  CUtensorMap tm_gu8, tm_wd8;
 };
 
 // Tile-shape overrides for sweeps, read once from DG_TUNE="key=value,..."
@@ -152,6 +156,8 @@ struct dg_model {
   dg_config c;
   Tune tune;
   bool bf;
+  bool fp8 = false;   // expert weights stored as E4M3 codes + block scales
+  void* f8_scratch = nullptr;   // bf16 staging of one expert tensor during init
   int esz;
   int L, d, hq, hkv, hd, G, E, k, ff, V, nqkv;
   int T_cap;         // canvas tokens (max_canvases * 256)
@@ -354,6 +360,45 @@ dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   return DG_OK;
 }
 
+// Expert GEMM over FP8 weights (persistent, 128-row tiles, BN 256): split-K
+// counts 128-input chunks; the device-side split factor and ring sizing come
+// from the permute kernel as for the bf16 persistent GEMM.
+dg_status gemm_f8(dg_model* m, const GemmCall& g, const CUtensorMap* tmA8, const float* scales, long long a_rows,
+                  int phase, cudaStream_t s) {
+  if (g.bn != 256 || !g.work) return DG_ERR_UNSUPPORTED;
+  LaunchScope ls(m, s, phase);
+  GemmArgs a{};
+  a.M = g.M;
+  a.m_tiles = cdiv(g.M, 128);
+  a.kb_total = cdiv(g.K, kF8Chunk);
+  a.k_splits = std::max(1, std::min(g.splits, a.kb_total));
+  a.n_tile = g.bn;
+  a.alpha = g.alpha;
+  a.out = g.out;
+  a.ldo = g.ldo;
+  a.split_stride = g.split_stride;
+  a.work = g.work;
+  a.work_count = g.work_count;
+  a.a_group_rows = g.a_group_rows;
+  a.k_splits_dev = g.k_splits_dev;
+  a.max_rows_dev = g.max_rows_dev;
+  a.err = &m->st->err;
+  const F8Args f8{scales, cdiv(g.K, kF8Chunk), a_rows};
+  constexpr int kBudget = 200 * 1024;
+  static bool attr = false;
+  if (!attr) {
+    CU_TRY(cudaFuncSetAttribute(k_gemm_f8w_persistent<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kBudget + 1024));
+    attr = true;
+  }
+  const long long max_tiles = (long long)a.m_tiles * a.k_splits * g.max_items;
+  if (max_tiles <= 0) return DG_OK;
+  const int grid = (int)std::min<long long>(max_tiles, kSMs);
+  launch_pdl(k_gemm_f8w_persistent<256>, grid, kF8Threads, kBudget + 1024, s, *tmA8, *g.tB, a, f8, 0, kBudget);
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
 dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   LaunchScope ls(m, s, phase);
   GemmArgs a{};
@@ -456,6 +501,7 @@ bool config_ok(const dg_config& c) {
   if (c.stop_mode != DG_STOP_MEAN && c.stop_mode != DG_STOP_EB) return false;
   if (!(c.logit_scale == c.logit_scale) || !(c.rope_theta > 0.0f) || !(c.rms_eps >= 0.0f)) return false;
   if (c.sample_topk < 0 || c.sample_topk > kTopkMax || c.sample_topk > c.vocab) return false;
+  if (c.expert_fp8 != 0 && (c.expert_fp8 != 1 || c.dtype != DG_BF16)) return false;
   return true;
 }
 
@@ -491,10 +537,23 @@ dg_status init_all_weights(dg_model* m, uint64_t seed, cudaStream_t s) {
     init_tensor<T>((T*)w.wr, E * d, E * d, E * d, 0, seed, tid_layer(l, 4), s);
     // gate | up interleaved in blocks of 64 rows: rows [128 i, 128 i + 64) of
     // an expert are gate rows 64 i.., the next 64 the matching up rows, so a
-    // 128-row GEMM tile holds both halves of 64 SwiGLU outputs
-    init_tensor<T>((T*)w.gu, E * ff * d, 64 * d, 128 * d, 0, seed, tid_layer(l, 5), s);
-    init_tensor<T>((T*)w.gu, E * ff * d, 64 * d, 128 * d, 64 * d, seed, tid_layer(l, 6), s);
-    init_tensor<T>((T*)w.wd, E * d * ff, E * d * ff, E * d * ff, 0, seed, tid_layer(l, 7), s);
+    // 128-row GEMM tile holds both halves of 64 SwiGLU outputs.  FP8 experts:
+    // generated in the model dtype into a scratch tensor, then quantised.
+    T* gu = m->fp8 ? (T*)m->f8_scratch : (T*)w.gu;
+    init_tensor<T>(gu, E * ff * d, 64 * d, 128 * d, 0, seed, tid_layer(l, 5), s);
+    init_tensor<T>(gu, E * ff * d, 64 * d, 128 * d, 64 * d, seed, tid_layer(l, 6), s);
+    if (m->fp8) {
+      const long long units = (long long)E * 2 * ff * cdiv((int)d, kF8Chunk);
+      k_quant_f8<<<(unsigned)cdiv(units, 8), 256, 0, s>>>((const bf16*)gu, (long long)E * 2 * ff, (int)d, w.gu8,
+                                                          w.gu_s);
+    }
+    T* wd = m->fp8 ? (T*)m->f8_scratch : (T*)w.wd;
+    init_tensor<T>(wd, E * d * ff, E * d * ff, E * d * ff, 0, seed, tid_layer(l, 7), s);
+    if (m->fp8) {
+      const long long units = (long long)E * d * cdiv((int)ff, kF8Chunk);
+      k_quant_f8<<<(unsigned)cdiv(units, 8), 256, 0, s>>>((const bf16*)wd, (long long)E * d, (int)ff, w.wd8,
+                                                          w.wd_s);
+    }
   }
   CU_TRY(cudaGetLastError());
   return DG_OK;
@@ -511,8 +570,13 @@ dg_status build_maps(dg_model* m) {
     LayerW& w = m->layers[l];
     ok &= map2d(&w.tm_qkv, w.qkv, m->nqkv, d, 128);
     ok &= map2d(&w.tm_wo, w.wo, d, (uint64_t)m->hq * m->hd, 128);
-    ok &= map2d(&w.tm_gu, w.gu, (uint64_t)m->E * 2 * m->ff, d, 128);
-    ok &= map2d(&w.tm_wd, w.wd, (uint64_t)m->E * d, m->ff, 128);
+    if (m->fp8) {
+      ok &= map2d_u8(&w.tm_gu8, w.gu8, (uint64_t)m->E * 2 * m->ff, d, 128);
+      ok &= map2d_u8(&w.tm_wd8, w.wd8, (uint64_t)m->E * d, m->ff, 128);
+    } else {
+      ok &= map2d(&w.tm_gu, w.gu, (uint64_t)m->E * 2 * m->ff, d, 128);
+      ok &= map2d(&w.tm_wd, w.wd, (uint64_t)m->E * d, m->ff, 128);
+    }
     ok &= map2d(&w.tm_wr, w.wr, (uint64_t)m->E, d, 128);
   }
   const uint64_t Tw = m->Tw, Tk = (uint64_t)m->Tw * m->k;
@@ -706,6 +770,14 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
     plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
     plan.fused0 = m->bf ? 1 : 0;
+    if (m->fp8) {
+      // FP8 experts: 128-row tiles, split-K over 128-input chunks, SwiGLU as
+      // its own kernel
+      plan.mt[0] = cdiv(2 * m->ff, 128);
+      plan.kb[0] = cdiv(d, kF8Chunk);
+      plan.kb[1] = cdiv(m->ff, kF8Chunk);
+      plan.fused0 = 0;
+    }
     plan.out = m->moe_splits;
     { LaunchScope ls(m, s, PH_PERMUTE);
       launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
@@ -722,12 +794,14 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     gu.splits = m->bf ? 8 : 1;
     // bf16: an unsplit gate|up GEMM applies SwiGLU in its epilogue
-    if (m->bf) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = true; }
-    DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
+    if (m->bf && !m->fp8) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = true; }
+    if (m->fp8) DG_TRY(gemm_f8(m, gu, &w.tm_gu8, w.gu_s, (long long)m->E * 2 * m->ff, PH_GU_GEMM, s));
+    else DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
     { LaunchScope ls(m, s, PH_SWIGLU);
       const long long n = (long long)n_pairs * m->ff;
       launch_pdl(k_swiglu<T>, std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s, m->ws, m->ff, n, (T*)m->act,
-                                                                        m->moe_splits, gu_stride, m->bf ? 1 : 0); }
+                                                                        m->moe_splits, gu_stride,
+                                                                        (m->bf && !m->fp8) ? 1 : 0); }
     GemmCall dn;
     dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
     dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;
@@ -736,7 +810,8 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
     dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     dn.splits = m->bf ? 8 : 1;
-    DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
+    if (m->fp8) DG_TRY(gemm_f8(m, dn, &w.tm_wd8, w.wd_s, (long long)m->E * d, PH_DOWN_GEMM, s));
+    else DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
       launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
                                                m->c.rms_eps, m->moe_splits + 1, dn_stride); }
@@ -1041,6 +1116,7 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   m->c = *cfg;
   m->tune = read_tune();
   m->bf = cfg->dtype == DG_BF16;
+  m->fp8 = cfg->expert_fp8 == 1;
   m->esz = m->bf ? 2 : 4;
   m->L = cfg->n_layers; m->d = cfg->d_model; m->hq = cfg->n_heads; m->hkv = cfg->n_kv_heads;
   m->hd = cfg->head_dim; m->G = m->hq / m->hkv; m->E = cfg->n_experts; m->k = cfg->top_k;
@@ -1074,8 +1150,15 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
     A(&w.qkv, (size_t)m->nqkv * d * es);
     A(&w.wo, d * nq * es);
     A(&w.wr, (size_t)m->E * d * es);
-    A(&w.gu, (size_t)m->E * 2 * m->ff * d * es);
-    A(&w.wd, (size_t)m->E * d * m->ff * es);
+    if (m->fp8) {
+      A((void**)&w.gu8, (size_t)m->E * 2 * m->ff * d);
+      A((void**)&w.wd8, (size_t)m->E * d * m->ff);
+      A((void**)&w.gu_s, (size_t)m->E * 2 * m->ff * cdiv((int)d, kF8Chunk) * sizeof(float));
+      A((void**)&w.wd_s, (size_t)m->E * d * cdiv(m->ff, kF8Chunk) * sizeof(float));
+    } else {
+      A(&w.gu, (size_t)m->E * 2 * m->ff * d * es);
+      A(&w.wd, (size_t)m->E * d * m->ff * es);
+    }
   }
   const int max_pos = cfg->max_prompt + kCanvas;
   A((void**)&m->rope, (size_t)max_pos * (m->hd / 2) * sizeof(float2));
@@ -1124,7 +1207,17 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   cudaMemsetAsync(m->st, 0, sizeof(DevState), s);
   cudaMemsetAsync(m->prev_amax, 0xFF, (size_t)m->T_cap * sizeof(int), s);
   cudaMemsetAsync(m->sc, 0, (size_t)m->T_cap * d * es, s);
-  st = m->bf ? init_all_weights<bf16>(m, seed, s) : init_all_weights<float>(m, seed, s);
+  if (m->fp8 && st == DG_OK) {
+    // scratch for one expert tensor in bf16 before quantisation (freed below)
+    const size_t n = std::max((size_t)m->E * 2 * m->ff * d, (size_t)m->E * d * m->ff);
+    if (cudaMalloc(&m->f8_scratch, n * es) != cudaSuccess) { m->f8_scratch = nullptr; st = DG_ERR_OOM; }
+  }
+  if (st == DG_OK) st = m->bf ? init_all_weights<bf16>(m, seed, s) : init_all_weights<float>(m, seed, s);
+  if (m->f8_scratch) {
+    if (cudaStreamSynchronize(s) != cudaSuccess) st = DG_ERR_CUDA;
+    cudaFree(m->f8_scratch);
+    m->f8_scratch = nullptr;
+  }
   if (st == DG_OK) {
     const int n = max_pos * (m->hd / 2);
     k_rope_table<<<cdiv(n, 256), 256, 0, s>>>(m->rope, max_pos, m->hd / 2, m->hd, (double)cfg->rope_theta);

@@ -56,7 +56,8 @@ enum { DG_STOP_MEAN = 0, DG_STOP_EB = 1 };
  * multiple of n_kv_heads with 128 % (n_heads / n_kv_heads) == 0;
  * d_model, d_ff multiples of 64; vocab a multiple of 64; top_k <= n_experts
  * <= 1024, top_k <= 64; 1 <= max_canvases; max_prompt >= 1;
- * 0 <= sample_topk <= min(256, vocab). */
+ * 0 <= sample_topk <= min(256, vocab); expert_fp8 in {0, 1}, 1 only with
+ * DG_BF16. */
 typedef struct dg_config {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim;
   int32_t n_experts, top_k, d_ff, vocab;
@@ -84,6 +85,12 @@ typedef struct dg_config {
                              as the exact draw), self-conditioning uses the
                              untempered probabilities renormalised over those K;
                              entropy, argmax, commit and stop are unchanged.    */
+  int32_t expert_fp8;     /* 1: expert weights (gate, up, down) stored as OCP E4M3
+                             codes with one power-of-two scale per 128 inputs of
+                             each row, s = 2^ceil(log2(amax / 448)), q = RNE(w/s)
+                             (a reading of the FP8 deployment in the release news,
+                             section "速度数据"); the model computes with q s,
+                             exactly a bf16 value.  DG_BF16 only.                */
 } dg_config;
 
 typedef struct dg_model dg_model;
