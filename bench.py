@@ -42,6 +42,8 @@ def parse():
                     help="override the round budget (short runs for profiler launch lists)")
     ap.add_argument("--no-fast-converging", action="store_true",
                     help="skip the committed-tokens measurement on the fast-converging workload")
+    ap.add_argument("--expert-fp8", action="store_true",
+                    help="expert weights as E4M3 codes with per-128-input power-of-two scales")
     ap.add_argument("--topk-study", action="store_true",
                     help="also compare exact and top-k-truncated sampling at batch 32 (mid workload)")
     ap.add_argument("--routing-study", action="store_true",
@@ -91,15 +93,23 @@ def round_work(w, B, P, touched):
     nq, nk = w.n_heads * hd, w.n_kv_heads * hd
     T = B * 256
     attn_w = (d * (nq + 2 * nk) + nq * d) * esz
-    expert = 3 * d * w.d_ff * esz
+    expert = 3 * d * w.d_ff * expert_weight_bytes(w)
     kv = 2 * B * w.n_kv_heads * (P + 256) * hd * esz
     per_layer = attn_w + w.n_experts * d * esz + kv
     logits = T * V * 4
     bytes_ = (L * per_layer + sum(touched) * expert + 2 * V * d * esz + d * d * esz + 2 * logits
               + T * V * esz * 2)
-    flops = L * (2 * T * (d * (nq + 2 * nk) + nq * d + w.n_experts * d + w.top_k * expert // esz)
+    flops = L * (2 * T * (d * (nq + 2 * nk) + nq * d + w.n_experts * d + w.top_k * 3 * d * w.d_ff)
                  + 4 * T * w.n_heads * hd * (P + 256)) + 2 * T * V * d * 2 + 2 * T * d * d
     return bytes_, flops
+
+
+def expert_weight_bytes(w):
+    """Bytes per expert weight: the storage dtype, or an E4M3 code plus its
+    share of a 4-byte scale per 128 inputs."""
+    if getattr(w, "expert_fp8", False):
+        return 1.0 + 4.0 / 128.0
+    return 2 if w.dtype == 1 else 4
 
 
 def gate_up_bytes(w, B, touched):
@@ -109,7 +119,7 @@ def gate_up_bytes(w, B, touched):
     esz = 2 if w.dtype == 1 else 4
     rows = B * 256 * w.top_k
     avg = sum(touched) / len(touched)
-    return avg * 2 * w.d_ff * w.d_model * esz + rows * w.d_model * esz + rows * 2 * w.d_ff * 4
+    return avg * 2 * w.d_ff * w.d_model * expert_weight_bytes(w) + rows * w.d_model * esz + rows * 2 * w.d_ff * 4
 
 
 class Clocks:
@@ -197,6 +207,8 @@ def run_ours(a):
     w = w.replace(sample_seed=w.sample_seed + 1000 * rank)
     if a.max_rounds:
         w = w.replace(max_steps=a.max_rounds)
+    if a.expert_fp8:
+        w = w.replace(name=w.name + "-fp8experts", expert_fp8=True)
     model = dg.Model(w, max_canvases=B, max_prompt=P)
     stream = torch.cuda.current_stream()
     prompt_h = torch.from_numpy(I.prompt_ids(w.sample_seed, B, P, w.vocab)).pin_memory()
