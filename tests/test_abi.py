@@ -73,3 +73,32 @@ def test_product_path_refuses_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(dg, "_lib", None)
     with pytest.raises(RuntimeError):
         dg.lib()
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    # the ctypes mirrors of dg_config and dg_step_out have the C layout
+    # (size and every field offset), compiled from the header with the host C compiler
+    import shutil
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    import block_text_diffusion_b200 as dg
+    structs = {"dg_config": dg.Config, "dg_step_out": dg.StepOut}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "dg.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'  printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.check_call([cc, "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = {}
+    for line in subprocess.check_output([str(exe)], text=True).splitlines():
+        cname, field, val = line.split()
+        got[(cname, field)] = int(val)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert got[(cname, f)] == getattr(py, f).offset, (cname, f)
