@@ -38,7 +38,9 @@ dg_status dg_test_sampler_topk(const float* logits, int32_t rows, int32_t vocab,
                                int32_t* tok, int32_t* amax, int64_t* s_q, int64_t* u_q, int32_t* cand_ids,
                                void* cand_w, int32_t w_bf16, void* stream);
 
-/* Self-conditioning gather of a truncated distribution: u [rows, d] =
+/* Self-conditioning gather of a truncated distribution (the previous
+ * round's prediction fed back, DiffusionGemma technical-report explainer,
+ * section 二, restricted to the top-k candidates of section 九): u [rows, d] =
  * sum_j cand_w[r][j] emb[cand_ids[r][j]] (fp32 in candidate order, stored
  * bf16 if bf16 else fp32; emb [*, d] in the same dtype).  d a multiple of
  * 64, 1 <= K <= 256.  Asynchronous. */
@@ -116,7 +118,8 @@ dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* coun
  * [rows, ceil(K / 128)].  Asynchronous. */
 dg_status dg_test_quant_fp8(const void* w, int64_t rows, int32_t K, uint8_t* codes, float* scales, void* stream);
 
-/* Grouped GEMM over FP8 weights: A8 codes [groups*M, K] with scales
+/* Grouped GEMM over FP8 weights (the experts of the Mixture-of-Experts FFN,
+ * explainer section 二, stored as in dg_test_quant_fp8): A8 codes [groups*M, K] with scales
  * [groups*M, ceil(K/128)], B bf16 [rows, K] ordered by group (counts host
  * int32 [groups]); out fp32 [k_splits][rows][M], the split-K partials
  * (K chunks of 128 divided evenly, the last split taking the rest):

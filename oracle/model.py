@@ -118,7 +118,9 @@ class Model:
         self.embed = weight_values(s, T_EMBED, (V, d), bf)
         self.wsc = weight_values(s, T_WSC, (d, d), bf)
         # optional per-token router bias of the canvas pass, [L, 256 * canvases, E]
-        # (a workload input that structures routing; None = no such term)
+        # (a workload input that structures routing, standing in for the expert
+        # locality of a trained router -- about 84 of 128 experts per round in
+        # the explainer's section 五; None = no such term)
         self.route_bias = None
         self.layers = []
         for l in range(cfg.n_layers if layers is None else layers):
