@@ -72,6 +72,7 @@ def lib():
             "dg_test_sampler_topk": ([P, I32, I32, I32, U64, I32, F, F, F, I32, P, P, P, P, P, P, P, I32, P], I32),
             "dg_test_sc_gather": ([P, P, I32, I32, P, I32, I32, P, P], I32),
             "dg_test_quant_fp8": ([P, I64, I32, P, P, P], I32),
+            "dg_test_attn_plan": ([I64, I32, I32, I32, I32, I64, I64, P], I32),
             "dg_test_grouped_gemm_fp8": ([P, P, P, P, I32, I32, I32, I32, I32, P, P], I32),
             "dg_test_commit": ([P, P, P, P, I32, I32, U64, I32, I32, I32, F, I32, F, P, P, P, P, P], I32),
             "dg_test_gemm": ([P, P, P, I32, I32, I32, I32, F, I32, I32, I32, P], I32),

@@ -111,6 +111,14 @@ dg_status dg_set_routing_bias(dg_model* m, const float* bias, int32_t n_tok);
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
                                int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);
 
+/* Split-KV plan of the bf16 attention kernel (host only, no device call):
+ * out int32[4] = {query tiles per (canvas, KV head), key splits, 64-key
+ * blocks per split, CTAs} for n_q queries per canvas, G query heads per KV
+ * head, n_keys keys, rows = query rows of the launch and part_rows_cap =
+ * rows the partial-output buffer holds per split sum. */
+dg_status dg_test_attn_plan(int64_t n_q, int32_t G, int32_t Hkv, int32_t n_canvas, int32_t n_keys, int64_t rows,
+                            int64_t part_rows_cap, int32_t* out);
+
 /* FP8 expert-weight quantisation (OCP E4M3, one power-of-two scale per 128
  * inputs of each row: s = 2^ceil(log2(amax / 448)), q = RNE(w / s); a
  * reading of the FP8 deployment in the DiffusionGemma release news, section

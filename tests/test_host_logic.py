@@ -1,0 +1,88 @@
+"""Host-side logic of the library that runs without a GPU: the attention
+split plan, and the validation of configs and arguments that must reject bad
+input before any device call."""
+import ctypes
+
+import pytest
+
+import block_text_diffusion_b200 as dg
+from block_text_diffusion_b200 import inputs as I
+
+SMS = 148
+BK = 64                      # keys per attention block
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_text_diffusion_b200 import build
+    build.build()
+    return dg.lib()
+
+
+def plan(lib, n_q, G, Hkv, n_canvas, n_keys, cap=1 << 40):
+    out = (ctypes.c_int32 * 4)()
+    rows = n_q * G * Hkv * n_canvas
+    assert lib.dg_test_attn_plan(n_q, G, Hkv, n_canvas, n_keys, rows, cap, out) == 0
+    return list(out), rows
+
+
+@pytest.mark.parametrize("n_q,G,Hkv,n_canvas,n_keys", [
+    (256, 2, 8, 1, 2304),        # 26B shape, 2048-token prompt
+    (256, 4, 2, 1, 1280),        # mid shape
+    (256, 4, 2, 1, 33024),       # long context
+    (256, 4, 2, 32, 2304),       # 32 canvases
+    (64, 1, 4, 1, 320),          # tiny
+    (256, 2, 8, 1, 1),           # a single key
+    (1024, 4, 2, 1, 1024),       # causal encode chunk
+])
+def test_attention_plan_covers_every_key_block_once(lib, n_q, G, Hkv, n_canvas, n_keys):
+    (q_tiles, n_splits, bps, ctas), rows = plan(lib, n_q, G, Hkv, n_canvas, n_keys)
+    nblocks = -(-n_keys // BK)
+    assert q_tiles * 128 >= n_q * G and (q_tiles - 1) * 128 < n_q * G
+    assert 1 <= n_splits <= nblocks
+    assert n_splits * bps >= nblocks and (n_splits - 1) * bps < nblocks      # no empty split
+    base = -(-q_tiles // 2) * Hkv * n_canvas
+    assert ctas == base * n_splits
+    if base <= SMS:
+        assert ctas <= SMS or n_splits == 1                                  # the grid fills the SMs once
+
+
+def test_attention_plan_respects_the_partial_buffer(lib):
+    (_, n_splits, _, _), rows = plan(lib, 256, 4, 2, 1, 33024, cap=3 * 256 * 4 * 2)
+    assert n_splits * rows <= 3 * 256 * 4 * 2
+    (_, n_splits, _, _), _ = plan(lib, 256, 4, 2, 1, 33024, cap=1)
+    assert n_splits == 1
+
+
+def _init_status(lib, w, **over):
+    cfg = dg.make_config(w)
+    for k, v in over.items():
+        setattr(cfg, k, v)
+    out = ctypes.c_void_p()
+    return lib.dg_init_weights(ctypes.byref(cfg), 0, None, ctypes.byref(out))
+
+
+@pytest.mark.parametrize("field,value", [
+    ("canvas_len", 128), ("head_dim", 96), ("n_kv_heads", 3), ("d_model", 100), ("vocab", 1000),
+    ("top_k", 0), ("max_steps", 0), ("commit_mode", 7), ("stop_mode", 7), ("max_canvases", 0),
+    ("sample_topk", 257), ("sample_topk", -1), ("expert_fp8", 2),
+])
+def test_invalid_configs_are_rejected_before_any_device_call(lib, field, value):
+    assert _init_status(lib, I.TINY_FP32, **{field: value}) == 1
+
+
+def test_fp8_experts_need_bf16(lib):
+    assert _init_status(lib, I.TINY_FP32, expert_fp8=1) == 1
+
+
+def test_hook_arguments_are_checked_before_any_device_call(lib):
+    P = ctypes.c_void_p(1)   # never dereferenced: the checks fail first
+    # top-k sampler: K = 0, K > 256, vocab not a multiple of 32
+    for K, V in ((0, 1024), (257, 1024), (16, 1000)):
+        assert lib.dg_test_sampler_topk(P, 4, V, 4, 0, 0, 0.5, 0.8, 0.4, K, P, P, P, None, None, P, P, 0, None) == 1
+    # FP8 GEMM: K not a multiple of 16, unsupported tile
+    c = (ctypes.c_int32 * 1)(4)
+    assert lib.dg_test_grouped_gemm_fp8(P, P, P, c, 1, 128, 100, 64, 1, P, None) == 1
+    assert lib.dg_test_grouped_gemm_fp8(P, P, P, c, 1, 128, 128, 48, 1, P, None) == 1
+    # routing bias: n_tok not a multiple of 256
+    assert lib.dg_set_routing_bias(None, P, 100) == 1
