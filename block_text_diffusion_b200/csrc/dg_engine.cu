@@ -272,11 +272,27 @@ dg_status dalloc_t(dg_model* m, P** p, size_t count) {
 
 // Per-launch hooks: count launches; in profiling mode bracket each launch
 // with events on its stream.
+#ifdef DG_PROBE
+// Round timeline (diagnostic builds only): a one-thread kernel after every
+// phase launch waits, as a dependent launch, for the launch before it to
+// complete and records the global time and the phase, so consecutive stamps
+// bracket each kernel as it runs inside the captured block loop.
+__device__ long long g_tl[8192];
+__device__ int g_tl_phase[8192];
+__device__ unsigned int g_tl_n;
+__global__ void k_tl_stamp(int phase) {
+  pdl_enter();
+  const unsigned i = atomicAdd(&g_tl_n, 1u);
+  if (i < 8192u) { g_tl[i] = (long long)global_ns(); g_tl_phase[i] = phase; }
+}
+#endif
+
 struct LaunchScope {
   dg_model* m;
   cudaStream_t s;
   int idx = -1;
-  LaunchScope(dg_model* mm, cudaStream_t ss, int phase) : m(mm), s(ss) {
+  int phase_ = 0;
+  LaunchScope(dg_model* mm, cudaStream_t ss, int phase) : m(mm), s(ss), phase_(phase) {
     m->launch_count++;
     if (m->prof.on) {
       cudaEvent_t a, b;
@@ -291,6 +307,9 @@ struct LaunchScope {
   }
   ~LaunchScope() {
     if (idx >= 0) cudaEventRecord(m->prof.ev[2 * idx + 1], s);
+#ifdef DG_PROBE
+    launch_pdl(k_tl_stamp, 1, 1, 0, s, phase_);
+#endif
   }
 };
 
