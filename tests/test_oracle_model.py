@@ -440,3 +440,17 @@ def test_topk_self_condition_is_dense_self_condition_of_the_sparse_distribution(
         a = om.self_condition_topk(model, ids, wt)
         b = om.self_condition(model, dense)
         assert np.allclose(a, b, rtol=1e-6, atol=1e-9)
+
+
+def test_router_bias_closed_form_with_zero_input():
+    # x = 0: the logits are the bias alone, so the selection is the top-k of
+    # the bias and the gates its softmax over the selected experts -- a bias
+    # that reached only the selection (not the gates) gives equal gates
+    E, k = 8, 2
+    x = np.zeros((3, 16))
+    wr = np.random.default_rng(0).standard_normal((E, 16))
+    b = np.array([[0, 0, 3, 1, 0, 0, 0, 0], [2, 0, 0, 0, 0, 0, 0, 2], [0, -1, 0, 5, 4, 0, 0, 0]], dtype=np.float64)
+    ids, gates = om.router(x, wr, k, extra=b)
+    assert ids.tolist() == [[2, 3], [0, 7], [3, 4]]
+    expect = [1 / (1 + math.exp(-2.0)), 0.5, 1 / (1 + math.exp(-1.0))]
+    assert np.allclose(gates[:, 0], expect, rtol=1e-14) and np.allclose(gates.sum(axis=1), 1.0)

@@ -159,3 +159,30 @@ def test_nonstrict_stop_is_caught():
     hq = sp.fixed_entropy(at)
     wrong = int(hq.sum()) <= 256 * sp.bound_fixed(0.1)
     assert wrong != sp.stop_decision(at, none, a, None, 1, 48, 0, 0.1)
+
+def test_route_bias_missing_from_gates_is_caught(monkeypatch):
+    # a router that selects with the per-token bias but forms the gates
+    # without it: the zero-input closed form fails
+    import test_oracle_model as tm
+    orig_logits = om.router_logits
+
+    def wrong_router(x, wr, top_k, zipf_s=0.0, extra=None):
+        r = orig_logits(x, wr, zipf_s, extra)
+        r0 = orig_logits(x, wr, zipf_s, None)
+        ids = np.array([sorted(range(r.shape[1]), key=lambda e: (-r[t, e], e))[:top_k] for t in range(r.shape[0])],
+                       dtype=np.int32)
+        sel = np.take_along_axis(r0, ids, axis=1)
+        ex = np.exp(sel - sel.max(axis=1, keepdims=True))
+        return ids, ex / ex.sum(axis=1, keepdims=True)
+
+    monkeypatch.setattr(om, "router", wrong_router)
+    with pytest.raises(AssertionError):
+        tm.test_router_bias_closed_form_with_zero_input()
+
+
+def test_topk_ties_to_the_higher_index_are_caught(monkeypatch):
+    import test_oracle_sampler as ts
+    monkeypatch.setattr(sp, "topk_ids", lambda l, K: np.lexsort((-np.arange(np.asarray(l).size),
+                                                                 -np.asarray(l, np.float64)))[:K].astype(np.int32))
+    with pytest.raises(AssertionError):
+        ts.test_topk_ids_brute_force("ties")
