@@ -501,6 +501,18 @@ def block_autoregressive(dg, I, torch, blocks=3):
 
 
 # --- CPU oracle (bounded sample) ---------------------------------------------------------
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_sample(w, P, budget_s=20.0):
     """Time the oracle on a bounded sample of one round of workload `w` and
     scale to a whole round.  Sample: one transformer layer (256 canvas tokens
@@ -573,7 +585,7 @@ def run_reference(a):
             "dtype": "f64 (bf16 storage rounding)" if w.dtype == 1 else "f64",
             "data": "synthetic", "config": {"workload": w.name, "canvases_per_gpu": 1, "prompt_len": w.prompt_len},
             "cpu_baseline": {"value": value, "unit": "denoise steps/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "cpu": cpu_model()},
             "e2e": {"value": value, "unit": "denoise steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -592,7 +604,7 @@ def main():
         w = I.WORKLOADS[a.workload]
         v, cores, sample, secs = oracle_sample(w, w.prompt_len)
         line["cpu_baseline"] = {"value": v, "unit": "denoise steps/s", "cores": cores, "kind": "oracle",
-                                "sample": sample, "cpu_seconds": secs}
+                                "sample": sample, "cpu_seconds": secs, "cpu": cpu_model()}
     print(json.dumps(line), flush=True)
 
 
