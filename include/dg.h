@@ -168,7 +168,11 @@ dg_status dg_generate_block(dg_model* model, void* kv, int32_t B, int32_t P, int
  *               bytes; holds the whole context on return.
  *   tokens_out  device int32 [B, n_blocks, 256]: each block's sampled tokens.
  *   steps_used, n_committed  device int32 [B, n_blocks].
- * P + 256 (n_blocks - 1) must not exceed max_prompt (DG_ERR_INVALID_ARG). */
+ * P + 256 (n_blocks - 1) must not exceed max_prompt, 1 <= B <= max_canvases
+ * and n_blocks >= 1 (DG_ERR_INVALID_ARG otherwise, nothing enqueued).
+ * Asynchronous on `stream`; a device-side wait that ran out is reported by the
+ * next call or dg_sync_status.  The block loop's graph is re-captured for each
+ * block (the canvas positions and the seed change). */
 dg_status dg_generate(dg_model* model, const int32_t* prompt, int32_t B, int32_t P, int32_t n_blocks, void* kv,
                       int32_t* tokens_out, int32_t* steps_used, int32_t* n_committed, void* stream);
 
