@@ -330,7 +330,7 @@ SLACK = dict(x=1.0, logit=2e-2, H=1e-3, sc=1e-2)
 
 
 def compare_bf16_round(g, r, trace, om_model, w, gx_final, rn, trace_n, min_stable=0.9, canvas_id=0):
-    """bf16 parity of one round against the oracle, judged by the storage-noise
+    """bf16 parity of one round against the oracle, assessed by the storage-noise
     envelope, plus the workload's 2e-2 on the LM head where it applies.
 
     * LM head: the logits equal logit_scale * x E^T of the path's own final
@@ -417,7 +417,7 @@ def test_mid_round_matches_oracle(layers):
 def test_mid_full_depth_round_statistics(mid):
     """All 8 layers: near-tie routing flips in early layers propagate through
     attention to every token, so no token set is routing-stable; the round is
-    judged by whole-round statistics against the storage-noise envelope, and
+    assessed by whole-round statistics against the storage-noise envelope, and
     the LM head by the workload's 2e-2 given the same normalised state."""
     w, gm, om_ = mid
     g, r, trace, _, gx, rn, trace_n = run_bf16_round(w, w.prompt_len, 9)
