@@ -48,6 +48,8 @@ def parse():
                     help="also compare exact and top-k-truncated sampling at batch 32 (mid workload)")
     ap.add_argument("--routing-study", action="store_true",
                     help="also sweep a structured router bias over expert-pool sizes (routing locality)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the throughput lines of the other workloads")
     return ap.parse_args()
 
 
@@ -114,12 +116,13 @@ def expert_weight_bytes(w):
 
 def gate_up_bytes(w, B, touched):
     """Algorithmic bytes of one expert gate|up GEMM launch, averaged over the
-    layers: touched experts' gate and up weights, the gathered rows read, the
-    fp32 outputs written."""
+    layers: touched experts' gate and up weights, the gathered rows read, and
+    the method's output -- the SwiGLU activation, one value per (row, hidden
+    unit) in the storage dtype."""
     esz = 2 if w.dtype == 1 else 4
     rows = B * 256 * w.top_k
     avg = sum(touched) / len(touched)
-    return avg * 2 * w.d_ff * w.d_model * expert_weight_bytes(w) + rows * w.d_model * esz + rows * 2 * w.d_ff * 4
+    return avg * 2 * w.d_ff * w.d_model * expert_weight_bytes(w) + rows * w.d_model * esz + rows * w.d_ff * esz
 
 
 class Clocks:
@@ -234,20 +237,26 @@ def run_ours(a):
         torch.cuda.synchronize()
 
     rounds = torch.zeros((), dtype=torch.int64, device="cuda")
+    loop_rounds = torch.zeros((), dtype=torch.int64, device="cuda")
     committed = torch.zeros((), dtype=torch.int64, device="cuda")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    model.reset_touched_experts()
     barrier()
     with Clocks(local) as clk:
         e0.record(stream)
         for _ in range(a.steps):
             block()
             rounds += steps.sum()
+            loop_rounds += steps.max()
             committed += ncom.sum()
         e1.record(stream)
         barrier()
     ms = e0.elapsed_time(e1)
     model.sync_status()
     n_rounds, n_com = int(rounds.item()), int(committed.item())
+    # distinct experts each layer streamed, averaged over every round of the
+    # timed blocks (counted on the device)
+    touched = [t / max(1, int(loop_rounds.item())) for t in model.touched_experts_sum(reset=True)]
 
     # end to end through the public API with host buffers
     canvas_h = torch.zeros((B, 256), dtype=torch.int32).pin_memory()
@@ -271,8 +280,6 @@ def run_ours(a):
 
     # per-kernel timing (CUDA events around each launch of single rounds)
     prof = model.profile_step(kv, B, P, reps=a.profile_reps)
-    # distinct experts each layer streamed in the profiled round (measured routing)
-    touched = model.touched_experts()
 
     study = None
     if a.routing_study:
@@ -280,6 +287,11 @@ def run_ours(a):
     topk = None
     if a.topk_study and world == 1:
         topk = topk_study(dg, I, torch)
+
+    # throughput and roofline fraction of the other workloads: single-GPU runs only
+    configs = None
+    if world == 1 and not a.no_per_config:
+        configs = per_config(dg, I, torch)
 
     # committed tokens on the fast-converging workload (logit scale 16), where
     # random-init weights still commit: single-GPU runs only
@@ -330,7 +342,8 @@ def run_ours(a):
         "ms_per_round": per_round_ms,
         "step_roofline": {"bound": "hbm" if b_round / hbm > f_round / tf_sus / 1e3 else "tensor",
                           "roof_ms": step_roof_ms, "frac": step_roof_ms / per_round_ms,
-                          "bytes": b_round, "flops": f_round, "touched_experts": touched},
+                          "bytes": b_round, "flops": f_round,
+                          "touched_experts_mean_over_timed_rounds": [round(t, 2) for t in touched]},
         "roofline": {"bound": "hbm", "kernel": "expert_gate_up_gemm", "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "traffic": measured_traffic(gu_bytes),
                      "peak_source": src, "avg_launch_ms": gu_avg, "algorithmic_bytes": gu_bytes},
@@ -338,6 +351,7 @@ def run_ours(a):
         "e2e": {"value": e_rounds / (e2e_ms * 1e-3), "unit": "denoise steps/s",
                 "h2d_bytes_per_step": B * P * 4 * world, "d2h_bytes_per_step": (B * 256 + 2 * B) * 4 * world,
                 "includes": "prompt H2D, causal prompt encode, block loop, result D2H"},
+        "per_config": configs,
         "fast_converging": fast,
         "routing_study": study,
         "topk_study": topk,
@@ -346,6 +360,63 @@ def run_ours(a):
     }
     model.close()
     return line
+
+
+def per_config(dg, I, torch, blocks=2):
+    """Rounds per second, committed tokens per second and the step-roofline
+    fraction of the workloads beside the headline one, each at its own bound
+    (HBM copy peak, or the sustained bf16 tensor peak where the round's FLOPs
+    dominate): the tiny fp32 decoder, the mid MoE, the Zipf-routed batch
+    workload at 1, 4, 8 and 32 canvases (2048-token prompts each) and the
+    long-context workload.  Device events around `blocks` full blocks after
+    one warm-up block; touched experts counted on the device over the timed
+    rounds."""
+    hbm, _, tf_sus, _ = peaks()
+    stream = torch.cuda.current_stream()
+    cases = [("tiny", I.TINY_FP32, 1), ("mid", I.MID_BF16, 1)]
+    cases += [("batch_B%d" % b, I.BATCH_ZIPF, b) for b in I.BATCH_SIZES]
+    cases += [("long", I.LONG_CTX, 1)]
+    out = {}
+    for key, w, B in cases:
+        P = w.prompt_len
+        model = dg.Model(w, max_canvases=B, max_prompt=P)
+        try:
+            kv = model.new_kv(B, P)
+            model.encode_prompt(torch.from_numpy(I.prompt_ids(w.sample_seed, B, P, w.vocab)).cuda(), kv)
+            z = lambda *shape: torch.zeros(shape, dtype=torch.int32, device="cuda")
+            canvas, steps, ncom = z(B, 256), z(B), z(B)
+            model.generate_block(kv, B, P, canvas, steps, ncom)
+            torch.cuda.synchronize()
+            model.reset_touched_experts()
+            rounds = torch.zeros((), dtype=torch.int64, device="cuda")
+            loop_rounds = torch.zeros((), dtype=torch.int64, device="cuda")
+            committed = torch.zeros((), dtype=torch.int64, device="cuda")
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(blocks):
+                model.generate_block(kv, B, P, canvas, steps, ncom)
+                rounds += steps.sum()
+                loop_rounds += steps.max()
+                committed += ncom.sum()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            model.sync_status()
+            ms = e0.elapsed_time(e1)
+            n_loop = max(1, int(loop_rounds.item()))
+            touched = [t / n_loop for t in model.touched_experts_sum(reset=True)]
+        finally:
+            model.close()
+        b_round, f_round = round_work(w, B, P, touched)
+        t_hbm, t_tc = b_round / (hbm * 1e9) * 1e3, f_round / (tf_sus * 1e12) * 1e3
+        ms_round = ms / n_loop
+        out[key] = {"workload": w.name, "canvases": B, "prompt_len": P,
+                    "denoise_steps_per_s": int(rounds.item()) / (ms * 1e-3),
+                    "committed_tokens_per_s": int(committed.item()) / (ms * 1e-3),
+                    "ms_per_round": ms_round, "rounds_per_block": n_loop / blocks,
+                    "step_roofline": {"bound": "hbm" if t_hbm >= t_tc else "tensor", "roof_ms": max(t_hbm, t_tc),
+                                      "frac": max(t_hbm, t_tc) / ms_round, "bytes": b_round, "flops": f_round,
+                                      "touched_experts_mean": sum(touched) / len(touched)}}
+    return out
 
 
 def fast_converging(dg, I, torch, blocks=3):

@@ -79,7 +79,7 @@ def lib():
             "dg_test_grouped_gemm": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
             "dg_test_router": ([P, P, P, P, I32, I32, I32, I32, P, P, P], I32),
             "dg_set_routing_bias": ([P, P, I32], I32),
-            "dg_test_attention": ([P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P], I32),
+            "dg_test_attention": ([P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P], I32),
             "dg_read_weight": ([P, I32, P, P], I32),
             "dg_load_kv": ([P, P, I32, I32, P, P, P], I32),
             "dg_profile_step": ([P, P, I32, I32, I32, P, P, I32, P], I32),
@@ -87,6 +87,8 @@ def lib():
             "dg_launches_per_round": ([P], I32),
             "dg_expert_counts": ([P, P, P], I32),
             "dg_debug_trace": ([P, P, P], I32),
+            "dg_test_layer": ([P, P, I32, I32, I32, P, P, P, P], I32),
+            "dg_touched_experts_sum": ([P, P, I32, P], I32),
             "dg_gemm_splitk_noalloc": ([P, P, P, I32, I32, I32, I32, P], I32),
         }
         for name, (args, res) in sig.items():
@@ -196,6 +198,14 @@ class Model:
         """Record per-layer hidden states and routing of later eager calls."""
         _check(lib().dg_debug_trace(self.h, _ptr(h_trace), _ptr(ids_trace)), "dg_debug_trace")
 
+    def run_layer(self, kv, B, P, layer, h_in, h_trace, ids, stream=None):
+        """Layer `layer` of the canvas pass from the residual state h_in
+        [B*256, d] (model dtype): h_trace fp32 [3, B*256, d] receives h after
+        the attention residual, after the MoE and RMSNorm of the latter; ids
+        int32 [B*256, top_k] the routing; the canvas keys/values go into kv."""
+        _check(lib().dg_test_layer(self.h, _ptr(kv), B, P, layer, _ptr(h_in), _ptr(h_trace), _ptr(ids),
+                                   _stream(stream)), "dg_test_layer")
+
     def expert_counts(self, counts, stream=None):
         """Per-layer expert row counts [n_layers, n_experts] of the most recent call."""
         _check(lib().dg_expert_counts(self.h, _ptr(counts), _stream(stream)), "dg_expert_counts")
@@ -211,6 +221,16 @@ class Model:
         n = bias.shape[1] if n_tok is None else n_tok
         _check(lib().dg_set_routing_bias(self.h, _ptr(bias), n), "dg_set_routing_bias")
         self._routing_bias = bias
+
+    def touched_experts_sum(self, reset=False, stream=None):
+        """Per layer, the distinct experts streamed summed over every canvas
+        pass since creation or the last reset (list of ints)."""
+        out = (ctypes.c_uint64 * self.w.n_layers)()
+        _check(lib().dg_touched_experts_sum(self.h, out, int(reset), _stream(stream)), "dg_touched_experts_sum")
+        return [int(x) for x in out]
+
+    def reset_touched_experts(self, stream=None):
+        _check(lib().dg_touched_experts_sum(self.h, None, 1, _stream(stream)), "dg_touched_experts_sum")
 
     def touched_experts(self, stream=None):
         """Distinct experts each layer of the most recent call routed to (list)."""
@@ -309,21 +329,26 @@ def test_router(x, wr, ids, gate, bias=None, tok_bias=None, stream=None):
 
 
 def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, sized_ring=False, swiglu=False,
-                      m256=False, stream=None):
+                      m256=False, streamk=False, stream=None):
     import torch
     K = A.shape[-1]
     c = (ctypes.c_int32 * groups)(*[int(x) for x in counts])
-    flags = int(persistent) | (2 if sized_ring else 0) | (4 if swiglu else 0) | (8 if m256 else 0)
+    flags = (int(persistent) | (2 if sized_ring else 0) | (4 if swiglu else 0) | (8 if m256 else 0)
+             | (16 if streamk else 0))
     _check(lib().dg_test_grouped_gemm(_ptr(A), _ptr(B), c, groups, M, K, 1 if A.dtype == torch.bfloat16 else 0,
                                       bn, flags, _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
 
 
-def test_attention(q, k, v, n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out, stream=None):
+def test_attention(q, k, v, n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out, force_path=0, stream=None):
+    """Returns the merge path taken: 1 = split partials + combine kernel,
+    2 = in-kernel cluster merge."""
     import torch
     hd = q.shape[-1]
+    path = ctypes.c_int32(0)
     _check(lib().dg_test_attention(_ptr(q), _ptr(k), _ptr(v), n_canvas, n_q, q_pos0, n_keys, int(causal), Hq,
-                                   Hkv, hd, 1 if q.dtype == torch.bfloat16 else 0, _ptr(out), _stream(stream)),
-           "dg_test_attention")
+                                   Hkv, hd, 1 if q.dtype == torch.bfloat16 else 0, int(force_path),
+                                   ctypes.byref(path), _ptr(out), _stream(stream)), "dg_test_attention")
+    return path.value
 
 
 def gemm_splitk_noalloc(A, B, out, k_splits=1, stream=None):
@@ -331,7 +356,15 @@ def gemm_splitk_noalloc(A, B, out, k_splits=1, stream=None):
     entry point that allocates no device memory (its split-K partial sums
     live in a fixed-size array inside the library).  For callers that must
     not call cudaMalloc: see dg_gemm_splitk_noalloc in include/dg.h."""
+    import torch
+    for name, t, dt in (("A", A, torch.bfloat16), ("B", B, torch.bfloat16), ("out", out, torch.float32)):
+        if t.dtype != dt or t.dim() != 2 or not t.is_contiguous() or t.device != A.device:
+            raise ValueError(f"gemm_splitk_noalloc: {name} must be a contiguous 2-D {dt} tensor on {A.device}")
     M, K = A.shape
     N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError(f"gemm_splitk_noalloc: B has {B.shape[1]} columns, A has {K}")
+    if tuple(out.shape) != (N, M):
+        raise ValueError(f"gemm_splitk_noalloc: out must be [{N}, {M}], got {list(out.shape)}")
     _check(lib().dg_gemm_splitk_noalloc(_ptr(A), _ptr(B), _ptr(out), M, N, K, k_splits, _stream(stream)),
            "dg_gemm_splitk_noalloc")

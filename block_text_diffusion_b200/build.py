@@ -2,11 +2,6 @@
 
 The shared object is written next to this file; `python -m
 block_text_diffusion_b200.build` rebuilds it when any source is newer.
-
-Diagnostics (performance analysis only, not used by the library):
-`--probe` also builds libdg_probe.so, the same library with the GEMM timeline
-probes compiled in (-DDG_PROBE), and `--mma-bench` builds diag/mma_bench, a
-tensor-core throughput microbenchmark.
 """
 from __future__ import annotations
 
@@ -37,11 +32,11 @@ def stale() -> bool:
     return any(os.path.getmtime(s) > t for s in SOURCES)
 
 
-def build(force: bool = False, verbose: bool = False, lib: str = LIB, defines=()) -> str:
+def build(force: bool = False, verbose: bool = False, lib: str = LIB) -> str:
     if not force and lib == LIB and not stale():
         return lib
     tmp = lib + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH, "-Xcompiler", "-fPIC", "-shared", *defines,
+    cmd = [nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH, "-Xcompiler", "-fPIC", "-shared",
            "-o", tmp, os.path.join(HERE, "csrc", "dg_engine.cu"), os.path.join(HERE, "csrc", "dg_noalloc.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -50,19 +45,5 @@ def build(force: bool = False, verbose: bool = False, lib: str = LIB, defines=()
     return lib
 
 
-def build_probe() -> str:
-    return build(force=True, lib=os.path.join(HERE, "libdg_probe.so"), defines=("-DDG_PROBE",))
-
-
-def build_mma_bench() -> str:
-    out = os.path.join(HERE, "diag", "mma_bench")
-    subprocess.check_call([nvcc(), "-std=c++17", "-O3", *ARCH, "-o", out, os.path.join(HERE, "diag", "mma_bench.cu")])
-    return out
-
-
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
-    if "--probe" in sys.argv:
-        print(build_probe())
-    if "--mma-bench" in sys.argv:
-        print(build_mma_bench())

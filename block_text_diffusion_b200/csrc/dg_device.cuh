@@ -237,15 +237,6 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 constexpr int kSMs = 148;   // streaming multiprocessors of a B200
-// Timeline probes of CTA 0 of a kernel (global-timer stamps into g_probe),
-// only in builds with -DDG_PROBE (performance diagnosis); no-ops otherwise.
-// Slots: persistent GEMM 0..1023, attention 2000..2199.
-#ifdef DG_PROBE
-__device__ long long g_probe[4096];
-#define DG_PROBE_STAMP(i) do { if (blockIdx.x == 0 && (i) < 4096) g_probe[(i)] = (long long)global_ns(); } while (0)
-#else
-#define DG_PROBE_STAMP(i) do { } while (0)
-#endif
 
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

@@ -33,15 +33,19 @@ typedef CUresult (*PFN_encode)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, vo
                                CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                CUtensorMapFloatOOBfill);
 
+// Looked up once; a function-local static is initialised once even when
+// several host threads get here first at the same time.
+PFN_encode lookup_encode() {
+  cudaDriverEntryPointQueryResult q;
+  void* p = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return (PFN_encode)p;
+  return nullptr;
+}
+
 PFN_encode encode_fn() {
-  static PFN_encode fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (PFN_encode)p;
-  }
+  static const PFN_encode fn = lookup_encode();
   return fn;
 }
 
@@ -183,9 +187,11 @@ struct dg_model {
   void* cand_w = nullptr;
   BMaps tm_x, tm_o, tm_xp, tm_act, tm_probs, tm_u;   // activation (B) operands
   float* ws = nullptr;
+  StreamK sk{};                      // stream-K expert GEMMs: partial slots [SMs][2][256][128], flags [SMs]
   float *o_part = nullptr, *lse_part = nullptr;
   int *ids = nullptr, *perm = nullptr, *inv = nullptr, *work_count = nullptr, *counts = nullptr;
   int* moe_splits = nullptr;         // [3] split-K of the gate|up and down GEMMs, largest item rows (set by permute)
+  unsigned long long* touched_acc = nullptr;   // [L] distinct experts streamed, summed over canvas passes
   float* gate = nullptr;
   int4* work = nullptr;
   float *logits = nullptr, *H = nullptr;
@@ -272,27 +278,12 @@ dg_status dalloc_t(dg_model* m, P** p, size_t count) {
 
 // Per-launch hooks: count launches; in profiling mode bracket each launch
 // with events on its stream.
-#ifdef DG_PROBE
-// Round timeline (diagnostic builds only): a one-thread kernel after every
-// phase launch waits, as a dependent launch, for the launch before it to
-// complete and records the global time and the phase, so consecutive stamps
-// bracket each kernel as it runs inside the captured block loop.
-__device__ long long g_tl[8192];
-__device__ int g_tl_phase[8192];
-__device__ unsigned int g_tl_n;
-__global__ void k_tl_stamp(int phase) {
-  pdl_enter();
-  const unsigned i = atomicAdd(&g_tl_n, 1u);
-  if (i < 8192u) { g_tl[i] = (long long)global_ns(); g_tl_phase[i] = phase; }
-}
-#endif
 
 struct LaunchScope {
   dg_model* m;
   cudaStream_t s;
   int idx = -1;
-  int phase_ = 0;
-  LaunchScope(dg_model* mm, cudaStream_t ss, int phase) : m(mm), s(ss), phase_(phase) {
+  LaunchScope(dg_model* mm, cudaStream_t ss, int phase) : m(mm), s(ss) {
     m->launch_count++;
     if (m->prof.on) {
       cudaEvent_t a, b;
@@ -307,9 +298,6 @@ struct LaunchScope {
   }
   ~LaunchScope() {
     if (idx >= 0) cudaEventRecord(m->prof.ev[2 * idx + 1], s);
-#ifdef DG_PROBE
-    launch_pdl(k_tl_stamp, 1, 1, 0, s, phase_);
-#endif
   }
 };
 
@@ -338,6 +326,8 @@ struct GemmCall {
   void* act = nullptr;               // persistent gate|up: SwiGLU output (bf16) when the GEMM runs unsplit
   int act_ld = 0;
   bool m256 = false;                 // dense, bn 256: 256-row M tiles (two accumulators share B)
+  bool streamk = false;              // grouped bf16, bn 256: stream-K over every SM (fused SwiGLU when act is set)
+  StreamK sk{};
   int qkv_on = 0;                    // dense bf16, one split: fused QKV post-process
   QkvEpi qkv{};
 };
@@ -375,6 +365,24 @@ dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   const int per_sm = std::max(1, (228 * 1024) / (C::kSmem + 2048));
   const int grid = (int)std::min<long long>(max_tiles, (long long)kSMs * std::min(per_sm, 2));
   launch_pdl(k_gemm_tc_persistent<BN, ST, MT>, grid, 192, C::kSmem, s, *g.tA, *g.tB, a, items_dense);
+  CU_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+// Stream-K grouped GEMM: one CTA per SM (every CTA resident at once);
+// MT = 2 for 256-row tiles.
+template <int MT>
+dg_status launch_tc_streamk(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
+  constexpr int kStages = MT == 2 ? 3 : 4;
+  using C = GemmTcCfg<256, kStages, MT>;
+  static bool attr = false;
+  if (!attr) {
+    CU_TRY(cudaFuncSetAttribute(k_gemm_tc_streamk<256, kStages, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::kSmem));
+    attr = true;
+  }
+  if (!g.sk.seg_ws || !g.sk.seg_flag) return DG_ERR_STATE;
+  launch_pdl(k_gemm_tc_streamk<256, kStages, MT>, kSMs, 192, C::kSmem, s, *g.tA, *g.tB, a, g.sk);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -451,6 +459,16 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   }
   a.m_tiles = cdiv(g.M, 128);
   a.n_tile = g.bn;
+  if (g.streamk) {
+    if (!g.work || g.bn != 256) return DG_ERR_UNSUPPORTED;
+    a.k_splits = 1;
+    a.max_rows_dev = g.max_rows_dev;
+    if (g.m256) {
+      a.m_tiles = cdiv(g.M, 256);
+      return launch_tc_streamk<2>(g, a, s);
+    }
+    return launch_tc_streamk<1>(g, a, s);
+  }
   if (g.persistent) {
     if (g.m256 && g.bn == 256) {   // 256-row tiles: two accumulators share each B tile
       a.m_tiles = cdiv(g.M, 256);
@@ -643,13 +661,47 @@ bool attn_maps(const dg_model* m, const KvGeom& g, int n_keys, int T_q, AttnMaps
   return ok;
 }
 
+// The tensor-core attention: one launch of the plan's CTAs; with the in-kernel
+// merge the split CTAs of a query-tile pair form one thread-block cluster.
+dg_status launch_attn_tc(const AttnPlan& ap, const AttnMaps& am, const AttnArgs& aa, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    CU_TRY(cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem));
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ap.ctas);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = kAttnSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  if (g_use_pdl) {
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (ap.cluster && ap.n_splits > 1) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = (unsigned)ap.n_splits;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = na;
+  CU_TRY(cudaLaunchKernelEx(&cfg, k_attn_tc, am.q, am.k, am.v, aa));
+  return DG_OK;
+}
+
 // ---------------------------------------------------------------------------
 // One transformer layer stack over `T` tokens of `n_canvas` canvases
 // (n_per tokens each, positions pos0..), writing keys/values into the cache.
 // ---------------------------------------------------------------------------
 template <typename T>
 dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_per, int pos0, int n_keys,
-                     bool causal, cudaStream_t s) {
+                     bool causal, cudaStream_t s, int l_first = 0, int l_end = -1) {
+  if (l_end < 0) l_end = m->L;
   const int Tn = n_canvas * n_per;
   const int d = m->d, nq = m->hq * m->hd;
   AttnMaps am;
@@ -662,7 +714,9 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
 
   // Precondition: m->x holds RMSNorm(h) of the first layer (written by the
   // embedding kernel); every layer leaves RMSNorm of its output in m->x.
-  for (int l = 0; l < m->L; ++l) {
+  // The diagnostic trace indexes layers from l_first.
+  for (int l = l_first; l < l_end; ++l) {
+    const int lt = l - l_first;
     const LayerW& w = m->layers[l];
     // QKV projection
     GemmCall qc;
@@ -703,17 +757,15 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     aa.n_canvas = n_canvas; aa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)m->hd));
     aa.o_part = m->o_part; aa.lse_part = m->lse_part; aa.err = &m->st->err;
     const long long rows = (long long)Tn * m->hq;
+    bool attn_merged = false;   // the attention kernel merged its key splits itself
     {
       LaunchScope ls(m, s, PH_ATTN);
       if (m->bf) {
         const AttnPlan ap = attn_plan(n_per, m->G, m->hkv, n_canvas, n_keys, rows, (long long)m->part_rows_cap);
         aa.q_tiles = ap.q_tiles; aa.n_splits = ap.n_splits; aa.blocks_per_split = ap.blocks_per_split;
-        static bool attr = false;
-        if (!attr) {
-          CU_TRY(cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem));
-          attr = true;
-        }
-        launch_pdl(k_attn_tc, ap.ctas, kAttnThreads, kAttnSmem, s, am.q, am.k, am.v, aa);
+        aa.cluster = ap.cluster; aa.o_out = (bf16*)m->o;
+        attn_merged = ap.cluster != 0;
+        DG_TRY(launch_attn_tc(ap, am, aa, s));
       } else {
         aa.q_tiles = 1; aa.n_splits = 1; aa.blocks_per_split = 1;
         const long long threads = rows * 32;
@@ -722,9 +774,11 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       }
       CU_TRY(cudaGetLastError());
     }
-    { LaunchScope ls(m, s, PH_ATTN_COMBINE);
-      launch_pdl(k_attn_combine<T>, (unsigned)cdiv(rows, 8), 256, 0, s, m->o_part, m->lse_part, aa.n_splits, rows, m->hd,
-                                                        (T*)m->o); }
+    if (!attn_merged) {
+      LaunchScope ls(m, s, PH_ATTN_COMBINE);
+      launch_pdl(k_attn_combine<T>, (unsigned)cdiv(rows, 8), 256, 0, s, m->o_part, m->lse_part, aa.n_splits, rows,
+                 m->hd, (T*)m->o);
+    }
     // output projection + residual
     GemmCall oc;
     oc.tA = &w.tm_wo; oc.tB = &m->tm_o; oc.A32 = (const float*)w.wo; oc.B32 = (const float*)m->o;
@@ -742,7 +796,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
       launch_pdl(k_residual_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, oc.split_stride,
                                             std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
     if (m->dbg_h)
-      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l) * Tn * d, (long long)Tn * d);
+      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * lt) * Tn * d, (long long)Tn * d);
     // MoE
     // per-token router bias: canvas passes only, rows of canvases b0 ..
     const float* tb = (!causal && m->tok_bias)
@@ -800,8 +854,8 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     plan.out = m->moe_splits;
     { LaunchScope ls(m, s, PH_PERMUTE);
       launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
-                                                             m->work, m->work_count, m->counts + (size_t)l * m->E,
-                                                             plan, &m->st->err); }
+                 m->work, m->work_count, m->counts + (size_t)l * m->E, plan,
+                 causal ? nullptr : m->touched_acc + l, &m->st->err); }
     { LaunchScope ls(m, s, PH_GATHER);
       launch_pdl(k_gather<T>, n_pairs, 128, 0, s, (const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
     GemmCall gu;
@@ -812,15 +866,18 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     gu.split_stride = gu_stride; gu.k_splits_dev = m->bf ? m->moe_splits : nullptr;
     gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     gu.splits = m->bf ? 8 : 1;
-    // bf16: an unsplit gate|up GEMM applies SwiGLU in its epilogue
-    if (m->bf && !m->fp8) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = true; }
+    // bf16: stream-K over every SM with SwiGLU in the epilogue (no partial
+    // slabs, no separate activation pass); FP8 experts: split-K then SwiGLU
+    const bool sk = m->bf && !m->fp8;
+    if (sk) { gu.act = m->act; gu.act_ld = m->ff; gu.streamk = true; gu.m256 = true; gu.sk = m->sk; }
     if (m->fp8) DG_TRY(gemm_f8(m, gu, &w.tm_gu8, w.gu_s, (long long)m->E * 2 * m->ff, PH_GU_GEMM, s));
     else DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
-    { LaunchScope ls(m, s, PH_SWIGLU);
+    if (!sk) {
+      LaunchScope ls(m, s, PH_SWIGLU);
       const long long n = (long long)n_pairs * m->ff;
       launch_pdl(k_swiglu<T>, std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s, m->ws, m->ff, n, (T*)m->act,
-                                                                        m->moe_splits, gu_stride,
-                                                                        (m->bf && !m->fp8) ? 1 : 0); }
+                 m->moe_splits, gu_stride, 0);
+    }
     GemmCall dn;
     dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
     dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;
@@ -829,19 +886,20 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
     dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
     dn.splits = m->bf ? 8 : 1;
+    if (sk) { dn.streamk = true; dn.sk = m->sk; }
     if (m->fp8) DG_TRY(gemm_f8(m, dn, &w.tm_wd8, w.wd_s, (long long)m->E * d, PH_DOWN_GEMM, s));
     else DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
     { LaunchScope ls(m, s, PH_COMBINE);
       launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
-                                               m->c.rms_eps, m->moe_splits + 1, dn_stride); }
+                 m->c.rms_eps, sk ? nullptr : m->moe_splits + 1, dn_stride); }
     if (m->dbg_h) {
-      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * l + 1) * Tn * d,
+      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * lt + 1) * Tn * d,
                                          (long long)Tn * d);
-      CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)l * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
+      CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)lt * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
                              cudaMemcpyDeviceToDevice, s));
-      if (l == m->L - 1)   // the final normalised state (input of the LM head)
-        launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->x, m->dbg_h + (size_t)(2 * m->L) * Tn * d,
-                                           (long long)Tn * d);
+      if (l == l_end - 1)   // the normalised state the layers leave (LM head input after the last layer)
+        launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->x,
+                   m->dbg_h + (size_t)(2 * (l_end - l_first)) * Tn * d, (long long)Tn * d);
     }
   }
   CU_TRY(cudaGetLastError());
@@ -1197,6 +1255,10 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   A(&m->u, (size_t)m->T_cap * d * es);
   A(&m->sc, (size_t)m->T_cap * d * es);
   A((void**)&m->ws, m->ws_elems * sizeof(float));
+  if (m->bf) {
+    A((void**)&m->sk.seg_ws, (size_t)kSMs * 2 * 256 * 128 * sizeof(float));
+    A((void**)&m->sk.seg_flag, (size_t)kSMs * sizeof(int));
+  }
   A((void**)&m->o_part, m->part_rows_cap * m->hd * sizeof(float));
   A((void**)&m->lse_part, m->part_rows_cap * sizeof(float));
   A((void**)&m->ids, Tk * sizeof(int));
@@ -1207,6 +1269,7 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   A((void**)&m->work_count, sizeof(int));
   A((void**)&m->moe_splits, 4 * sizeof(int));
   A((void**)&m->counts, (size_t)m->L * m->E * sizeof(int));
+  A((void**)&m->touched_acc, (size_t)m->L * sizeof(unsigned long long));
   A((void**)&m->logits, (size_t)m->T_cap * V * sizeof(float));
   A((void**)&m->H, (size_t)m->T_cap * sizeof(float));
   A((void**)&m->tok, (size_t)m->T_cap * sizeof(int));
@@ -1226,6 +1289,8 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   cudaMemsetAsync(m->st, 0, sizeof(DevState), s);
   cudaMemsetAsync(m->prev_amax, 0xFF, (size_t)m->T_cap * sizeof(int), s);
   cudaMemsetAsync(m->sc, 0, (size_t)m->T_cap * d * es, s);
+  if (m->sk.seg_flag) cudaMemsetAsync(m->sk.seg_flag, 0, (size_t)kSMs * sizeof(int), s);
+  if (m->touched_acc) cudaMemsetAsync(m->touched_acc, 0, (size_t)m->L * sizeof(unsigned long long), s);
   if (m->fp8 && st == DG_OK) {
     // scratch for one expert tensor in bf16 before quantisation (freed below)
     const size_t n = std::max((size_t)m->E * 2 * m->ff * d, (size_t)m->E * d * m->ff);
@@ -1261,10 +1326,11 @@ int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   (void)B; (void)P;
   // per layer: qkv gemm (bf16: with the RoPE / cache scatter; fp32: + qkv
   // post), attention, attention combine, o gemm, residual+norm, router (bf16:
-  // one kernel; fp32: gemm + top-k), permute, gather, gate/up gemm, swiglu,
+  // one kernel; fp32: gemm + top-k), permute, gather, gate/up gemm, swiglu
+  // (fp32 and FP8 experts; bf16 fuses it into the stream-K gate|up GEMM),
   // down gemm, combine+norm; then embed+norm, lm head, sampler, commit,
   // 4 self-cond.
-  const int per_layer = (m->bf ? 12 : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
+  const int per_layer = (m->bf ? (m->fp8 ? 12 : 11) : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
   return per_layer * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          (m->c.sample_topk > 0 ? 3 : 4) /*self-conditioning*/;
 }

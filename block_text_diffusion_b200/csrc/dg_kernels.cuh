@@ -125,6 +125,23 @@ __global__ void k_embed_norm(const int* __restrict__ ids, const T* __restrict__ 
   rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
 }
 
+// A given residual state as a layer's input: h[t] = h_in[t];  x[t] = RMSNorm(h[t]).
+template <typename T>
+__global__ void k_load_norm(const T* __restrict__ h_in, T* __restrict__ h, T* __restrict__ x, int d, float eps) {
+  pdl_enter();
+  __shared__ float red[32];
+  const long long t = blockIdx.x;
+  T* hr = h + t * d;
+  float ss = 0.0f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    const T hv = h_in[t * d + i];
+    hr[i] = hv;
+    const float f = to_f(hv);
+    ss = fmaf(f, f, ss);
+  }
+  rownorm_store<T>(hr, x + t * d, d, eps, ss, red);
+}
+
 // Attention residual fused with the MoE RMSNorm:
 // h = round(h + sum_s ws[s]);  x = RMSNorm(h).  One CTA per row.  Rows of up
 // to 16 values per thread stay in registers, with every load issued before
@@ -469,7 +486,7 @@ __device__ __forceinline__ int block_scan_excl(int v, int* wsum, int* total) {
 
 __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int bn, int* __restrict__ perm,
                           int* __restrict__ inv, int4* __restrict__ work, int* __restrict__ work_count,
-                          int* __restrict__ counts_out, SplitPlan plan, int* err) {
+                          int* __restrict__ counts_out, SplitPlan plan, unsigned long long* touched_acc, int* err) {
   // Warp w owns the contiguous pair range [w*chunk, (w+1)*chunk).  A pair's
   // position is offs[e] (pairs of lower experts) + pairs of expert e in
   // earlier warps + pairs of e earlier in this warp's range, which keeps the
@@ -507,8 +524,8 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
   __syncthreads();
   // expert offsets and work items: block-wide exclusive scans of the expert
   // row counts and item counts (chunks of blockDim experts, with carries)
-  __shared__ int wsum[32], s_max_rows;
-  if (threadIdx.x == 0) s_max_rows = 0;
+  __shared__ int wsum[32], s_max_rows, s_touched;
+  if (threadIdx.x == 0) { s_max_rows = 0; s_touched = 0; }
   int carry_rows = 0, carry_items = 0;
   for (int e0 = 0; e0 < E; e0 += blockDim.x) {
     const int e = e0 + threadIdx.x;
@@ -523,7 +540,7 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
       offs[e] = acc;
       for (int j = 0; j < it; ++j)
         work[nw0 + j] = make_int4(e, acc + j * bn, min(bn, c - j * bn), acc + j * bn);
-      if (c > 0) atomicMax(&s_max_rows, min(c, bn));
+      if (c > 0) { atomicMax(&s_max_rows, min(c, bn)); atomicAdd(&s_touched, 1); }
     }
     carry_rows += tot_rows;
     carry_items += tot_items;
@@ -533,6 +550,8 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
     const int nw = carry_items;
     offs[E] = carry_rows;
     *work_count = nw;
+    // running total of distinct experts this layer streamed (measurement)
+    if (touched_acc) *touched_acc += (unsigned long long)s_touched;
     if (plan.out) {
       // Split-K factor per GEMM: the persistent kernel runs ceil(tiles / SMs)
       // waves of tiles that each take 1/s of a full-K tile, and every split

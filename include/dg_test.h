@@ -106,16 +106,22 @@ dg_status dg_set_routing_bias(dg_model* m, const float* bias, int32_t n_tok);
  * (persistent, bf16, M % 128 == 0) applies SwiGLU in the epilogue: A rows
  * interleave gate / up in blocks of 64 and out receives bf16 [rows][M/2],
  * out[r][f] = round(silu(g) u) with g, u the rows 128 (f/64) + f%64 (+64);
- * bit 3 (persistent, bn 256) uses 256-row tiles (two accumulators per CTA).
- * Allocates. */
+ * bit 3 (persistent, bn 256) uses 256-row tiles (two accumulators per CTA);
+ * bit 4 (bf16, bn 256) runs the stream-K kernel the expert GEMMs use (one
+ * CTA per SM, equal runs of (tile, k block) iterations, cut tiles finished
+ * in k order by the CTA holding their first k range; with bit 2 it writes the
+ * SwiGLU activation) and returns DG_ERR_STATE if a partial-slot flag is left
+ * set afterwards.  Allocates. */
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
                                int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);
 
 /* Split-KV plan of the bf16 attention kernel (host only, no device call):
- * out int32[4] = {query tiles per (canvas, KV head), key splits, 64-key
- * blocks per split, CTAs} for n_q queries per canvas, G query heads per KV
- * head, n_keys keys, rows = query rows of the launch and part_rows_cap =
- * rows the partial-output buffer holds per split sum. */
+ * out int32[5] = {query tiles per (canvas, KV head), key splits, 64-key
+ * blocks per split, CTAs, 1 if the splits of a query-tile pair merge inside
+ * the kernel as one thread-block cluster (at most 8 splits) else 0} for n_q
+ * queries per canvas, G query heads per KV head, n_keys keys, rows = query
+ * rows of the launch and part_rows_cap = rows the partial-output buffer
+ * holds per split sum (binding only when the splits merge through it). */
 dg_status dg_test_attn_plan(int64_t n_q, int32_t G, int32_t Hkv, int32_t n_canvas, int32_t n_keys, int64_t rows,
                             int64_t part_rows_cap, int32_t* out);
 
@@ -138,13 +144,18 @@ dg_status dg_test_grouped_gemm_fp8(const uint8_t* A8, const float* scales, const
                                    void* stream);
 
 /* Attention kernels (tcgen05 for bf16, SIMT for fp32) plus the split
- * combine, on plain layouts: q [n_canvas*n_q, Hq, hd], k and v
+ * merge, on plain layouts: q [n_canvas*n_q, Hq, hd], k and v
  * [n_canvas, Hkv, n_keys, hd] -> out fp32 [n_canvas*n_q, Hq*hd].  Query i of
  * a canvas sits at position q_pos0 + i; causal != 0 hides keys after it.
+ * force_path (bf16): 0 = the plan's choice, 1 = split partials in global
+ * memory merged by the combine kernel, 2 = merge inside the kernel across a
+ * cluster of at most 8 splits (bf16 output, widened to fp32 here); path_out
+ * (host, may be NULL) receives the path taken (1 or 2; 1 for fp32).
  * Allocates. */
 dg_status dg_test_attention(const void* q, const void* k, const void* v, int32_t n_canvas, int32_t n_q,
                             int32_t q_pos0, int32_t n_keys, int32_t causal, int32_t Hq, int32_t Hkv,
-                            int32_t head_dim, int32_t bf16, float* out, void* stream);
+                            int32_t head_dim, int32_t bf16, int32_t force_path, int32_t* path_out, float* out,
+                            void* stream);
 
 /* Copy weight tensor `tensor_id` (0 = E [V,d], 1 = W_sc [d,d]; layer l:
  * 16+16l + {0 Wq,1 Wk,2 Wv,3 Wo,4 Wr,5 Wg [E,ff,d],6 Wu,7 Wd [E,d,ff]})
@@ -170,6 +181,13 @@ const char* dg_phase_name(int32_t i);
  * experts layer l streamed. */
 dg_status dg_expert_counts(const dg_model* model, int32_t* counts, void* stream);
 
+/* Distinct experts each layer streamed, summed over every canvas pass (one
+ * per layer per denoising round, in single steps and in the block loop; the
+ * prompt encode is not counted) since the model was created or last reset:
+ * per_layer host uint64 [n_layers] (may be NULL when only resetting);
+ * reset != 0 zeroes the sums afterwards.  Synchronises when reading. */
+dg_status dg_touched_experts_sum(dg_model* model, uint64_t* per_layer, int32_t reset, void* stream);
+
 /* Diagnostic trace of later eager calls (dg_denoise_step, dg_encode_prompt):
  * for every layer l, h after the attention residual -> h_trace[l][0][T][d]
  * and after the MoE -> h_trace[l][1][T][d], then the final RMSNorm(h) ->
@@ -177,6 +195,21 @@ dg_status dg_expert_counts(const dg_model* model, int32_t* counts, void* stream)
  * routing ids -> ids_trace[l][T][top_k] (T = tokens of the call).  Both NULL turns it off;
  * the block-loop graph never traces.  Buffers are the caller's. */
 dg_status dg_debug_trace(dg_model* model, float* h_trace, int32_t* ids_trace);
+
+/* One transformer layer of the canvas pass from a given residual state
+ * (DiffusionGemma technical-report explainer, section 二: a pre-norm block
+ * of bidirectional attention over [prompt KV ; canvas] and the top-k MoE
+ * FFN).  h_in: device [B*256][d] in the model dtype, the residual stream
+ * entering layer `layer`; the layer normalises it, attends with the canvas
+ * at positions P..P+255 over the prompt keys/values the caller stored in
+ * `kv` (dg_load_kv) plus its own, and writes the canvas keys/values of that
+ * layer into `kv`.  Outputs (device, caller-owned): h_trace fp32
+ * [3][B*256][d] = h after the attention residual, h after the MoE, and
+ * RMSNorm of the latter; ids int32 [B*256][top_k] = the routing (slot order).
+ * A per-token router bias set by dg_set_routing_bias applies.  Synchronises;
+ * DG_ERR_INVALID_ARG for a bad layer or shape, a device error code otherwise. */
+dg_status dg_test_layer(dg_model* model, void* kv, int32_t B, int32_t P, int32_t layer, const void* h_in,
+                        float* h_trace, int32_t* ids, void* stream);
 
 /* Kernel launches recorded in one captured block-loop round (graph body). */
 int32_t dg_launches_per_round(const dg_model* model);

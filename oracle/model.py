@@ -14,13 +14,18 @@ section 一):
     26B-A4B model (top-k of E in the smaller workloads);
   * a self-conditioning input carrying the previous round's prediction.
 The remaining architecture (pre-norm RMSNorm, rotate-half RoPE, SwiGLU
-experts, tied LM head, logit scale) is the workload definition's.  Readings
-where the pages are silent are listed in the design notes; the main ones:
-no sqrt(d) embedding scale; RoPE theta 10000 at absolute positions (prompt
-0..P-1, canvas P..P+255); RMSNorm eps 1e-6 with unit gains; self-
-conditioning s = (softmax(l) E) W_sc^T, added to the canvas token embeddings
-(zero at round 0); router softmax over the k selected logits (plus a Zipf
-bias -s ln(e+1) when configured), ties to the lower expert id.
+experts, tied LM head, logit scale) is the workload definition's.  Where
+the pages are silent this oracle reads them so: no sqrt(d) embedding scale;
+RoPE theta 10000 at absolute positions (prompt 0..P-1, canvas P..P+255);
+RMSNorm eps 1e-6 with unit gains (random gains would scale the signal
+away); the "logit scale" multiplies the final logits before temperature and
+entropy; self-conditioning s = (softmax(l) E) W_sc^T with the tied embedding
+E and a d x d W_sc (a linear V -> d map of about 7.8 M parameters at the
+26B-A4B width, where a dense V x d matrix would hold 738 M), added to the
+canvas token embeddings and zero at round 0; router softmax over the k
+selected logits (plus a Zipf bias -s ln(e+1) when configured, in selection
+and gates alike), ties to the lower expert id, slots in descending logit
+order.
 
 Arithmetic: float64 everywhere.  Values are rounded to the model's storage
 dtype (bf16 round-to-nearest-even, or binary32) at the storage points of the
@@ -105,36 +110,72 @@ class Layer:
     wd: np.ndarray
 
 
-class Model:
-    """Weights of one workload (float32 arrays holding the stored values)."""
+class ExpertTensor:
+    """An expert weight tensor [E, out, in] whose experts are generated one at
+    a time on first use and kept (the per-layer checks of the large
+    workloads touch a few experts of each layer).  Indexing by expert id
+    gives the [out, in] matrix; FP8 workloads give the dequantised values."""
 
-    def __init__(self, cfg, layers=None):
+    def __init__(self, seed, tensor_id, shape, bf16, fp8=False):
+        self.seed, self.tensor_id, self.shape, self.bf16, self.fp8 = seed, tensor_id, tuple(shape), bf16, fp8
+        self._cache = {}
+
+    def __getitem__(self, e):
+        e = int(e)
+        if e not in self._cache:
+            _, o, i = self.shape
+            n = o * i
+            if _native.lib() is not None:
+                w = _native.weights(self.seed, self.tensor_id, e * n, n, self.bf16)
+            else:
+                w = _normal_weights(self.seed, self.tensor_id, e * n, n, self.bf16)
+            w = w.reshape(o, i)
+            self._cache[e] = f8.quantize(w)[2] if self.fp8 else w
+        return self._cache[e]
+
+
+def layer_weights(cfg, l, lazy_experts=False) -> Layer:
+    """Weights of layer l; with lazy_experts the expert tensors are
+    ExpertTensor objects (generated per expert when first indexed)."""
+    bf = cfg.dtype == DTYPE_BF16
+    d, E, ff = cfg.d_model, cfg.n_experts, cfg.d_ff
+    hq, hkv = cfg.n_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim
+    s = cfg.weight_seed
+    fp8 = bool(getattr(cfg, "expert_fp8", False))
+    t = lambda w: layer_tensor_id(l, w)
+    if lazy_experts:
+        wg, wu, wd = (ExpertTensor(s, t("wg"), (E, ff, d), bf, fp8), ExpertTensor(s, t("wu"), (E, ff, d), bf, fp8),
+                      ExpertTensor(s, t("wd"), (E, d, ff), bf, fp8))
+    else:
+        wg, wu, wd = (weight_values(s, t("wg"), (E, ff, d), bf), weight_values(s, t("wu"), (E, ff, d), bf),
+                      weight_values(s, t("wd"), (E, d, ff), bf))
+        if fp8:
+            # FP8 expert weights: the GEMMs use the dequantised values q s
+            # (exact in bf16), every other weight stays as generated
+            wg, wu, wd = f8.quantize(wg)[2], f8.quantize(wu)[2], f8.quantize(wd)[2]
+    return Layer(wq=weight_values(s, t("wq"), (hq, d), bf), wk=weight_values(s, t("wk"), (hkv, d), bf),
+                 wv=weight_values(s, t("wv"), (hkv, d), bf), wo=weight_values(s, t("wo"), (d, hq), bf),
+                 wr=weight_values(s, t("wr"), (E, d), bf), wg=wg, wu=wu, wd=wd)
+
+
+class Model:
+    """Weights of one workload (float32 arrays holding the stored values).
+    `layers` limits how many layers are generated; with_embed=False skips the
+    embedding and W_sc (for checks of single layers)."""
+
+    def __init__(self, cfg, layers=None, with_embed=True):
         self.cfg = cfg
         bf = cfg.dtype == DTYPE_BF16
         d, V = cfg.d_model, cfg.vocab
-        hq, hkv, hd = cfg.n_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim, cfg.head_dim
-        E, ff = cfg.n_experts, cfg.d_ff
         s = cfg.weight_seed
-        self.embed = weight_values(s, T_EMBED, (V, d), bf)
-        self.wsc = weight_values(s, T_WSC, (d, d), bf)
+        self.embed = weight_values(s, T_EMBED, (V, d), bf) if with_embed else None
+        self.wsc = weight_values(s, T_WSC, (d, d), bf) if with_embed else None
         # optional per-token router bias of the canvas pass, [L, 256 * canvases, E]
         # (a workload input that structures routing, standing in for the expert
         # locality of a trained router -- about 84 of 128 experts per round in
         # the explainer's section 五; None = no such term)
         self.route_bias = None
-        self.layers = []
-        for l in range(cfg.n_layers if layers is None else layers):
-            t = lambda w: layer_tensor_id(l, w)
-            self.layers.append(Layer(
-                wq=weight_values(s, t("wq"), (hq, d), bf), wk=weight_values(s, t("wk"), (hkv, d), bf),
-                wv=weight_values(s, t("wv"), (hkv, d), bf), wo=weight_values(s, t("wo"), (d, hq), bf),
-                wr=weight_values(s, t("wr"), (E, d), bf), wg=weight_values(s, t("wg"), (E, ff, d), bf),
-                wu=weight_values(s, t("wu"), (E, ff, d), bf), wd=weight_values(s, t("wd"), (E, d, ff), bf)))
-            if getattr(cfg, "expert_fp8", False):
-                # FP8 expert weights: the GEMMs use the dequantised values q s
-                # (exact in bf16), every other weight stays as generated
-                L = self.layers[-1]
-                L.wg, L.wu, L.wd = (f8.quantize(L.wg)[2], f8.quantize(L.wu)[2], f8.quantize(L.wd)[2])
+        self.layers = [layer_weights(cfg, l) for l in range(cfg.n_layers if layers is None else layers)]
 
     def store(self, x):
         """Round float64 values to the storage dtype (returned as float64)."""

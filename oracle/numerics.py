@@ -21,8 +21,11 @@ result is fixed bit-for-bit by the definition itself:
 Each operation is one IEEE-754 binary32 operation with round-to-nearest-even
 (numpy float32 arithmetic, no fused multiply-add), so any other faithful
 implementation of the same operation sequence returns identical bits.  The
-pages never fix these details; they are the "Philox-counter sampling"
-reading recorded in the design notes.
+pages never fix these details: they only name Philox-counter sampling, and
+this is how it is read -- the sampler's decisions (tokens, commit masks) must
+come out the same on two implementations, so every draw is a Philox4x32-10
+word turned into an exact binary32 uniform and passed through this fixed
+operation sequence, never through a library log or exp.
 """
 from __future__ import annotations
 

@@ -310,7 +310,7 @@ def test_gemm_f32():
     (1024, 256, [0, 9, 64, 65, 1], 64, False),
     (1408, 2816, [17, 3, 0, 31, 12, 1, 9, 20], 256, True),
 ])
-@pytest.mark.parametrize("persistent", [False, True, "sized_ring", "m256"])
+@pytest.mark.parametrize("persistent", [False, True, "sized_ring", "m256", "streamk", "streamk256"])
 def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     g = np.random.default_rng(sum(counts) + M)
     G = len(counts)
@@ -326,9 +326,15 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     # item (more stages in flight), as the expert GEMMs run in the step
     # "m256": 256-row tiles (two accumulators), as the expert GEMMs run, with the
     # ring sized from the largest item
+    # "streamk": every SM takes an equal run of (tile, k block) iterations; a
+    # tile cut between runs is summed in k order by the CTA holding its start
+    # ("streamk256": the same over 256-row weight tiles)
+    sk = persistent in ("streamk", "streamk256")
+    if sk and not (bf and bn == 256):
+        pytest.skip("stream-K runs bf16 with 256-row item tiles")
     dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn, persistent=bool(persistent) and bf,
                          sized_ring=persistent in ("sized_ring", "m256") and bf,
-                         m256=persistent == "m256" and bf and bn == 256)
+                         m256=persistent in ("m256", "streamk256") and bf and bn == 256, streamk=sk)
     got = host(out).astype(np.float64)
     r0 = 0
     for e, c in enumerate(counts):
@@ -339,8 +345,9 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
         r0 += c
 
 
-@pytest.mark.parametrize("M,K,counts", [(1408, 2816, [17, 3, 0, 200, 12, 1, 256, 20]), (2048, 1024, [64, 65, 0, 9])])
-@pytest.mark.parametrize("m256", [False, True])
+@pytest.mark.parametrize("M,K,counts", [(1408, 2816, [17, 3, 0, 200, 12, 1, 256, 20]), (2048, 1024, [64, 65, 0, 9]),
+                                         (1408, 2816, [300, 1, 0, 5]), (1408, 2816, [16] * 120 + [40])])
+@pytest.mark.parametrize("m256", [False, True, "streamk", "streamk256"])
 def test_grouped_gemm_fused_swiglu(M, K, counts, m256):
     # the unsplit gate|up GEMM writes round(silu(g) u) itself; A rows interleave
     # gate / up in blocks of 64
@@ -350,7 +357,8 @@ def test_grouped_gemm_fused_swiglu(M, K, counts, m256):
     B = I._bf16_grid(g.standard_normal((rows, K)).astype(F32))
     out = torch.zeros((rows, M), dtype=torch.float32, device="cuda")
     dg.test_grouped_gemm(bf16_tensor(A), bf16_tensor(B), counts, G, M, out, bn=256, persistent=True,
-                         sized_ring=True, swiglu=True, m256=m256)
+                         sized_ring=True, swiglu=True, m256=m256 in (True, "streamk256"),
+                         streamk=m256 in ("streamk", "streamk256"))
     act = out.view(torch.bfloat16).reshape(-1)[:rows * ff].reshape(rows, ff)
     got = act.float().cpu().numpy().astype(np.float64)
     f = np.arange(ff)
@@ -426,7 +434,12 @@ def _attn_ref(q, k, v, n_canvas, n_q, q_pos0, causal, rows=None):
     (1, 256, 64, 320, False, 4, 4, False),
     (1, 64, 0, 64, True, 4, 4, False),
 ])
-def test_attention(n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, bf):
+@pytest.mark.parametrize("path", [0, 1, 2])
+def test_attention(n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, bf, path):
+    # path 0: the plan's choice; 1: split partials + combine kernel; 2: the
+    # splits of a query-tile pair merged inside the kernel (thread-block cluster)
+    if path and not bf:
+        pytest.skip("the merge paths are the bf16 kernel's")
     g = np.random.default_rng(n_keys + Hq)
     hd = 128 if bf else 64
     q = g.standard_normal((n_canvas * n_q, Hq, hd)).astype(F32)
@@ -436,14 +449,18 @@ def test_attention(n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, bf):
         q, k, v = I._bf16_grid(q), I._bf16_grid(k), I._bf16_grid(v)
     mk = bf16_tensor if bf else cu
     out = torch.empty((n_canvas * n_q, Hq * hd), dtype=torch.float32, device="cuda")
-    dg.test_attention(mk(q), mk(k), mk(v), n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out)
+    took = dg.test_attention(mk(q), mk(k), mk(v), n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out,
+                             force_path=path)
+    if path:
+        assert took == path
     got = host(out)
     ref = _attn_ref(q, k, v, n_canvas, n_q, q_pos0, causal)
     tol = 1.2e-2 if bf else 1e-5
     assert np.abs(got - ref).max() <= tol, np.abs(got - ref).max()
 
 
-def test_attention_long_context_sampled_rows():
+@pytest.mark.parametrize("path", [0, 2])
+def test_attention_long_context_sampled_rows(path):
     # 256 canvas queries over 32768 prompt + 256 canvas keys (split-KV path);
     # rows checked one by one against the definition.
     n_q, P, Hq, Hkv, hd = 256, 32768, 8, 2, 128
@@ -453,7 +470,8 @@ def test_attention_long_context_sampled_rows():
     k = I._bf16_grid(g.standard_normal((1, Hkv, n_keys, hd)).astype(F32))
     v = I._bf16_grid(g.standard_normal((1, Hkv, n_keys, hd)).astype(F32))
     out = torch.empty((n_q, Hq * hd), dtype=torch.float32, device="cuda")
-    dg.test_attention(bf16_tensor(q), bf16_tensor(k), bf16_tensor(v), 1, n_q, P, n_keys, False, Hq, Hkv, out)
+    dg.test_attention(bf16_tensor(q), bf16_tensor(k), bf16_tensor(v), 1, n_q, P, n_keys, False, Hq, Hkv, out,
+                      force_path=path)
     got = host(out).reshape(n_q, Hq, hd)
     for t in (0, 1, 77, 128, 255):
         for h in (0, 3, 7):

@@ -20,7 +20,7 @@ def lib():
 
 
 def plan(lib, n_q, G, Hkv, n_canvas, n_keys, cap=1 << 40):
-    out = (ctypes.c_int32 * 4)()
+    out = (ctypes.c_int32 * 5)()
     rows = n_q * G * Hkv * n_canvas
     assert lib.dg_test_attn_plan(n_q, G, Hkv, n_canvas, n_keys, rows, cap, out) == 0
     return list(out), rows
@@ -36,7 +36,7 @@ def plan(lib, n_q, G, Hkv, n_canvas, n_keys, cap=1 << 40):
     (1024, 4, 2, 1, 1024),       # causal encode chunk
 ])
 def test_attention_plan_covers_every_key_block_once(lib, n_q, G, Hkv, n_canvas, n_keys):
-    (q_tiles, n_splits, bps, ctas), rows = plan(lib, n_q, G, Hkv, n_canvas, n_keys)
+    (q_tiles, n_splits, bps, ctas, cluster), rows = plan(lib, n_q, G, Hkv, n_canvas, n_keys)
     nblocks = -(-n_keys // BK)
     assert q_tiles * 128 >= n_q * G and (q_tiles - 1) * 128 < n_q * G
     assert 1 <= n_splits <= nblocks
@@ -45,13 +45,24 @@ def test_attention_plan_covers_every_key_block_once(lib, n_q, G, Hkv, n_canvas, 
     assert ctas == base * n_splits
     if base <= SMS:
         assert ctas <= SMS or n_splits == 1                                  # the grid fills the SMs once
+    if cluster:
+        assert n_splits <= 8                                                 # a portable cluster merges the splits
 
 
 def test_attention_plan_respects_the_partial_buffer(lib):
-    (_, n_splits, _, _), rows = plan(lib, 256, 4, 2, 1, 33024, cap=3 * 256 * 4 * 2)
-    assert n_splits * rows <= 3 * 256 * 4 * 2
-    (_, n_splits, _, _), _ = plan(lib, 256, 4, 2, 1, 33024, cap=1)
-    assert n_splits == 1
+    (_, n_splits, _, _, cluster), rows = plan(lib, 256, 4, 2, 1, 33024, cap=3 * 256 * 4 * 2)
+    assert cluster or n_splits * rows <= 3 * 256 * 4 * 2
+    (_, n_splits, _, _, cluster), _ = plan(lib, 256, 4, 2, 1, 33024, cap=1)
+    assert cluster or n_splits == 1
+
+
+def test_attention_plan_merges_short_key_ranges_in_the_kernel(lib):
+    # the 26B-A4B canvas pass (2304 keys, 16 pairs x heads) and the mid one
+    # merge their splits inside a cluster; the 33k-key long context splits
+    # wider through the partial buffer
+    assert plan(lib, 256, 2, 8, 1, 2304)[0][4] == 1
+    assert plan(lib, 256, 4, 2, 1, 1280)[0][4] == 1
+    assert plan(lib, 256, 4, 2, 1, 33024)[0][4] == 0
 
 
 def _init_status(lib, w, **over):
@@ -86,3 +97,28 @@ def test_hook_arguments_are_checked_before_any_device_call(lib):
     assert lib.dg_test_grouped_gemm_fp8(P, P, P, c, 1, 128, 128, 48, 1, P, None) == 1
     # routing bias: n_tok not a multiple of 256
     assert lib.dg_set_routing_bias(None, P, 100) == 1
+
+
+@pytest.mark.parametrize("A,B,out", [
+    ((256, 64, "bf16"), (32, 64, "bf16"), (32, 128, "f32")),   # out too small for [N, M]
+    ((256, 64, "bf16"), (32, 48, "bf16"), (32, 256, "f32")),   # B's K differs from A's
+    ((256, 64, "f32"), (32, 64, "bf16"), (32, 256, "f32")),    # A not bf16
+    ((256, 64, "bf16"), (32, 64, "bf16"), (32, 256, "bf16")),  # out not fp32
+])
+def test_noalloc_binding_rejects_mismatched_tensors_before_any_call(A, B, out):
+    # the allocation-free GEMM writes out[N][M] through a raw pointer: a
+    # wrong shape or dtype must be refused on the host
+    torch = pytest.importorskip("torch")
+    dt = {"bf16": torch.bfloat16, "f32": torch.float32}
+    mk = lambda r, c, t: torch.zeros((r, c), dtype=dt[t])
+    with pytest.raises(ValueError):
+        dg.gemm_splitk_noalloc(mk(*A), mk(*B), mk(*out))
+
+
+def test_noalloc_binding_rejects_non_contiguous_operands():
+    torch = pytest.importorskip("torch")
+    A = torch.zeros((64, 256), dtype=torch.bfloat16).t()      # [256, 64], not contiguous
+    B = torch.zeros((32, 64), dtype=torch.bfloat16)
+    out = torch.zeros((32, 256), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        dg.gemm_splitk_noalloc(A, B, out)

@@ -454,3 +454,15 @@ def test_router_bias_closed_form_with_zero_input():
     assert ids.tolist() == [[2, 3], [0, 7], [3, 4]]
     expect = [1 / (1 + math.exp(-2.0)), 0.5, 1 / (1 + math.exp(-1.0))]
     assert np.allclose(gates[:, 0], expect, rtol=1e-14) and np.allclose(gates.sum(axis=1), 1.0)
+
+
+def test_lazy_expert_weights_equal_the_whole_tensor():
+    # per-expert generation (used for single-layer checks of the large
+    # workloads) is the same counter range of the same generator
+    for w in (I.TINY_FP32, I.MID_BF16.replace(n_layers=1)):
+        eager = om.layer_weights(w, 0)
+        lazy = om.layer_weights(w, 0, lazy_experts=True)
+        for name in ("wg", "wu", "wd"):
+            full = getattr(eager, name)
+            for e in (0, w.n_experts // 2, w.n_experts - 1):
+                assert np.array_equal(lazy.__dict__[name][e].view(np.uint32), full[e].view(np.uint32)), (name, e)

@@ -5,9 +5,10 @@ device memory at start-up, or code that must never block other streams
 (cudaMalloc/cudaFree can synchronise the device and fail under memory
 pressure).  dg_gemm_splitk_noalloc keeps its partial sums in a fixed-size
 array inside the library instead.  These tests call it through the C ABI and
-check it against the existing GEMM entry point (dg_test_gemm) on two calls in
-a row -- the second call reuses the array the first one filled -- and that
-it refuses a problem larger than the array.  This file is collected last."""
+check it against the existing GEMM entry point (dg_test_gemm) and against an
+fp64 host product on calls in a row -- each later call reuses the array the
+earlier, larger one filled -- and that it refuses a problem larger than the
+array.  This file is collected last."""
 import ctypes
 
 import numpy as np
@@ -31,21 +32,33 @@ def _bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda().to(torch.bfloat16)
 
 
+# (M, N, K, k_splits): the larger problem first, so the second call runs on an
+# array still holding the first call's bigger slabs; M and K tails (M not a
+# multiple of 128, K not a multiple of 64) and a split count above the number
+# of 64-wide K blocks (clamped to it).
+CASES = ((4096, 200, 2816, 3), (1000, 77, 1000, 64), (1536, 256, 1024, 4))
+
+
 def test_noalloc_gemm_matches_existing_entry_point_on_two_calls():
-    for M, N, K, splits in ((1536, 256, 1024, 4), (4096, 200, 2816, 3)):
+    for M, N, K, splits in CASES:
         g = np.random.default_rng(M + N + K)
         A = I._bf16_grid(g.standard_normal((M, K)).astype(np.float32))
         B = I._bf16_grid(g.standard_normal((N, K)).astype(np.float32))
         At, Bt = _bf16(A), _bf16(B)
-        ref = torch.zeros((splits, N, M), dtype=torch.float32, device="cuda")
-        dg.test_gemm(At, Bt, ref, alpha=1.0, k_splits=splits, bn=256)
+        used = min(splits, -(-K // 64))
+        ref = torch.zeros((used, N, M), dtype=torch.float32, device="cuda")
+        dg.test_gemm(At, Bt, ref, alpha=1.0, k_splits=used, bn=256)
         out = torch.full((N, M), float("nan"), dtype=torch.float32, device="cuda")
         dg.gemm_splitk_noalloc(At, Bt, out, k_splits=splits)
         torch.cuda.synchronize()
         got = out.cpu().numpy().astype(np.float64)
         want = ref.cpu().numpy().astype(np.float64).sum(axis=0)
+        exact = B.astype(np.float64) @ A.astype(np.float64).T
         bound = np.abs(B.astype(np.float64)) @ np.abs(A.astype(np.float64)).T
-        assert np.all(np.abs(got - want) <= 2e-6 * bound), np.abs(got - want).max()
+        # against the existing entry point and against the fp64 product, with
+        # the bound the GEMM parity tests use
+        assert np.all(np.abs(got - want) <= 2e-6 * bound), (M, N, K, np.abs(got - want).max())
+        assert np.all(np.abs(got - exact) <= 2e-6 * bound), (M, N, K, np.abs(got - exact).max())
 
 
 def test_noalloc_gemm_rejects_problems_larger_than_its_array():
