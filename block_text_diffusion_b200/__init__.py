@@ -88,6 +88,8 @@ def lib():
             "dg_expert_counts": ([P, P, P], I32),
             "dg_debug_trace": ([P, P, P], I32),
             "dg_test_layer": ([P, P, I32, I32, I32, P, P, P, P], I32),
+            "dg_test_moe": ([P, I32, I32, P, P, P, P], I32),
+            "dg_test_attn_capacity": ([P], I32),
             "dg_touched_experts_sum": ([P, P, I32, P], I32),
             "dg_gemm_splitk_noalloc": ([P, P, P, I32, I32, I32, I32, P], I32),
         }
@@ -205,6 +207,14 @@ class Model:
         int32 [B*256, top_k] the routing; the canvas keys/values go into kv."""
         _check(lib().dg_test_layer(self.h, _ptr(kv), B, P, layer, _ptr(h_in), _ptr(h_trace), _ptr(ids),
                                    _stream(stream)), "dg_test_layer")
+
+    def run_moe(self, B, layer, h_attn, h_trace, ids, stream=None):
+        """The MoE half of layer `layer` from the residual state h_attn
+        [B*256, d] (model dtype) after its attention: h_trace fp32
+        [3, B*256, d] receives h after the MoE in row 1 and its RMSNorm in
+        row 2; ids int32 [B*256, top_k] the routing."""
+        _check(lib().dg_test_moe(self.h, B, layer, _ptr(h_attn), _ptr(h_trace), _ptr(ids), _stream(stream)),
+               "dg_test_moe")
 
     def expert_counts(self, counts, stream=None):
         """Per-layer expert row counts [n_layers, n_experts] of the most recent call."""
@@ -329,12 +339,11 @@ def test_router(x, wr, ids, gate, bias=None, tok_bias=None, stream=None):
 
 
 def test_grouped_gemm(A, B, counts, groups, M, out, bn=64, persistent=False, sized_ring=False, swiglu=False,
-                      m256=False, streamk=False, stream=None):
+                      m256=False, stream=None):
     import torch
     K = A.shape[-1]
     c = (ctypes.c_int32 * groups)(*[int(x) for x in counts])
-    flags = (int(persistent) | (2 if sized_ring else 0) | (4 if swiglu else 0) | (8 if m256 else 0)
-             | (16 if streamk else 0))
+    flags = int(persistent) | (2 if sized_ring else 0) | (4 if swiglu else 0) | (8 if m256 else 0)
     _check(lib().dg_test_grouped_gemm(_ptr(A), _ptr(B), c, groups, M, K, 1 if A.dtype == torch.bfloat16 else 0,
                                       bn, flags, _ptr(out), _stream(stream)), "dg_test_grouped_gemm")
 
@@ -349,6 +358,14 @@ def test_attention(q, k, v, n_canvas, n_q, q_pos0, n_keys, causal, Hq, Hkv, out,
                                    Hkv, hd, 1 if q.dtype == torch.bfloat16 else 0, int(force_path),
                                    ctypes.byref(path), _ptr(out), _stream(stream)), "dg_test_attention")
     return path.value
+
+
+def attn_cluster_capacity():
+    """Resident thread-block clusters of the bf16 attention kernel per cluster
+    size 1..8 (index 0 unused), as the device reports them."""
+    out = (ctypes.c_int32 * 9)()
+    _check(lib().dg_test_attn_capacity(out), "dg_test_attn_capacity")
+    return list(out)
 
 
 def gemm_splitk_noalloc(A, B, out, k_splits=1, stream=None):

@@ -65,33 +65,36 @@ static_assert(256 * 128 * 4 <= kAttnSmem - 1024, "the merge staging reuses the p
 // per CTA; the key range is split so that pairs x splits fill the SMs about
 // once (one CTA per SM), capped by the partial-output rows available.  The
 // in-kernel cluster merge (at most kAttnMaxCluster splits, no partial
-// outputs in global memory, no combine launch) is taken when its estimated
-// time -- key blocks per split plus the merge -- beats the wider split with
-// the global partials and the combine kernel.
+// outputs in global memory, no combine launch) is taken when its clusters
+// all fit on the GPU at once (max_clusters[c] = clusters of c CTAs that can
+// be resident together; null: SMs / c) and its estimated time -- key blocks
+// per split plus the merge -- beats the wider split with the global partials
+// and the combine kernel.
 struct AttnPlan {
   int q_tiles, n_splits, blocks_per_split, ctas, cluster;
 };
 inline AttnPlan attn_plan(long long n_q, int G, int Hkv, int n_canvas, int n_keys, long long rows,
-                          long long part_rows_cap) {
+                          long long part_rows_cap, const int* max_clusters = nullptr) {
   AttnPlan p;
   p.q_tiles = (int)((n_q * G + 127) / 128);
   const int nblocks = (n_keys + kAttnBK - 1) / kAttnBK;
   const int base = (p.q_tiles + 1) / 2 * Hkv * n_canvas;
   const int wide = std::max(1, std::min(nblocks, kSMs / std::max(1, base)));
-  const int narrow = std::min(wide, kAttnMaxCluster);
   // microseconds: ~0.8 per key block, ~1.5 for the cluster merge, ~7.5 for
   // the partial outputs plus the combine kernel
-  const double t_narrow = 0.8 * ((nblocks + narrow - 1) / narrow) + 1.5;
-  const double t_wide = 0.8 * ((nblocks + wide - 1) / wide) + 7.5;
-  int splits;
-  if (t_narrow <= t_wide) {
-    splits = narrow;
-    p.cluster = 1;
-  } else {
-    splits = wide;
-    while (splits > 1 && (long long)splits * rows > part_rows_cap) --splits;
-    p.cluster = 0;
+  auto blocks_of = [&](int splits) { return (nblocks + splits - 1) / splits; };
+  double best = 0.8 * blocks_of(wide) + 7.5;
+  int splits = wide;
+  p.cluster = 0;
+  for (int c = std::min(wide, kAttnMaxCluster); c >= 1; --c) {
+    const int n = (nblocks + blocks_of(c) - 1) / blocks_of(c);   // splits actually used
+    const int fit = max_clusters ? max_clusters[n] : kSMs / n;
+    if (base > fit) continue;
+    const double t = 0.8 * blocks_of(c) + 1.5;
+    if (t < best) { best = t; splits = c; p.cluster = 1; }
   }
+  if (!p.cluster)
+    while (splits > 1 && (long long)splits * rows > part_rows_cap) --splits;
   p.blocks_per_split = (nblocks + splits - 1) / splits;
   p.n_splits = (nblocks + p.blocks_per_split - 1) / p.blocks_per_split;
   p.ctas = base * p.n_splits;

@@ -178,6 +178,19 @@ __device__ __forceinline__ long long q40_trunc(float x) {
   return (b >> 31) ? -(long long)v : (long long)v;
 }
 
+// Adds trunc(x * 2^40) to a Q40 sum kept in two parts.  A binary32 x with
+// |x| >= 2^-17 is a multiple of 2^-40, so trunc(x 2^40) = x 2^40 exactly and
+// a float64 sum of such x is exact while it stays below 2^13 in magnitude
+// (a thread adds at most a few hundred terms of magnitude <= 1); smaller
+// terms take the integer truncation.  q40_total joins the parts exactly.
+__device__ __forceinline__ void q40_add(float x, long long& iq, double& dq) {
+  if (fabsf(x) >= 7.62939453125e-06f) dq += (double)x;
+  else iq += q40_trunc(x);
+}
+__device__ __forceinline__ long long q40_total(long long iq, double dq) {
+  return iq + (long long)(dq * 1099511627776.0);   // dq 2^40 is an integer below 2^53
+}
+
 // cos(2 pi u) for u in (0,1): fold to b in [0,1/8] by the cosine symmetries,
 // then the Taylor series of cos (through x^10) or sin (through x^11).
 __device__ __forceinline__ float dg_cos2pif(float u) {

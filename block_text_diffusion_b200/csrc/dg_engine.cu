@@ -127,9 +127,12 @@ struct LayerW {
 
 // Tile-shape overrides for sweeps, read once from DG_TUNE="key=value,..."
 // (dense_bn, dense_splits, router_bn, router_splits, qkv_fused; 0 keeps the
-// default).
+// default; attn_merge = 1 always merges attention key splits with the
+// combine kernel, 2 always inside the kernel when the splits fit a cluster;
+// down_m256 = 1 runs the down GEMM on 256-row tiles).
 struct Tune {
-  int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0, qkv_fused = 0;
+  int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0, qkv_fused = 0, attn_merge = 0,
+      down_m256 = 0;
 };
 inline Tune read_tune() {
   Tune t;
@@ -150,6 +153,8 @@ inline Tune read_tune() {
       else if (k == "router_bn") t.router_bn = v;
       else if (k == "router_splits") t.router_splits = v;
       else if (k == "qkv_fused") t.qkv_fused = v;
+      else if (k == "attn_merge") t.attn_merge = v;
+      else if (k == "down_m256") t.down_m256 = v;
     }
     pos = end + 1;
   }
@@ -187,7 +192,6 @@ struct dg_model {
   void* cand_w = nullptr;
   BMaps tm_x, tm_o, tm_xp, tm_act, tm_probs, tm_u;   // activation (B) operands
   float* ws = nullptr;
-  StreamK sk{};                      // stream-K expert GEMMs: partial slots [SMs][2][256][128], flags [SMs]
   float *o_part = nullptr, *lse_part = nullptr;
   int *ids = nullptr, *perm = nullptr, *inv = nullptr, *work_count = nullptr, *counts = nullptr;
   int* moe_splits = nullptr;         // [3] split-K of the gate|up and down GEMMs, largest item rows (set by permute)
@@ -326,8 +330,6 @@ struct GemmCall {
   void* act = nullptr;               // persistent gate|up: SwiGLU output (bf16) when the GEMM runs unsplit
   int act_ld = 0;
   bool m256 = false;                 // dense, bn 256: 256-row M tiles (two accumulators share B)
-  bool streamk = false;              // grouped bf16, bn 256: stream-K over every SM (fused SwiGLU when act is set)
-  StreamK sk{};
   int qkv_on = 0;                    // dense bf16, one split: fused QKV post-process
   QkvEpi qkv{};
 };
@@ -365,24 +367,6 @@ dg_status launch_tc_persistent(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
   const int per_sm = std::max(1, (228 * 1024) / (C::kSmem + 2048));
   const int grid = (int)std::min<long long>(max_tiles, (long long)kSMs * std::min(per_sm, 2));
   launch_pdl(k_gemm_tc_persistent<BN, ST, MT>, grid, 192, C::kSmem, s, *g.tA, *g.tB, a, items_dense);
-  CU_TRY(cudaGetLastError());
-  return DG_OK;
-}
-
-// Stream-K grouped GEMM: one CTA per SM (every CTA resident at once);
-// MT = 2 for 256-row tiles.
-template <int MT>
-dg_status launch_tc_streamk(const GemmCall& g, GemmArgs& a, cudaStream_t s) {
-  constexpr int kStages = MT == 2 ? 3 : 4;
-  using C = GemmTcCfg<256, kStages, MT>;
-  static bool attr = false;
-  if (!attr) {
-    CU_TRY(cudaFuncSetAttribute(k_gemm_tc_streamk<256, kStages, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                C::kSmem));
-    attr = true;
-  }
-  if (!g.sk.seg_ws || !g.sk.seg_flag) return DG_ERR_STATE;
-  launch_pdl(k_gemm_tc_streamk<256, kStages, MT>, kSMs, 192, C::kSmem, s, *g.tA, *g.tB, a, g.sk);
   CU_TRY(cudaGetLastError());
   return DG_OK;
 }
@@ -459,16 +443,6 @@ dg_status gemm(dg_model* m, const GemmCall& g, int phase, cudaStream_t s) {
   }
   a.m_tiles = cdiv(g.M, 128);
   a.n_tile = g.bn;
-  if (g.streamk) {
-    if (!g.work || g.bn != 256) return DG_ERR_UNSUPPORTED;
-    a.k_splits = 1;
-    a.max_rows_dev = g.max_rows_dev;
-    if (g.m256) {
-      a.m_tiles = cdiv(g.M, 256);
-      return launch_tc_streamk<2>(g, a, s);
-    }
-    return launch_tc_streamk<1>(g, a, s);
-  }
   if (g.persistent) {
     if (g.m256 && g.bn == 256) {   // 256-row tiles: two accumulators share each B tile
       a.m_tiles = cdiv(g.M, 256);
@@ -661,6 +635,40 @@ bool attn_maps(const dg_model* m, const KvGeom& g, int n_keys, int T_q, AttnMaps
   return ok;
 }
 
+// Clusters of c attention CTAs (c = 1 .. kAttnMaxCluster) that can be
+// resident on the current device at once, from the occupancy calculator
+// (queried once; entry 0 unused).
+const int* attn_cluster_capacity() {
+  static const std::vector<int> cap = [] {
+    std::vector<int> v(kAttnMaxCluster + 1, 0);
+    if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess) {
+      cudaGetLastError();
+      return v;
+    }
+    for (int c = 1; c <= kAttnMaxCluster; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)c);
+      cfg.blockDim = dim3(kAttnThreads);
+      cfg.dynamicSmemBytes = kAttnSmem;
+      cudaLaunchAttribute at;
+      at.id = cudaLaunchAttributeClusterDimension;
+      at.val.clusterDim.x = (unsigned)c;
+      at.val.clusterDim.y = 1;
+      at.val.clusterDim.z = 1;
+      cfg.attrs = &at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, (void*)k_attn_tc, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      v[c] = n;
+    }
+    return v;
+  }();
+  return cap.data();
+}
+
 // The tensor-core attention: one launch of the plan's CTAs; with the in-kernel
 // merge the split CTAs of a query-tile pair form one thread-block cluster.
 dg_status launch_attn_tc(const AttnPlan& ap, const AttnMaps& am, const AttnArgs& aa, cudaStream_t s) {
@@ -694,6 +702,126 @@ dg_status launch_attn_tc(const AttnPlan& ap, const AttnMaps& am, const AttnArgs&
   return DG_OK;
 }
 
+// The MoE half of layer l over Tn tokens: router and top-k on m->x (RMSNorm
+// of the residual state m->h), permutation, expert gate|up GEMM, SwiGLU,
+// down GEMM, and the weighted combine into m->h with RMSNorm of the result
+// left in m->x.  lt is the diagnostic trace slot of the layer; `last` also
+// traces the normalised state the layer leaves.
+template <typename T>
+dg_status run_moe(dg_model* m, int l, int lt, int Tn, int b0, int n_per, bool causal, bool last, cudaStream_t s) {
+  const LayerW& w = m->layers[l];
+  const int d = m->d;
+  const int n_pairs = Tn * m->k;
+  // one work item per expert (up to 256 rows): each expert's weights are
+  // streamed once per split however many rows it received
+  const int bn_g = m->bf ? 256 : 64;
+  const int max_items = m->E + cdiv(n_pairs, bn_g);
+  // per-token router bias: canvas passes only, rows of canvases b0 ..
+  const float* tb = (!causal && m->tok_bias)
+                        ? m->tok_bias + ((size_t)l * m->tok_bias_n + (size_t)b0 * n_per) * m->E : nullptr;
+  if (tb && b0 * n_per + Tn > m->tok_bias_n) return DG_ERR_INVALID_ARG;
+  // expert GEMM split-K factors are picked on the device from the routing
+  // (bf16 persistent path only; the fp32 path keeps one split)
+  const long long gu_stride = (long long)n_pairs * 2 * m->ff, dn_stride = (long long)n_pairs * d;
+  SplitPlan plan{};
+  // bf16 gate|up runs 256-row tiles (two accumulators per CTA share each B
+  // tile; its long K amortises the unoverlapped epilogue); down keeps
+  // 128-row tiles with double-buffered accumulators (K = ff is short)
+  plan.mt[0] = cdiv(2 * m->ff, m->bf ? 256 : 128); plan.kb[0] = cdiv(d, 64);
+  const bool down256 = m->bf && !m->fp8 && m->tune.down_m256 == 1;
+  plan.mt[1] = cdiv(d, down256 ? 256 : 128); plan.kb[1] = cdiv(m->ff, 64);
+  plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
+  plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
+  plan.fused0 = m->bf ? 1 : 0;
+  if (m->fp8) {
+    // FP8 experts: 128-row tiles, split-K over 128-input chunks, SwiGLU as
+    // its own kernel
+    plan.mt[0] = cdiv(2 * m->ff, 128);
+    plan.kb[0] = cdiv(d, kF8Chunk);
+    plan.kb[1] = cdiv(m->ff, kF8Chunk);
+    plan.fused0 = 0;
+  }
+  plan.out = m->moe_splits;
+  const PermuteArgs pa{m->ids, n_pairs, m->E, bn_g, m->perm, m->inv, m->work, m->work_count,
+                       m->counts + (size_t)l * m->E, plan, causal ? nullptr : m->touched_acc + l, &m->st->err};
+  // router: logits r = x Wr^T (fp32 accumulation) and top-k.  Up to 128
+  // experts (bf16): one clustered kernel; otherwise a GEMM then a top-k kernel.
+  if (m->bf && m->E <= 128 && m->k <= 32) {
+    LaunchScope ls(m, s, PH_ROUTER);
+    static bool attr = false;
+    if (!attr) {
+      CU_TRY(cudaFuncSetAttribute(k_router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterSmem));
+      attr = true;
+    }
+    RouterArgs ra{m->E, m->k, Tn, cdiv(d, 64), m->rbias, tb, m->ids, m->gate, &m->st->err};
+    launch_pdl(k_router_tc, cdiv(Tn, kRouterBN) * kRouterSplits, 128, kRouterSmem, s, w.tm_wr, m->tm_x.m[0], ra);
+    CU_TRY(cudaGetLastError());
+  } else {
+  GemmCall rc;
+  rc.tA = &w.tm_wr; rc.tB = &m->tm_x; rc.A32 = (const float*)w.wr; rc.B32 = (const float*)m->x;
+  rc.lda = d; rc.ldb = d; rc.M = m->E; rc.K = d; rc.N = Tn; rc.out = m->ws; rc.ldo = m->E;
+  rc.bn = tuned_bn(dense_bn(Tn), m->tune.router_bn);
+  {
+    const int mt = m->bf ? cdiv(m->E, 128) : cdiv(m->E, 64);
+    const int items = m->bf ? cdiv(Tn, rc.bn) : cdiv(Tn, 64);
+    rc.splits = pick_splits(mt, items, cdiv(d, 64), m->tune.router_splits ? m->tune.router_splits : 8);
+    while (rc.splits > 1 && (size_t)rc.splits * Tn * m->E > m->ws_elems) --rc.splits;
+    rc.split_stride = (long long)Tn * m->E;
+  }
+  DG_TRY(gemm(m, rc, PH_ROUTER, s));
+  { LaunchScope ls(m, s, PH_ROUTER);
+    launch_pdl(k_router_topk, cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s, 
+        m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, tb, m->E, m->k, Tn, m->ids, m->gate); }
+  }
+  { LaunchScope ls(m, s, PH_PERMUTE);
+    launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, pa); }
+  { LaunchScope ls(m, s, PH_GATHER);
+    launch_pdl(k_gather<T>, n_pairs, 128, 0, s, (const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
+  GemmCall gu;
+  gu.tA = &w.tm_gu; gu.tB = &m->tm_xp; gu.A32 = (const float*)w.gu; gu.B32 = (const float*)m->xp;
+  gu.lda = d; gu.ldb = d; gu.M = 2 * m->ff; gu.K = d; gu.out = m->ws; gu.ldo = 2 * m->ff;
+  gu.work = m->work; gu.work_count = m->work_count; gu.a_group_rows = 2 * m->ff;
+  gu.max_items = max_items; gu.bn = bn_g; gu.persistent = m->bf;
+  gu.split_stride = gu_stride; gu.k_splits_dev = m->bf ? m->moe_splits : nullptr;
+  gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
+  gu.splits = m->bf ? 8 : 1;
+  // bf16: an unsplit gate|up GEMM applies SwiGLU in its epilogue
+  if (m->bf && !m->fp8) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = true; }
+  if (m->fp8) DG_TRY(gemm_f8(m, gu, &w.tm_gu8, w.gu_s, (long long)m->E * 2 * m->ff, PH_GU_GEMM, s));
+  else DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
+  // sums the split-K partials and applies SwiGLU; nothing to do when the
+  // bf16 gate|up GEMM ran unsplit and applied it in its epilogue.  One wave
+  // of CTAs (a grid-stride loop), so an empty pass drains at once.
+  { LaunchScope ls(m, s, PH_SWIGLU);
+    const long long n = (long long)n_pairs * m->ff;
+    launch_pdl(k_swiglu<T>, std::min(cdiv(n / 4, 256), kSMs * 8), 256, 0, s, m->ws, m->ff, n, (T*)m->act,
+               m->moe_splits, gu_stride, (m->bf && !m->fp8) ? 1 : 0); }
+  GemmCall dn;
+  dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
+  dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;
+  dn.work = m->work; dn.work_count = m->work_count; dn.a_group_rows = d;
+  dn.max_items = max_items; dn.bn = bn_g; dn.persistent = m->bf;
+  dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
+  dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
+  dn.splits = m->bf ? 8 : 1;
+  dn.m256 = down256;
+  if (m->fp8) DG_TRY(gemm_f8(m, dn, &w.tm_wd8, w.wd_s, (long long)m->E * d, PH_DOWN_GEMM, s));
+  else DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
+  { LaunchScope ls(m, s, PH_COMBINE);
+    launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
+               m->c.rms_eps, m->moe_splits + 1, dn_stride); }
+  if (m->dbg_h) {
+    launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * lt + 1) * Tn * d,
+                                       (long long)Tn * d);
+    CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)lt * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
+                           cudaMemcpyDeviceToDevice, s));
+    if (last)   // the normalised state the layers leave (LM head input after the last layer)
+      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->x, m->dbg_h + (size_t)(2 * lt + 2) * Tn * d,
+                 (long long)Tn * d);
+  }
+  return DG_OK;
+}
+
 // ---------------------------------------------------------------------------
 // One transformer layer stack over `T` tokens of `n_canvas` canvases
 // (n_per tokens each, positions pos0..), writing keys/values into the cache.
@@ -706,11 +834,6 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
   const int d = m->d, nq = m->hq * m->hd;
   AttnMaps am;
   if (m->bf && !attn_maps(m, g, n_keys, Tn, am)) return DG_ERR_CUDA;
-  const int n_pairs = Tn * m->k;
-  // one work item per expert (up to 256 rows): each expert's weights are
-  // streamed once per split however many rows it received
-  const int bn_g = m->bf ? 256 : 64;
-  const int max_items = m->E + cdiv(n_pairs, bn_g);
 
   // Precondition: m->x holds RMSNorm(h) of the first layer (written by the
   // embedding kernel); every layer leaves RMSNorm of its output in m->x.
@@ -761,7 +884,15 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
     {
       LaunchScope ls(m, s, PH_ATTN);
       if (m->bf) {
-        const AttnPlan ap = attn_plan(n_per, m->G, m->hkv, n_canvas, n_keys, rows, (long long)m->part_rows_cap);
+        // attn_merge tuning: 1 = combine kernel, 2 = in-kernel merge whenever the clusters fit
+        static int cap_all[kAttnMaxCluster + 1];
+        const int* cap = attn_cluster_capacity();
+        if (m->tune.attn_merge == 1) {
+          for (int c = 0; c <= kAttnMaxCluster; ++c) cap_all[c] = 0;
+          cap = cap_all;
+        }
+        AttnPlan ap = attn_plan(n_per, m->G, m->hkv, n_canvas, n_keys, rows, (long long)m->part_rows_cap, cap);
+        if (m->tune.attn_merge == 1 && ap.cluster) ap.cluster = 0;
         aa.q_tiles = ap.q_tiles; aa.n_splits = ap.n_splits; aa.blocks_per_split = ap.blocks_per_split;
         aa.cluster = ap.cluster; aa.o_out = (bf16*)m->o;
         attn_merged = ap.cluster != 0;
@@ -797,110 +928,7 @@ dg_status run_layers(dg_model* m, const KvGeom& g, int b0, int n_canvas, int n_p
                                             std::min(oc.splits, cdiv(nq, 64)), d, m->c.rms_eps); }
     if (m->dbg_h)
       launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * lt) * Tn * d, (long long)Tn * d);
-    // MoE
-    // per-token router bias: canvas passes only, rows of canvases b0 ..
-    const float* tb = (!causal && m->tok_bias)
-                          ? m->tok_bias + ((size_t)l * m->tok_bias_n + (size_t)b0 * n_per) * m->E : nullptr;
-    if (tb && (b0 + n_canvas) * n_per > m->tok_bias_n) return DG_ERR_INVALID_ARG;
-    // router: logits r = x Wr^T (fp32 accumulation) and top-k.  Up to 128
-    // experts (bf16): one clustered kernel; otherwise a GEMM then a top-k kernel.
-    if (m->bf && m->E <= 128 && m->k <= 32) {
-      LaunchScope ls(m, s, PH_ROUTER);
-      static bool attr = false;
-      if (!attr) {
-        CU_TRY(cudaFuncSetAttribute(k_router_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterSmem));
-        attr = true;
-      }
-      RouterArgs ra{m->E, m->k, Tn, cdiv(d, 64), m->rbias, tb, m->ids, m->gate, &m->st->err};
-      launch_pdl(k_router_tc, cdiv(Tn, kRouterBN) * kRouterSplits, 128, kRouterSmem, s, w.tm_wr, m->tm_x.m[0], ra);
-      CU_TRY(cudaGetLastError());
-    } else {
-    GemmCall rc;
-    rc.tA = &w.tm_wr; rc.tB = &m->tm_x; rc.A32 = (const float*)w.wr; rc.B32 = (const float*)m->x;
-    rc.lda = d; rc.ldb = d; rc.M = m->E; rc.K = d; rc.N = Tn; rc.out = m->ws; rc.ldo = m->E;
-    rc.bn = tuned_bn(dense_bn(Tn), m->tune.router_bn);
-    {
-      const int mt = m->bf ? cdiv(m->E, 128) : cdiv(m->E, 64);
-      const int items = m->bf ? cdiv(Tn, rc.bn) : cdiv(Tn, 64);
-      rc.splits = pick_splits(mt, items, cdiv(d, 64), m->tune.router_splits ? m->tune.router_splits : 8);
-      while (rc.splits > 1 && (size_t)rc.splits * Tn * m->E > m->ws_elems) --rc.splits;
-      rc.split_stride = (long long)Tn * m->E;
-    }
-    DG_TRY(gemm(m, rc, PH_ROUTER, s));
-    { LaunchScope ls(m, s, PH_ROUTER);
-      launch_pdl(k_router_topk, cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s, 
-          m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, tb, m->E, m->k, Tn, m->ids, m->gate); }
-    }
-    // expert GEMM split-K factors are picked on the device from the routing
-    // (bf16 persistent path only; the fp32 path keeps one split)
-    const long long gu_stride = (long long)n_pairs * 2 * m->ff, dn_stride = (long long)n_pairs * d;
-    SplitPlan plan{};
-    // bf16 gate|up runs 256-row tiles (two accumulators per CTA share each B
-    // tile; its long K amortises the unoverlapped epilogue); down keeps
-    // 128-row tiles with double-buffered accumulators (K = ff is short)
-    plan.mt[0] = cdiv(2 * m->ff, m->bf ? 256 : 128); plan.kb[0] = cdiv(d, 64);
-    plan.mt[1] = cdiv(d, 128); plan.kb[1] = cdiv(m->ff, 64);
-    plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
-    plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
-    plan.fused0 = m->bf ? 1 : 0;
-    if (m->fp8) {
-      // FP8 experts: 128-row tiles, split-K over 128-input chunks, SwiGLU as
-      // its own kernel
-      plan.mt[0] = cdiv(2 * m->ff, 128);
-      plan.kb[0] = cdiv(d, kF8Chunk);
-      plan.kb[1] = cdiv(m->ff, kF8Chunk);
-      plan.fused0 = 0;
-    }
-    plan.out = m->moe_splits;
-    { LaunchScope ls(m, s, PH_PERMUTE);
-      launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, m->ids, n_pairs, m->E, bn_g, m->perm, m->inv,
-                 m->work, m->work_count, m->counts + (size_t)l * m->E, plan,
-                 causal ? nullptr : m->touched_acc + l, &m->st->err); }
-    { LaunchScope ls(m, s, PH_GATHER);
-      launch_pdl(k_gather<T>, n_pairs, 128, 0, s, (const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
-    GemmCall gu;
-    gu.tA = &w.tm_gu; gu.tB = &m->tm_xp; gu.A32 = (const float*)w.gu; gu.B32 = (const float*)m->xp;
-    gu.lda = d; gu.ldb = d; gu.M = 2 * m->ff; gu.K = d; gu.out = m->ws; gu.ldo = 2 * m->ff;
-    gu.work = m->work; gu.work_count = m->work_count; gu.a_group_rows = 2 * m->ff;
-    gu.max_items = max_items; gu.bn = bn_g; gu.persistent = m->bf;
-    gu.split_stride = gu_stride; gu.k_splits_dev = m->bf ? m->moe_splits : nullptr;
-    gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
-    gu.splits = m->bf ? 8 : 1;
-    // bf16: stream-K over every SM with SwiGLU in the epilogue (no partial
-    // slabs, no separate activation pass); FP8 experts: split-K then SwiGLU
-    const bool sk = m->bf && !m->fp8;
-    if (sk) { gu.act = m->act; gu.act_ld = m->ff; gu.streamk = true; gu.m256 = true; gu.sk = m->sk; }
-    if (m->fp8) DG_TRY(gemm_f8(m, gu, &w.tm_gu8, w.gu_s, (long long)m->E * 2 * m->ff, PH_GU_GEMM, s));
-    else DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
-    if (!sk) {
-      LaunchScope ls(m, s, PH_SWIGLU);
-      const long long n = (long long)n_pairs * m->ff;
-      launch_pdl(k_swiglu<T>, std::min(cdiv(n / 4, 256), kSMs * 16), 256, 0, s, m->ws, m->ff, n, (T*)m->act,
-                 m->moe_splits, gu_stride, 0);
-    }
-    GemmCall dn;
-    dn.tA = &w.tm_wd; dn.tB = &m->tm_act; dn.A32 = (const float*)w.wd; dn.B32 = (const float*)m->act;
-    dn.lda = m->ff; dn.ldb = m->ff; dn.M = d; dn.K = m->ff; dn.out = m->ws; dn.ldo = d;
-    dn.work = m->work; dn.work_count = m->work_count; dn.a_group_rows = d;
-    dn.max_items = max_items; dn.bn = bn_g; dn.persistent = m->bf;
-    dn.split_stride = dn_stride; dn.k_splits_dev = m->bf ? m->moe_splits + 1 : nullptr;
-    dn.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
-    dn.splits = m->bf ? 8 : 1;
-    if (sk) { dn.streamk = true; dn.sk = m->sk; }
-    if (m->fp8) DG_TRY(gemm_f8(m, dn, &w.tm_wd8, w.wd_s, (long long)m->E * d, PH_DOWN_GEMM, s));
-    else DG_TRY(gemm(m, dn, PH_DOWN_GEMM, s));
-    { LaunchScope ls(m, s, PH_COMBINE);
-      launch_pdl(k_moe_combine_norm<T>, Tn, 256, 0, s, (T*)m->h, (T*)m->x, m->ws, m->inv, m->gate, m->k, d,
-                 m->c.rms_eps, sk ? nullptr : m->moe_splits + 1, dn_stride); }
-    if (m->dbg_h) {
-      launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->h, m->dbg_h + (size_t)(2 * lt + 1) * Tn * d,
-                                         (long long)Tn * d);
-      CU_TRY(cudaMemcpyAsync(m->dbg_ids + (size_t)lt * n_pairs, m->ids, (size_t)n_pairs * sizeof(int),
-                             cudaMemcpyDeviceToDevice, s));
-      if (l == l_end - 1)   // the normalised state the layers leave (LM head input after the last layer)
-        launch_pdl(k_cast_f32<T>, kSMs, 256, 0, s, (const T*)m->x,
-                   m->dbg_h + (size_t)(2 * (l_end - l_first)) * Tn * d, (long long)Tn * d);
-    }
+    DG_TRY(run_moe<T>(m, l, lt, Tn, b0, n_per, causal, l == l_end - 1, s));
   }
   CU_TRY(cudaGetLastError());
   return DG_OK;
@@ -1255,10 +1283,6 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   A(&m->u, (size_t)m->T_cap * d * es);
   A(&m->sc, (size_t)m->T_cap * d * es);
   A((void**)&m->ws, m->ws_elems * sizeof(float));
-  if (m->bf) {
-    A((void**)&m->sk.seg_ws, (size_t)kSMs * 2 * 256 * 128 * sizeof(float));
-    A((void**)&m->sk.seg_flag, (size_t)kSMs * sizeof(int));
-  }
   A((void**)&m->o_part, m->part_rows_cap * m->hd * sizeof(float));
   A((void**)&m->lse_part, m->part_rows_cap * sizeof(float));
   A((void**)&m->ids, Tk * sizeof(int));
@@ -1289,7 +1313,6 @@ dg_status dg_init_weights(const dg_config* cfg, uint64_t seed, void* stream, dg_
   cudaMemsetAsync(m->st, 0, sizeof(DevState), s);
   cudaMemsetAsync(m->prev_amax, 0xFF, (size_t)m->T_cap * sizeof(int), s);
   cudaMemsetAsync(m->sc, 0, (size_t)m->T_cap * d * es, s);
-  if (m->sk.seg_flag) cudaMemsetAsync(m->sk.seg_flag, 0, (size_t)kSMs * sizeof(int), s);
   if (m->touched_acc) cudaMemsetAsync(m->touched_acc, 0, (size_t)m->L * sizeof(unsigned long long), s);
   if (m->fp8 && st == DG_OK) {
     // scratch for one expert tensor in bf16 before quantisation (freed below)
@@ -1324,13 +1347,13 @@ size_t dg_kv_bytes(const dg_model* m, int32_t B, int32_t P) {
 int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   if (!m) return 0;
   (void)B; (void)P;
-  // per layer: qkv gemm (bf16: with the RoPE / cache scatter; fp32: + qkv
-  // post), attention, attention combine, o gemm, residual+norm, router (bf16:
-  // one kernel; fp32: gemm + top-k), permute, gather, gate/up gemm, swiglu
-  // (fp32 and FP8 experts; bf16 fuses it into the stream-K gate|up GEMM),
-  // down gemm, combine+norm; then embed+norm, lm head, sampler, commit,
-  // 4 self-cond.
-  const int per_layer = (m->bf ? (m->fp8 ? 12 : 11) : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
+  // per layer: qkv gemm (with the RoPE / cache scatter when fused; else +
+  // qkv post), attention (+ combine unless the splits merge in the kernel),
+  // o gemm, residual+norm, router (bf16: one kernel; fp32: gemm + top-k),
+  // permute, gather, gate/up gemm, swiglu, down gemm, combine+norm; then
+  // embed+norm, lm head, sampler, commit, 4 self-cond.  The attention merge
+  // is decided per shape, so this is the count with the combine kernel.
+  const int per_layer = (m->bf ? 12 : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
   return per_layer * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          (m->c.sample_topk > 0 ? 3 : 4) /*self-conditioning*/;
 }

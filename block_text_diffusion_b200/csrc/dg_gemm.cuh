@@ -401,6 +401,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps
 // ---------------------------------------------------------------------------
 constexpr int kWorkSmem = 512;   // work items staged in shared memory (more are read from global)
 
+
 // Barrier among the four epilogue warps (threads 64..191) of the persistent kernel.
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
@@ -443,11 +444,12 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
   // the split factor and the work list are written by the permute kernel
   pdl_wait();
   if (p.k_splits_dev) p.k_splits = max(1, min(*p.k_splits_dev, p.kb_total));
+  constexpr int tile_rows = kTileRows, nbuf = kNBuf, acc_stride = MT, a_bytes = C::kABytes;
   const int n_items = p.work ? *p.work_count : items_dense;
   // ring geometry from the largest B tile any work item loads
   int rows_max = BN;
   if (p.max_rows_dev) rows_max = min(BN, max(kBoxRowsB, *p.max_rows_dev));
-  const int stage_bytes = C::kABytes + ((rows_max + kBoxRowsB - 1) / kBoxRowsB) * kBoxRowsB * 128;
+  const int stage_bytes = a_bytes + ((rows_max + kBoxRowsB - 1) / kBoxRowsB) * kBoxRowsB * 128;
   const int n_stages = min(kMaxStages, (STAGES * C::kStage) / stage_bytes);
   const int total = p.m_tiles * p.k_splits * n_items;
   // work items are read by all three roles once per tile: stage them on chip
@@ -490,10 +492,10 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
           const uint32_t ph = (it / n_stages) & 1;
           if (it >= n_stages && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) { ok = false; break; }
           uint8_t* a_s = smem + s * stage_bytes;
-          uint8_t* b_s = a_s + C::kABytes;
+          uint8_t* b_s = a_s + a_bytes;
           mbar_expect_tx(&full_bar[s], tx);
           for (int h = 0; h < nh; ++h)
-            tma_load_2d(a_s + h * 16384, &tmA, kb * 64, t.a_row0 + t.m_tile * kTileRows + h * 128, &full_bar[s]);
+            tma_load_2d(a_s + h * 16384, &tmA, kb * 64, t.a_row0 + t.m_tile * tile_rows + h * 128, &full_bar[s]);
           tma_load_b_rows(b_s, &tmB, kb * 64, t.b_row0, n_boxes * kBoxRowsB, &full_bar[s]);
         }
       }
@@ -514,22 +516,22 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         split_range(p, split, kb0, kb1);
         const int n_mma = min(BN, (n_valid + 15) & ~15);
         const uint32_t idesc = idesc_bf16(128, n_mma);
-        const int buf = local % kNBuf;
-        // wait until the epilogue drained this buffer (kNBuf tiles ago)
-        if (local >= kNBuf &&
-            !mbar_wait(&acc_empty[buf], ((local / kNBuf) & 1) ^ 1, p.err, DGDEV_TIMEOUT_MMA)) {
+        const int buf = local % nbuf;
+        // wait until the epilogue drained this buffer (nbuf tiles ago)
+        if (local >= nbuf &&
+            !mbar_wait(&acc_empty[buf], ((local / nbuf) & 1) ^ 1, p.err, DGDEV_TIMEOUT_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + buf * MT * kAccCols;
+        const uint32_t d_tmem = tmem + buf * acc_stride * kAccCols;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % n_stages;
           const uint32_t ph = (it / n_stages) & 1;
           if (!mbar_wait(&full_bar[s], ph, p.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
-          const uint64_t bd = sdesc_sw128(a_addr + C::kABytes);
+          const uint64_t bd = sdesc_sw128(a_addr + a_bytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
@@ -560,9 +562,9 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
       split_range(p, split, kb0, kb1);
       const int n_mma = min(BN, (n_valid + 15) & ~15);
       const int nh = halves(m_t);
-      const int buf = local % kNBuf;
+      const int buf = local % nbuf;
       const bool ok =
-          __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local / kNBuf) & 1, p.err, DGDEV_TIMEOUT_EPI));
+          __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (local / nbuf) & 1, p.err, DGDEV_TIMEOUT_EPI));
       tc_fence_after();
       if (p.act && p.k_splits == 1) {
         // fused SwiGLU: in each 128-row half, rows 0..63 are gate rows of SwiGLU
@@ -575,8 +577,8 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const bool ok_all = s_epi_fail == 0;
         bf16* act = reinterpret_cast<bf16*>(p.act);
         for (int h = 0; h < nh; ++h) {
-          const int f = (m_t * MT + h) * 64 + (quad & 1) * 32 + lane;
-          const uint32_t tbase = tmem + (buf * MT + h) * kAccCols + ((uint32_t)(quad * 32) << 16);
+          const int f = (m_t * (tile_rows / 128) + h) * 64 + (quad & 1) * 32 + lane;
+          const uint32_t tbase = tmem + (buf * acc_stride + h) * kAccCols + ((uint32_t)(quad * 32) << 16);
           for (int c0 = 0; c0 < n_mma; c0 += 16) {
             uint32_t v[16];
             if (ok_all && kb1 > kb0) {
@@ -611,11 +613,11 @@ k_gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_const
         continue;
       }
       for (int h = 0; h < nh; ++h) {
-        const int m0 = m_t * kTileRows + h * 128;
+        const int m0 = m_t * tile_rows + h * 128;
         const bool m_ok = (m0 + row) < p.M;
         float* outp = p.out + (long long)split * p.split_stride + (long long)out_row0 * p.ldo + m0 + row;
         if (ok && kb1 > kb0) {
-          epilogue_store(tmem + (buf * MT + h) * kAccCols + ((uint32_t)(quad * 32) << 16), n_mma, n_valid, m_ok,
+          epilogue_store(tmem + (buf * acc_stride + h) * kAccCols + ((uint32_t)(quad * 32) << 16), n_mma, n_valid, m_ok,
                          outp, p.ldo, p.alpha);
         } else if (ok && m_ok) {
           for (int n = 0; n < n_valid; ++n) outp[(long long)n * p.ldo] = 0.0f;
@@ -681,303 +683,4 @@ k_gemm_f32(const float* __restrict__ A, long long lda, const float* __restrict__
       if (n < t.n_valid) outp[(long long)(t.out_row0 + n) * p.ldo + m] = acc[i][j] * p.alpha;
     }
   }
-}
-
-// ---------------------------------------------------------------------------
-// Stream-K grouped GEMM (the expert GEMMs).  The iterations (tile, k block)
-// of the whole launch -- I = m_tiles x work items x k blocks, tiles of
-// 128 MT rows -- are divided into gridDim.x equal contiguous runs, one per
-// persistent CTA (one per SM), so every SM streams weights whatever the
-// number of experts a layer touches, without split-K slabs for the whole
-// output.
-//
-// A run is a sequence of segments (tile, k range).  A tile whose k range
-// lies inside one run is finished by that CTA's epilogue (the fp32 store, or
-// the SwiGLU activation when `act` is set).  A tile cut between runs is
-// finished by the CTA holding its first k range: that segment is the last of
-// its run, while the later ranges are the first segments of the following
-// runs, so their CTAs publish them early (fp32 partial in their slot of
-// `seg_ws`, then a release flag) and the owner adds them in k order to its
-// own accumulator -- a fixed order, so results are deterministic.  Waits
-// point only from a CTA to later CTAs' first segments, which depend on
-// nothing: no cycle.  Every CTA of the grid must be resident at once
-// (gridDim.x <= SMs, one CTA per SM by shared memory).  The owner clears the
-// flags it consumed, so they are zero again for the next launch.
-//
-// MT = 2: 256-row tiles (two 128-row accumulators share every B tile, half
-// the activation traffic of 128-row tiles), accumulators single-buffered;
-// MT = 1: 128-row tiles, accumulators double-buffered.  The epilogue drains
-// 32 columns per TMEM wait.
-// Warps: 0 = TMA producer, 1 = MMA issuer, 2..5 = epilogue.
-// ---------------------------------------------------------------------------
-struct StreamK {
-  float* seg_ws;   // [gridDim.x][MT][BN][128] fp32 partial accumulators (column-major per 128-row half)
-  int* seg_flag;   // [gridDim.x]; 0 outside a launch, 1 = slot published
-};
-
-__device__ __forceinline__ long long sk_run_start(long long g, long long I, long long G) { return g * I / G; }
-
-template <int BN, int STAGES, int MT>
-__global__ void __launch_bounds__(192, 1)
-k_gemm_tc_streamk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB, GemmArgs p_in,
-                  StreamK sk) {
-  using C = GemmTcCfg<BN, STAGES, MT>;
-  constexpr int kAccCols = C::kTmemCols;
-  constexpr int kNBuf = MT == 1 ? 2 : 1;
-  constexpr int kAllocCols = kNBuf * MT * kAccCols;
-  static_assert(kAllocCols <= 512, "tensor memory holds 512 columns");
-  constexpr int kTileRows = 128 * MT;
-  constexpr int kMaxStages = 3 * STAGES;
-  constexpr long long kSlot = (long long)MT * BN * 128;   // floats per partial slot
-  pdl_launch();
-  GemmArgs p = p_in;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages], acc_full[2], acc_empty[2];
-  __shared__ uint32_t tmem_base;
-  __shared__ int4 s_work[kWorkSmem];
-  __shared__ float s_xfer[64 * 33];   // SwiGLU: up values of one 32-column chunk
-  __shared__ int s_fail;              // an epilogue wait ran out
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kMaxStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
-    fence_mbar_init();
-    prefetch_tmap(&tmA);
-    for (int i = 0; i < 4; ++i) prefetch_tmap(&tmB.m[i]);
-    s_fail = 0;
-  }
-  if (warp == 0) tmem_alloc(&tmem_base, kAllocCols);
-  // the work list is written by the permute kernel
-  pdl_wait();
-  const int n_items = *p.work_count;
-  int rows_max = BN;
-  if (p.max_rows_dev) rows_max = min(BN, max(kBoxRowsB, *p.max_rows_dev));
-  const int stage_bytes = C::kABytes + ((rows_max + kBoxRowsB - 1) / kBoxRowsB) * kBoxRowsB * 128;
-  const int n_stages = min(kMaxStages, (STAGES * C::kStage) / stage_bytes);
-  const bool work_smem = n_items <= kWorkSmem;
-  if (work_smem)
-    for (int i = threadIdx.x; i < n_items; i += blockDim.x) s_work[i] = p.work[i];
-  const int4* work = work_smem ? s_work : p.work;
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base;
-
-  const long long kb = p.kb_total;
-  const long long I = (long long)p.m_tiles * n_items * kb;
-  const long long G = gridDim.x, g = blockIdx.x;
-  const long long lo = sk_run_start(g, I, G), hi = sk_run_start(g + 1, I, G);
-  // segment at iteration x: tile t = x / kb, k range [x - t kb, min(kb, hi - t kb))
-  auto segment = [&](long long x, long long& t, int& k0, int& k1) {
-    t = x / kb;
-    k0 = (int)(x - t * kb);
-    k1 = (int)min(kb, hi - t * kb);
-  };
-  // 128-row halves of tile m_t that hold rows below M
-  auto halves = [&](int m_t) { return MT == 1 ? 1 : min(MT, (p.M - m_t * kTileRows + 127) / 128); };
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (long long x = lo; x < hi && ok;) {
-        long long t;
-        int k0, k1;
-        segment(x, t, k0, k1);
-        const int m_tile = (int)(t % p.m_tiles);
-        const int4 w = work[t / p.m_tiles];
-        const int nh = halves(m_tile);
-        const int n_boxes = (min(BN, (w.z + 15) & ~15) + kBoxRowsB - 1) / kBoxRowsB;
-        const uint32_t tx = nh * 16384 + n_boxes * kBoxRowsB * 128;
-        for (int k = k0; k < k1; ++k, ++it) {
-          const int s = it % n_stages;
-          const uint32_t ph = (it / n_stages) & 1;
-          if (it >= n_stages && !mbar_wait(&empty_bar[s], ph ^ 1, p.err, DGDEV_TIMEOUT_TMA)) { ok = false; break; }
-          uint8_t* a_s = smem + s * stage_bytes;
-          mbar_expect_tx(&full_bar[s], tx);
-          for (int h = 0; h < nh; ++h)
-            tma_load_2d(a_s + h * 16384, &tmA, k * 64, w.x * p.a_group_rows + m_tile * kTileRows + h * 128,
-                        &full_bar[s]);
-          tma_load_b_rows(a_s + C::kABytes, &tmB, k * 64, w.y, n_boxes * kBoxRowsB, &full_bar[s]);
-        }
-        x = t * kb + k1;
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      int it = 0, local = 0;
-      bool ok = true;
-      for (long long x = lo; x < hi && ok; ++local) {
-        long long t;
-        int k0, k1;
-        segment(x, t, k0, k1);
-        const int nh = halves((int)(t % p.m_tiles));
-        const int n_mma = min(BN, (work[t / p.m_tiles].z + 15) & ~15);
-        const uint32_t idesc = idesc_bf16(128, n_mma);
-        const int buf = local % kNBuf;
-        if (local >= kNBuf &&
-            !mbar_wait(&acc_empty[buf], ((local / kNBuf) & 1) ^ 1, p.err, DGDEV_TIMEOUT_MMA)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + buf * MT * kAccCols;
-        for (int k = k0; k < k1; ++k, ++it) {
-          const int s = it % n_stages;
-          const uint32_t ph = (it / n_stages) & 1;
-          if (!mbar_wait(&full_bar[s], ph, p.err, DGDEV_TIMEOUT_MMA)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
-          const uint64_t bd = sdesc_sw128(a_addr + C::kABytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-            for (int h = 0; h < MT; ++h)
-              if (h < nh)
-                tc_mma_bf16(d_tmem + h * kAccCols, sdesc_sw128(a_addr + h * 16384) + 2 * kk, bd + 2 * kk, idesc,
-                            (k > k0 || kk > 0) ? 1u : 0u);
-          tc_commit(&empty_bar[s]);
-        }
-        tc_commit(&acc_full[buf]);
-        x = t * kb + k1;
-      }
-    }
-    __syncwarp();
-  } else {
-    // epilogue warps 2..5: warp w drains TMEM lanes 32 (w % 4) ..  Failure
-    // decisions are read between two barriers so that all four warps take
-    // the same branches (s_fail only ever goes from 0 to 1).
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    int local = 0;
-    for (long long x = lo; x < hi; ++local) {
-      long long t;
-      int k0, k1;
-      segment(x, t, k0, k1);
-      const int m_tile = (int)(t % p.m_tiles);
-      const int4 w = work[t / p.m_tiles];
-      const int n_valid = w.z, out_row0 = w.w;
-      const int n_mma = min(BN, (n_valid + 15) & ~15);
-      const int nh = halves(m_tile);
-      const int buf = local % kNBuf;
-      if (lane == 0 && !mbar_wait(&acc_full[buf], (local / kNBuf) & 1, p.err, DGDEV_TIMEOUT_EPI)) s_fail = 1;
-      epi_sync();
-      bool ok = s_fail == 0;
-      epi_sync();
-      tc_fence_after();
-      const uint32_t tbase = tmem + buf * MT * kAccCols + ((uint32_t)(quad * 32) << 16);
-      if (k0 > 0) {
-        // a later k range of a cut tile (this run's first segment): publish
-        float* slot = sk.seg_ws + g * kSlot;
-        for (int h = 0; h < nh; ++h)
-          for (int c0 = 0; c0 < n_mma; c0 += 32) {
-            uint32_t v[2][16];
-            if (ok) {
-              tmem_ld16_nw(tbase + h * kAccCols + c0, v[0]);
-              if (c0 + 16 < n_mma) tmem_ld16_nw(tbase + h * kAccCols + c0 + 16, v[1]);
-              tmem_wait_ld();
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c0 + j < n_mma)
-                __stcg(slot + ((long long)h * BN + c0 + j) * 128 + row, ok ? __uint_as_float(v[j >> 4][j & 15]) : 0.0f);
-          }
-        __threadfence();
-        epi_sync();
-        if (threadIdx.x == 64 && ok)
-          asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(sk.seg_flag + g), "r"(1) : "memory");
-      } else {
-        // this tile starts here: gather the later k ranges (runs g+1 .. g_last)
-        long long g_last = g;
-        if (k1 < kb) {
-          const long long t_end = (t + 1) * kb;
-          while (g_last + 1 < G && sk_run_start(g_last + 1, I, G) < t_end) ++g_last;
-          if (threadIdx.x == 64 && ok) {
-            for (long long q = g + 1; q <= g_last; ++q) {
-              if (sk_run_start(q + 1, I, G) == sk_run_start(q, I, G)) continue;   // an empty run
-              const uint64_t t0 = global_ns();
-              bool got = false;
-              for (uint32_t it = 0;; ++it) {
-                int f;
-                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(sk.seg_flag + q) : "memory");
-                if (f == 1) { got = true; break; }
-                if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) break;
-              }
-              if (!got) {
-                dev_error(p.err, DGDEV_TIMEOUT_EPI);
-                s_fail = 1;
-                break;
-              }
-            }
-          }
-          epi_sync();
-          ok = s_fail == 0;
-          epi_sync();
-        }
-        bf16* act = reinterpret_cast<bf16*>(p.act);
-        for (int h = 0; h < nh; ++h) {
-          const int m0 = m_tile * kTileRows + h * 128;
-          const bool m_ok = (m0 + row) < p.M;
-          for (int c0 = 0; c0 < n_mma; c0 += 32) {
-            uint32_t v[2][16];
-            if (ok) {
-              tmem_ld16_nw(tbase + h * kAccCols + c0, v[0]);
-              if (c0 + 16 < n_mma) tmem_ld16_nw(tbase + h * kAccCols + c0 + 16, v[1]);
-              tmem_wait_ld();
-            }
-            float acc[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = (ok && c0 + j < n_mma) ? __uint_as_float(v[j >> 4][j & 15]) : 0.0f;
-            if (ok)
-              for (long long q = g + 1; q <= g_last; ++q) {
-                if (sk_run_start(q + 1, I, G) == sk_run_start(q, I, G)) continue;
-                const float* slot = sk.seg_ws + q * kSlot + ((long long)h * BN + c0) * 128 + row;
-                float part[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) part[j] = (c0 + j < n_mma) ? __ldcg(slot + (long long)j * 128) : 0.0f;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) acc[j] += part[j];
-              }
-            if (act) {
-              // SwiGLU: rows 0..63 of each 128-row half are gate rows of
-              // outputs f = 64 (2 m_tile + h) .., rows 64..127 the matching up rows
-              if (quad >= 2) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) s_xfer[((quad - 2) * 32 + lane) * 33 + j] = acc[j];
-              }
-              epi_sync();
-              if (quad < 2 && ok) {
-                const int f = (m_tile * MT + h) * 64 + quad * 32 + lane;
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (c0 + j < n_valid) {
-                    const float gv = acc[j];
-                    const float u = s_xfer[(quad * 32 + lane) * 33 + j];
-                    act[(long long)(out_row0 + c0 + j) * p.act_ld + f] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * u);
-                  }
-              }
-              epi_sync();
-            } else if (m_ok && ok) {
-              float* outp = p.out + (long long)out_row0 * p.ldo + m0 + row;
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (c0 + j < n_valid) outp[(long long)(c0 + j) * p.ldo] = acc[j] * p.alpha;
-            }
-          }
-        }
-        // the consumed flags are cleared for the next launch
-        if (threadIdx.x == 64)
-          for (long long q = g + 1; q <= g_last; ++q) sk.seg_flag[q] = 0;
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
-      x = t * kb + k1;
-      if (!ok) break;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kAllocCols);
 }

@@ -220,8 +220,13 @@ __global__ void k_residual_norm(T* __restrict__ h, T* __restrict__ x, const floa
 // order);  x[t] = RMSNorm(h[t]).
 // y holds `splits` partial slabs (split_stride apart; count read from the
 // device) that are summed before weighting.  Vectorised by 4 (d % 64 == 0).
+// Rows of up to kCombineG float4 per thread with up to kCombineK slots keep
+// every value in registers, with all loads of the row issued before the
+// first use (one round trip instead of one per chunk, and no re-read of h
+// for the norm); the arithmetic and its order are those of the general loop.
+constexpr int kCombineK = 8, kCombineG = 3;
 template <typename T>
-__global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ y,
+__global__ void __launch_bounds__(256, 2) k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const float* __restrict__ y,
                                    const int* __restrict__ inv, const float* __restrict__ gate, int k, int d,
                                    float eps, const int* __restrict__ splits_dev, long long split_stride) {
   pdl_enter();
@@ -236,6 +241,80 @@ __global__ void k_moe_combine_norm(T* __restrict__ h, T* __restrict__ x, const f
   }
   __syncthreads();
   T* hr = h + t * d;
+  if (k <= kCombineK && d <= kCombineG * 4 * (int)blockDim.x) {
+    // slots in two groups of kCombineK / 2: every load of a group is issued
+    // before its first use, and the weighted sums run in slot order
+    constexpr int kHalf = kCombineK / 2;
+    float4 hv[kCombineG];
+    float acc[kCombineG][4];
+#pragma unroll
+    for (int g = 0; g < kCombineG; ++g) {
+      const int i = (threadIdx.x + g * blockDim.x) * 4;
+      hv[g] = i < d ? load4<T>(hr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.0f;
+    }
+#pragma unroll
+    for (int j0 = 0; j0 < kCombineK; j0 += kHalf) {
+      if (j0 >= k) break;
+      float4 v[kCombineG][kHalf];
+#pragma unroll
+      for (int g = 0; g < kCombineG; ++g) {
+        const int i = (threadIdx.x + g * blockDim.x) * 4;
+        if (i < d) {
+#pragma unroll
+          for (int jj = 0; jj < kHalf; ++jj)
+            if (j0 + jj < k) v[g][jj] = *reinterpret_cast<const float4*>(y + rows[j0 + jj] + i);
+        }
+      }
+      for (int s = 1; s < ns; ++s) {
+#pragma unroll
+        for (int g = 0; g < kCombineG; ++g) {
+          const int i = (threadIdx.x + g * blockDim.x) * 4;
+          if (i < d) {
+#pragma unroll
+            for (int jj = 0; jj < kHalf; ++jj)
+              if (j0 + jj < k) {
+                const float4 v2 = *reinterpret_cast<const float4*>(y + rows[j0 + jj] + i + s * split_stride);
+                v[g][jj].x += v2.x; v[g][jj].y += v2.y; v[g][jj].z += v2.z; v[g][jj].w += v2.w;
+              }
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < kCombineG; ++g)
+#pragma unroll
+        for (int jj = 0; jj < kHalf; ++jj)
+          if (j0 + jj < k) {
+            const float gj = gw[j0 + jj];
+            acc[g][0] = fmaf(gj, v[g][jj].x, acc[g][0]);
+            acc[g][1] = fmaf(gj, v[g][jj].y, acc[g][1]);
+            acc[g][2] = fmaf(gj, v[g][jj].z, acc[g][2]);
+            acc[g][3] = fmaf(gj, v[g][jj].w, acc[g][3]);
+          }
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int g = 0; g < kCombineG; ++g) {
+      const int i = (threadIdx.x + g * blockDim.x) * 4;
+      if (i < d) {
+        hv[g] = make_float4(to_f(from_f<T>(hv[g].x + acc[g][0])), to_f(from_f<T>(hv[g].y + acc[g][1])),
+                            to_f(from_f<T>(hv[g].z + acc[g][2])), to_f(from_f<T>(hv[g].w + acc[g][3])));
+        store4<T>(hr + i, hv[g].x, hv[g].y, hv[g].z, hv[g].w);
+        ss = fmaf(hv[g].x, hv[g].x, ss);
+        ss = fmaf(hv[g].y, hv[g].y, ss);
+        ss = fmaf(hv[g].z, hv[g].z, ss);
+        ss = fmaf(hv[g].w, hv[g].w, ss);
+      }
+    }
+    const float tot = block_sum(ss, red);
+    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)d), eps)));
+#pragma unroll
+    for (int g = 0; g < kCombineG; ++g) {
+      const int i = (threadIdx.x + g * blockDim.x) * 4;
+      if (i < d) store4<T>(x + t * d + i, hv[g].x * r, hv[g].y * r, hv[g].z * r, hv[g].w * r);
+    }
+    return;
+  }
   float ss = 0.0f;
   for (int i = threadIdx.x * 4; i < d; i += blockDim.x * 4) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -453,7 +532,7 @@ __global__ void k_router_bias_f32(float* bias, int E, float s) {
 struct SplitPlan {
   int mt[2], kb[2], cap[2];
   int fused0;   // the gate|up GEMM writes the SwiGLU output itself when it runs unsplit
-  int* out;
+  int* out;     // [0] gate|up split, [1] down split, [2] rows of the largest item
 };
 
 // Exclusive prefix sum of one int per thread over the block (blockDim a
@@ -484,15 +563,35 @@ __device__ __forceinline__ int block_scan_excl(int v, int* wsum, int* total) {
   return base + x - v;
 }
 
-__global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int bn, int* __restrict__ perm,
-                          int* __restrict__ inv, int4* __restrict__ work, int* __restrict__ work_count,
-                          int* __restrict__ counts_out, SplitPlan plan, unsigned long long* touched_acc, int* err) {
+struct PermuteArgs {
+  const int* ids;          // [n_pairs] expert of each (token, slot)
+  int n_pairs, E, bn;
+  int* perm;               // [n_pairs] pair at each expert-ordered position
+  int* inv;                // [n_pairs] position of each pair
+  int4* work;              // work items (expert, first row, rows, first row)
+  int* work_count;
+  int* counts_out;         // [E] rows per expert, or null
+  SplitPlan plan;
+  unsigned long long* touched_acc;   // running total of distinct experts, or null
+  int* err;
+};
+
+// The permute by one CTA (any multiple of 32 threads); psm holds
+// (warps x E + E + 1) ints.  ids are read through L2: they may have been
+// written by other CTAs of the same kernel.
+__device__ void permute_body(const PermuteArgs& a, int* psm) {
+  const int* __restrict__ ids = a.ids;
+  const int n_pairs = a.n_pairs, E = a.E, bn = a.bn;
+  int* __restrict__ perm = a.perm;
+  int* __restrict__ inv = a.inv;
+  int4* __restrict__ work = a.work;
+  int* __restrict__ counts_out = a.counts_out;
+  SplitPlan plan = a.plan;
+  int* err = a.err;
   // Warp w owns the contiguous pair range [w*chunk, (w+1)*chunk).  A pair's
   // position is offs[e] (pairs of lower experts) + pairs of expert e in
   // earlier warps + pairs of e earlier in this warp's range, which keeps the
   // (token, slot) order within each expert.
-  pdl_enter();
-  extern __shared__ int psm[];
   const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* hist = psm;                  // [nwarps][E]
   int* offs = psm + nwarps * E;     // [E + 1]
@@ -504,7 +603,7 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
   int* my = hist + warp * E;
   for (int p0 = p_begin; p0 < p_end; p0 += 32) {
     const int p = p0 + lane;
-    int e = p < p_end ? ids[p] : -1;
+    int e = p < p_end ? __ldcg(ids + p) : -1;
     if (e >= E || (p < p_end && e < 0)) { dev_error(err, DGDEV_BAD_INDEX); e = -1; }
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && (same & lt_mask) == 0) my[e] += __popc(same);
@@ -549,9 +648,9 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
   if (threadIdx.x == 0) {
     const int nw = carry_items;
     offs[E] = carry_rows;
-    *work_count = nw;
+    *a.work_count = nw;
     // running total of distinct experts this layer streamed (measurement)
-    if (touched_acc) *touched_acc += (unsigned long long)s_touched;
+    if (a.touched_acc) *a.touched_acc += (unsigned long long)s_touched;
     if (plan.out) {
       // Split-K factor per GEMM: the persistent kernel runs ceil(tiles / SMs)
       // waves of tiles that each take 1/s of a full-K tile, and every split
@@ -579,7 +678,7 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
   __syncthreads();
   for (int p0 = p_begin; p0 < p_end; p0 += 32) {
     const int p = p0 + lane;
-    int e = p < p_end ? ids[p] : -1;
+    int e = p < p_end ? __ldcg(ids + p) : -1;
     if (e >= E) e = -1;
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
@@ -591,6 +690,12 @@ __global__ void k_permute(const int* __restrict__ ids, int n_pairs, int E, int b
     if (e >= 0 && (same & lt_mask) == 0) my[e] += __popc(same);
     __syncwarp();
   }
+}
+
+__global__ void k_permute(PermuteArgs a) {
+  pdl_enter();
+  extern __shared__ int psm[];
+  permute_body(a, psm);
 }
 
 // Threads of the permute kernel: whole warps, with the per-warp histograms
@@ -786,6 +891,7 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
 
   // pass 2
   long long sq = 0, uq = 0;
+  double sd = 0.0, ud = 0.0;
   for (int i = threadIdx.x; i < n4; i += blockDim.x) {
     const float4 l = l4[i];
     const float lv[4] = {l.x, l.y, l.z, l.w};
@@ -793,10 +899,12 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
     for (int j = 0; j < 4; ++j) {
       const float dlt = __fsub_rn(lv[j], m);
       const float e = dg_expf(dlt);
-      sq += q40_trunc(e);
-      uq += q40_trunc(__fmul_rn(e, dlt));
+      q40_add(e, sq, sd);
+      q40_add(__fmul_rn(e, dlt), uq, ud);
     }
   }
+  sq = q40_total(sq, sd);
+  uq = q40_total(uq, ud);
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
     sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -1029,6 +1137,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
 
   // pass 2: S, U of the full row (as in k_sampler)
   long long sq = 0, uq = 0;
+  double sd = 0.0, ud = 0.0;
   for (int i = threadIdx.x; i < n4; i += blockDim.x) {
     const float4 l = l4[i];
     const float lv[4] = {l.x, l.y, l.z, l.w};
@@ -1036,10 +1145,12 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
     for (int j = 0; j < 4; ++j) {
       const float dlt = __fsub_rn(lv[j], m);
       const float e = dg_expf(dlt);
-      sq += q40_trunc(e);
-      uq += q40_trunc(__fmul_rn(e, dlt));
+      q40_add(e, sq, sd);
+      q40_add(__fmul_rn(e, dlt), uq, ud);
     }
   }
+  sq = q40_total(sq, sd);
+  uq = q40_total(uq, ud);
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
     sq += __shfl_xor_sync(0xffffffffu, sq, o);

@@ -106,12 +106,8 @@ dg_status dg_set_routing_bias(dg_model* m, const float* bias, int32_t n_tok);
  * (persistent, bf16, M % 128 == 0) applies SwiGLU in the epilogue: A rows
  * interleave gate / up in blocks of 64 and out receives bf16 [rows][M/2],
  * out[r][f] = round(silu(g) u) with g, u the rows 128 (f/64) + f%64 (+64);
- * bit 3 (persistent, bn 256) uses 256-row tiles (two accumulators per CTA);
- * bit 4 (bf16, bn 256) runs the stream-K kernel the expert GEMMs use (one
- * CTA per SM, equal runs of (tile, k block) iterations, cut tiles finished
- * in k order by the CTA holding their first k range; with bit 2 it writes the
- * SwiGLU activation) and returns DG_ERR_STATE if a partial-slot flag is left
- * set afterwards.  Allocates. */
+ * bit 3 (persistent, bn 256) uses 256-row tiles (two accumulators per CTA).
+ * Allocates. */
 dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* counts, int32_t groups, int32_t M,
                                int32_t K, int32_t bf16, int32_t bn, int32_t flags, float* out, void* stream);
 
@@ -122,6 +118,12 @@ dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* coun
  * queries per canvas, G query heads per KV head, n_keys keys, rows = query
  * rows of the launch and part_rows_cap = rows the partial-output buffer
  * holds per split sum (binding only when the splits merge through it). */
+/* Thread-block clusters of the bf16 attention kernel that the device can
+ * hold at once, per cluster size (the capacity the split-KV plan is given):
+ * out int32[9], out[c] for c = 1..8, out[0] = 0; 0 where the device refuses
+ * the query.  Host memory; needs a device; does not synchronise. */
+dg_status dg_test_attn_capacity(int32_t* out);
+
 dg_status dg_test_attn_plan(int64_t n_q, int32_t G, int32_t Hkv, int32_t n_canvas, int32_t n_keys, int64_t rows,
                             int64_t part_rows_cap, int32_t* out);
 
@@ -210,6 +212,20 @@ dg_status dg_debug_trace(dg_model* model, float* h_trace, int32_t* ids_trace);
  * DG_ERR_INVALID_ARG for a bad layer or shape, a device error code otherwise. */
 dg_status dg_test_layer(dg_model* model, void* kv, int32_t B, int32_t P, int32_t layer, const void* h_in,
                         float* h_trace, int32_t* ids, void* stream);
+
+/* The MoE half of one layer of the canvas pass from a given state
+ * (DiffusionGemma technical-report explainer, section 二: the top-k MoE FFN
+ * after the attention residual).  h_attn: device [B*256][d] in the model
+ * dtype, the residual stream after the layer's attention; the call
+ * normalises it, routes each token to its top-k experts (a router bias set
+ * by dg_set_routing_bias applies), runs the experts and adds the gated sum
+ * to the stream.  Outputs (device, caller-owned): h_trace fp32 [3][B*256][d]
+ * whose rows [1] = h after the MoE and [2] = RMSNorm of it (rows [0] are not
+ * written); ids int32 [B*256][top_k] = the routing (slot order).
+ * Synchronises; DG_ERR_INVALID_ARG for a bad layer or B, a device error code
+ * otherwise. */
+dg_status dg_test_moe(dg_model* model, int32_t B, int32_t layer, const void* h_attn, float* h_trace,
+                      int32_t* ids, void* stream);
 
 /* Kernel launches recorded in one captured block-loop round (graph body). */
 int32_t dg_launches_per_round(const dg_model* model);

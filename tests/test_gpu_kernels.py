@@ -310,7 +310,7 @@ def test_gemm_f32():
     (1024, 256, [0, 9, 64, 65, 1], 64, False),
     (1408, 2816, [17, 3, 0, 31, 12, 1, 9, 20], 256, True),
 ])
-@pytest.mark.parametrize("persistent", [False, True, "sized_ring", "m256", "streamk", "streamk256"])
+@pytest.mark.parametrize("persistent", [False, True, "sized_ring", "m256"])
 def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     g = np.random.default_rng(sum(counts) + M)
     G = len(counts)
@@ -326,15 +326,9 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
     # item (more stages in flight), as the expert GEMMs run in the step
     # "m256": 256-row tiles (two accumulators), as the expert GEMMs run, with the
     # ring sized from the largest item
-    # "streamk": every SM takes an equal run of (tile, k block) iterations; a
-    # tile cut between runs is summed in k order by the CTA holding its start
-    # ("streamk256": the same over 256-row weight tiles)
-    sk = persistent in ("streamk", "streamk256")
-    if sk and not (bf and bn == 256):
-        pytest.skip("stream-K runs bf16 with 256-row item tiles")
     dg.test_grouped_gemm(At, Bt, counts, G, M, out, bn=bn, persistent=bool(persistent) and bf,
                          sized_ring=persistent in ("sized_ring", "m256") and bf,
-                         m256=persistent in ("m256", "streamk256") and bf and bn == 256, streamk=sk)
+                         m256=persistent == "m256" and bf and bn == 256)
     got = host(out).astype(np.float64)
     r0 = 0
     for e, c in enumerate(counts):
@@ -347,7 +341,7 @@ def test_grouped_gemm(M, K, counts, bn, bf, persistent):
 
 @pytest.mark.parametrize("M,K,counts", [(1408, 2816, [17, 3, 0, 200, 12, 1, 256, 20]), (2048, 1024, [64, 65, 0, 9]),
                                          (1408, 2816, [300, 1, 0, 5]), (1408, 2816, [16] * 120 + [40])])
-@pytest.mark.parametrize("m256", [False, True, "streamk", "streamk256"])
+@pytest.mark.parametrize("m256", [False, True])
 def test_grouped_gemm_fused_swiglu(M, K, counts, m256):
     # the unsplit gate|up GEMM writes round(silu(g) u) itself; A rows interleave
     # gate / up in blocks of 64
@@ -357,8 +351,7 @@ def test_grouped_gemm_fused_swiglu(M, K, counts, m256):
     B = I._bf16_grid(g.standard_normal((rows, K)).astype(F32))
     out = torch.zeros((rows, M), dtype=torch.float32, device="cuda")
     dg.test_grouped_gemm(bf16_tensor(A), bf16_tensor(B), counts, G, M, out, bn=256, persistent=True,
-                         sized_ring=True, swiglu=True, m256=m256 in (True, "streamk256"),
-                         streamk=m256 in ("streamk", "streamk256"))
+                         sized_ring=True, swiglu=True, m256=m256)
     act = out.view(torch.bfloat16).reshape(-1)[:rows * ff].reshape(rows, ff)
     got = act.float().cpu().numpy().astype(np.float64)
     f = np.arange(ff)
