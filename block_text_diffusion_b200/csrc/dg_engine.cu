@@ -129,10 +129,12 @@ struct LayerW {
 // (dense_bn, dense_splits, router_bn, router_splits, qkv_fused; 0 keeps the
 // default; attn_merge = 1 always merges attention key splits with the
 // combine kernel, 2 always inside the kernel when the splits fit a cluster;
-// down_m256 = 1 runs the down GEMM on 256-row tiles).
+// down_m256 = 1 runs the down GEMM on 256-row tiles; gu_m128 = 1 runs the
+// gate|up GEMM on 128-row tiles; gu_cap / dn_cap > 0 cap the split-K factor
+// the device may pick for the gate|up / down GEMM).
 struct Tune {
   int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0, qkv_fused = 0, attn_merge = 0,
-      down_m256 = 0;
+      down_m256 = 0, gu_m128 = 0, gu_cap = 0, dn_cap = 0;
 };
 inline Tune read_tune() {
   Tune t;
@@ -155,6 +157,9 @@ inline Tune read_tune() {
       else if (k == "qkv_fused") t.qkv_fused = v;
       else if (k == "attn_merge") t.attn_merge = v;
       else if (k == "down_m256") t.down_m256 = v;
+      else if (k == "gu_m128") t.gu_m128 = v;
+      else if (k == "gu_cap") t.gu_cap = v;
+      else if (k == "dn_cap") t.dn_cap = v;
     }
     pos = end + 1;
   }
@@ -727,11 +732,14 @@ dg_status run_moe(dg_model* m, int l, int lt, int Tn, int b0, int n_per, bool ca
   // bf16 gate|up runs 256-row tiles (two accumulators per CTA share each B
   // tile; its long K amortises the unoverlapped epilogue); down keeps
   // 128-row tiles with double-buffered accumulators (K = ff is short)
-  plan.mt[0] = cdiv(2 * m->ff, m->bf ? 256 : 128); plan.kb[0] = cdiv(d, 64);
+  const bool gu256 = m->bf && m->tune.gu_m128 != 1;
+  plan.mt[0] = cdiv(2 * m->ff, gu256 ? 256 : 128); plan.kb[0] = cdiv(d, 64);
   const bool down256 = m->bf && !m->fp8 && m->tune.down_m256 == 1;
   plan.mt[1] = cdiv(d, down256 ? 256 : 128); plan.kb[1] = cdiv(m->ff, 64);
   plan.cap[0] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / gu_stride)) : 1;
   plan.cap[1] = m->bf ? (int)std::min<long long>(8, (long long)(m->ws_elems / dn_stride)) : 1;
+  if (m->tune.gu_cap > 0) plan.cap[0] = std::max(1, std::min(plan.cap[0], m->tune.gu_cap));
+  if (m->tune.dn_cap > 0) plan.cap[1] = std::max(1, std::min(plan.cap[1], m->tune.dn_cap));
   plan.fused0 = m->bf ? 1 : 0;
   if (m->fp8) {
     // FP8 experts: 128-row tiles, split-K over 128-input chunks, SwiGLU as
@@ -786,7 +794,7 @@ dg_status run_moe(dg_model* m, int l, int lt, int Tn, int b0, int n_per, bool ca
   gu.max_rows_dev = m->bf ? m->moe_splits + 2 : nullptr;
   gu.splits = m->bf ? 8 : 1;
   // bf16: an unsplit gate|up GEMM applies SwiGLU in its epilogue
-  if (m->bf && !m->fp8) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = true; }
+  if (m->bf && !m->fp8) { gu.act = m->act; gu.act_ld = m->ff; gu.m256 = gu256; }
   if (m->fp8) DG_TRY(gemm_f8(m, gu, &w.tm_gu8, w.gu_s, (long long)m->E * 2 * m->ff, PH_GU_GEMM, s));
   else DG_TRY(gemm(m, gu, PH_GU_GEMM, s));
   // sums the split-K partials and applies SwiGLU; nothing to do when the
