@@ -131,10 +131,11 @@ struct LayerW {
 // combine kernel, 2 always inside the kernel when the splits fit a cluster;
 // down_m256 = 1 runs the down GEMM on 256-row tiles; gu_m128 = 1 runs the
 // gate|up GEMM on 128-row tiles; gu_cap / dn_cap > 0 cap the split-K factor
-// the device may pick for the gate|up / down GEMM).
+// the device may pick for the gate|up / down GEMM; gather_sep = 1 keeps the
+// permute and the row gather as two kernels).
 struct Tune {
   int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0, qkv_fused = 0, attn_merge = 0,
-      down_m256 = 0, gu_m128 = 0, gu_cap = 0, dn_cap = 0;
+      down_m256 = 0, gu_m128 = 0, gu_cap = 0, dn_cap = 0, gather_sep = 0;
 };
 inline Tune read_tune() {
   Tune t;
@@ -160,6 +161,7 @@ inline Tune read_tune() {
       else if (k == "gu_m128") t.gu_m128 = v;
       else if (k == "gu_cap") t.gu_cap = v;
       else if (k == "dn_cap") t.dn_cap = v;
+      else if (k == "gather_sep") t.gather_sep = v;
     }
     pos = end + 1;
   }
@@ -707,6 +709,13 @@ dg_status launch_attn_tc(const AttnPlan& ap, const AttnMaps& am, const AttnArgs&
   return DG_OK;
 }
 
+// Shared memory cap of the fused permute + gather kernel (each CTA holds the
+// whole permutation); larger pair counts take the two-kernel path.
+constexpr size_t kPermuteGatherSmem = 96 * 1024;
+bool permute_gather_fused(const dg_model* m, int n_pairs) {
+  return m->tune.gather_sep != 1 && permute_smem(m->E) + (size_t)n_pairs * sizeof(int) <= kPermuteGatherSmem;
+}
+
 // The MoE half of layer l over Tn tokens: router and top-k on m->x (RMSNorm
 // of the residual state m->h), permutation, expert gate|up GEMM, SwiGLU,
 // down GEMM, and the weighted combine into m->h with RMSNorm of the result
@@ -781,10 +790,23 @@ dg_status run_moe(dg_model* m, int l, int lt, int Tn, int b0, int n_per, bool ca
     launch_pdl(k_router_topk, cdiv(Tn, 8), 256, (size_t)8 * m->E * sizeof(float), s, 
         m->ws, std::min(rc.splits, cdiv(d, 64)), rc.split_stride, m->rbias, tb, m->E, m->k, Tn, m->ids, m->gate); }
   }
-  { LaunchScope ls(m, s, PH_PERMUTE);
-    launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, pa); }
-  { LaunchScope ls(m, s, PH_GATHER);
-    launch_pdl(k_gather<T>, n_pairs, 128, 0, s, (const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
+  if (permute_gather_fused(m, n_pairs)) {
+    // one kernel: every CTA sorts the pairs, each copies its share of the rows
+    LaunchScope ls(m, s, PH_PERMUTE);
+    static bool attr = false;
+    if (!attr) {
+      CU_TRY(cudaFuncSetAttribute(k_permute_gather<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kPermuteGatherSmem));
+      attr = true;
+    }
+    launch_pdl(k_permute_gather<T>, std::min(kSMs, cdiv(n_pairs, 8)), permute_threads(m->E),
+               permute_smem(m->E) + (size_t)n_pairs * sizeof(int), s, pa, (const T*)m->x, m->k, d, (T*)m->xp);
+  } else {
+    { LaunchScope ls(m, s, PH_PERMUTE);
+      launch_pdl(k_permute, 1, permute_threads(m->E), permute_smem(m->E), s, pa); }
+    { LaunchScope ls(m, s, PH_GATHER);
+      launch_pdl(k_gather<T>, n_pairs, 128, 0, s, (const T*)m->x, m->perm, m->k, d, (T*)m->xp); }
+  }
   GemmCall gu;
   gu.tA = &w.tm_gu; gu.tB = &m->tm_xp; gu.A32 = (const float*)w.gu; gu.B32 = (const float*)m->xp;
   gu.lda = d; gu.ldb = d; gu.M = 2 * m->ff; gu.K = d; gu.out = m->ws; gu.ldo = 2 * m->ff;
@@ -1354,14 +1376,16 @@ size_t dg_kv_bytes(const dg_model* m, int32_t B, int32_t P) {
 
 int32_t dg_kernels_per_step(const dg_model* m, int32_t B, int32_t P) {
   if (!m) return 0;
-  (void)B; (void)P;
+  (void)P;
   // per layer: qkv gemm (with the RoPE / cache scatter when fused; else +
   // qkv post), attention (+ combine unless the splits merge in the kernel),
   // o gemm, residual+norm, router (bf16: one kernel; fp32: gemm + top-k),
-  // permute, gather, gate/up gemm, swiglu, down gemm, combine+norm; then
+  // permute and gather (one kernel when the permutation fits shared memory),
+  // gate/up gemm, swiglu, down gemm, combine+norm; then
   // embed+norm, lm head, sampler, commit, 4 self-cond.  The attention merge
   // is decided per shape, so this is the count with the combine kernel.
-  const int per_layer = (m->bf ? 12 : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0);
+  const int per_layer = (m->bf ? 12 : 14) + ((m->bf && m->tune.qkv_fused != 1) ? 1 : 0) -
+                        (permute_gather_fused(m, std::max(1, B) * kCanvas * m->k) ? 1 : 0);
   return per_layer * m->L + 1 /*set round*/ + 1 /*embed*/ + 1 /*lm head*/ + 1 /*sampler*/ + 1 /*commit*/ +
          (m->c.sample_topk > 0 ? 3 : 4) /*self-conditioning*/;
 }

@@ -578,8 +578,10 @@ struct PermuteArgs {
 
 // The permute by one CTA (any multiple of 32 threads); psm holds
 // (warps x E + E + 1) ints.  ids are read through L2: they may have been
-// written by other CTAs of the same kernel.
-__device__ void permute_body(const PermuteArgs& a, int* psm) {
+// written by other CTAs of the same kernel.  Only a `writer` CTA stores the
+// results to global memory (perm, inv, work items, counts, split plan);
+// perm_s (shared, n_pairs ints, or null) receives the permutation locally.
+__device__ void permute_body(const PermuteArgs& a, int* psm, bool writer = true, int* perm_s = nullptr) {
   const int* __restrict__ ids = a.ids;
   const int n_pairs = a.n_pairs, E = a.E, bn = a.bn;
   int* __restrict__ perm = a.perm;
@@ -635,19 +637,21 @@ __device__ void permute_body(const PermuteArgs& a, int* psm) {
     const int pi = block_scan_excl(it, wsum, &tot_items);
     if (e < E) {
       const int acc = carry_rows + pr, nw0 = carry_items + pi;
-      if (counts_out) counts_out[e] = c;
       offs[e] = acc;
-      for (int j = 0; j < it; ++j)
-        work[nw0 + j] = make_int4(e, acc + j * bn, min(bn, c - j * bn), acc + j * bn);
-      if (c > 0) { atomicMax(&s_max_rows, min(c, bn)); atomicAdd(&s_touched, 1); }
+      if (writer) {
+        if (counts_out) counts_out[e] = c;
+        for (int j = 0; j < it; ++j)
+          work[nw0 + j] = make_int4(e, acc + j * bn, min(bn, c - j * bn), acc + j * bn);
+        if (c > 0) { atomicMax(&s_max_rows, min(c, bn)); atomicAdd(&s_touched, 1); }
+      }
     }
     carry_rows += tot_rows;
     carry_items += tot_items;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0) offs[E] = carry_rows;
+  if (threadIdx.x == 0 && writer) {
     const int nw = carry_items;
-    offs[E] = carry_rows;
     *a.work_count = nw;
     // running total of distinct experts this layer streamed (measurement)
     if (a.touched_acc) *a.touched_acc += (unsigned long long)s_touched;
@@ -683,8 +687,11 @@ __device__ void permute_body(const PermuteArgs& a, int* psm) {
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
       const int pos = offs[e] + my[e] + __popc(same & lt_mask);
-      perm[pos] = p;
-      inv[p] = pos;
+      if (writer) {
+        perm[pos] = p;
+        inv[p] = pos;
+      }
+      if (perm_s) perm_s[pos] = p;
     }
     __syncwarp();
     if (e >= 0 && (same & lt_mask) == 0) my[e] += __popc(same);
@@ -696,6 +703,34 @@ __global__ void k_permute(PermuteArgs a) {
   pdl_enter();
   extern __shared__ int psm[];
   permute_body(a, psm);
+}
+
+// Permute and gather in one kernel: every CTA sorts all (token, slot) pairs in
+// shared memory (the same stable counting sort), CTA 0 publishes the
+// permutation, work items and split plan, and each CTA copies its share of
+// the expert-ordered rows xp[pos] = x[perm[pos] / k].  Dynamic shared memory:
+// permute_smem(E) + n_pairs ints.
+template <typename T>
+__global__ void __launch_bounds__(1024) k_permute_gather(PermuteArgs a, const T* __restrict__ x, int k, int d,
+                                                         T* __restrict__ xp) {
+  pdl_enter();
+  extern __shared__ int psm[];
+  const int nwarps = blockDim.x >> 5;
+  int* perm_s = psm + nwarps * a.E + a.E + 1;
+  // positions of pairs with an invalid expert id (reported as an error) stay
+  // unplaced: they copy row 0 rather than an undefined one
+  for (int i = threadIdx.x; i < a.n_pairs; i += blockDim.x) perm_s[i] = 0;
+  permute_body(a, psm, blockIdx.x == 0, perm_s);
+  __syncthreads();
+  const int per = (a.n_pairs + gridDim.x - 1) / gridDim.x;
+  const int p0 = min(a.n_pairs, (int)blockIdx.x * per), p1 = min(a.n_pairs, p0 + per);
+  const int nv = d * (int)sizeof(T) / 16;
+  const long long n = (long long)(p1 - p0) * nv;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+    const int pos = p0 + (int)(i / nv), c = (int)(i % nv);
+    const long long src = perm_s[pos] / k;
+    reinterpret_cast<uint4*>(xp + (long long)pos * d)[c] = reinterpret_cast<const uint4*>(x + src * d)[c];
+  }
 }
 
 // Threads of the permute kernel: whole warps, with the per-warp histograms
