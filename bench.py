@@ -348,7 +348,9 @@ def run_ours(a):
                           "bytes": b_round, "flops": f_round,
                           "touched_experts_mean_over_timed_rounds": [round(t, 2) for t in touched]},
         "roofline": {"bound": "hbm", "kernel": "expert_gate_up_gemm", "achieved": achieved, "peak": hbm,
-                     "unit": "GB/s", "frac": achieved / hbm, "traffic": measured_traffic(gu_bytes),
+                     "unit": "GB/s", "frac": achieved / hbm,
+                     # the committed capture is of the bf16 expert GEMM: no ratio for the FP8 kernel
+                     "traffic": None if getattr(w, "expert_fp8", False) else measured_traffic(gu_bytes),
                      "peak_source": src, "avg_launch_ms": gu_avg, "algorithmic_bytes": gu_bytes},
         "phases_ms_per_round": {k: v[0] / a.profile_reps for k, v in prof.items() if v[1]},
         "e2e": {"value": e_rounds / (e2e_ms * 1e-3), "unit": "denoise steps/s",
