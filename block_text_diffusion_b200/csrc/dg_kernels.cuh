@@ -1070,11 +1070,48 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
   const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab) + g0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
 
-  // pass 1: row max / argmax and the slice's K best
-  if (threadIdx.x == 0) { s_cnt = 0; s_have = 0; s_tau = -INFINITY; }
-  __syncthreads();
+  // pass 1: row max / argmax and the slice's K best.  First each thread's
+  // maximum: the K-th largest of those maxima (K <= blockDim.x) is a floor
+  // with at least K values of the slice at or above it, so every value of the
+  // slice's K best -- ties included -- is at or above it.  The values at or
+  // above the floor are then collected and sorted once.  Should they overflow
+  // the buffer (flat rows), the threshold loop below finds the K best instead.
   ArgBest bm{-INFINITY, -1};
-  for (int base = 0; base < n4; base += blockDim.x) {
+  {
+    float tmax = -INFINITY;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      const float4 l = l4[i];
+      const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bm = arg_better(bm, ArgBest{lv[j], (g0 + i) * 4 + j});
+        tmax = fmaxf(tmax, lv[j]);
+      }
+    }
+    cv[threadIdx.x] = tmax;
+    ci[threadIdx.x] = threadIdx.x;
+    if (threadIdx.x == 0) s_cnt = 0;
+    __syncthreads();
+    cand_sort(cv, ci, blockDim.x);
+    const float floor_k = cv[K - 1];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      const float4 l = l4[i];
+      const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (lv[j] >= floor_k) {
+          const int slot = atomicAdd(&s_cnt, 1);
+          if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = (g0 + i) * 4 + j; }
+        }
+    }
+    __syncthreads();
+  }
+  const bool bounded = s_cnt <= kCandCap;
+  __syncthreads();
+  if (threadIdx.x == 0) { s_cnt = bounded ? s_cnt : 0; s_have = 0; s_tau = -INFINITY; }
+  __syncthreads();
+  for (int base = 0; !bounded && base < n4; base += blockDim.x) {
     const int cnt = s_cnt;
     __syncthreads();                       // every thread has read cnt before any append
     if (cnt + 4 * (int)blockDim.x > kCandCap) {
@@ -1095,7 +1132,6 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int v = (g0 + i) * 4 + j;
-        bm = arg_better(bm, ArgBest{lv[j], v});
         if (!have || lv[j] > tau) {
           const int slot = atomicAdd(&s_cnt, 1);
           if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = v; }
