@@ -851,6 +851,8 @@ constexpr int kSampThreads = 256;
 struct SampPart {
   ArgBest m, g;
   long long s, u;
+  float fl;   // top-k: this slice's candidate floor
+  int cnt;    // top-k: this slice's buffered candidates
 };
 
 template <typename T>
@@ -1070,12 +1072,17 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
   const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab) + g0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
 
-  // pass 1: row max / argmax and the slice's K best.  First each thread's
+  // pass 1: row max / argmax and the row's K best.  First each thread's
   // maximum: the K-th largest of those maxima (K <= blockDim.x) is a floor
-  // with at least K values of the slice at or above it, so every value of the
-  // slice's K best -- ties included -- is at or above it.  The values at or
-  // above the floor are then collected and sorted once.  Should they overflow
-  // the buffer (flat rows), the threshold loop below finds the K best instead.
+  // with at least K values of the slice at or above it, and the largest of
+  // the cluster's floors F has at least K values of the row at or above it,
+  // so every value of the row's K best -- ties included -- is at or above F.
+  // Each CTA buffers its values >= F.  When the cluster's buffers together
+  // fit one buffer, rank 0 gathers them and sorts once; otherwise every CTA
+  // sorts its own down to its K best (by the threshold loop below when even
+  // its own values >= F overflow, as on flat rows) and rank 0 merges the
+  // lists.  Both ways the K best come out in the same order (value
+  // descending, index ascending).
   ArgBest bm{-INFINITY, -1};
   {
     float tmax = -INFINITY;
@@ -1090,92 +1097,123 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
     }
     cv[threadIdx.x] = tmax;
     ci[threadIdx.x] = threadIdx.x;
-    if (threadIdx.x == 0) s_cnt = 0;
     __syncthreads();
     cand_sort(cv, ci, blockDim.x);
-    const float floor_k = cv[K - 1];
-    __syncthreads();
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-      const float4 l = l4[i];
-      const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (lv[j] >= floor_k) {
-          const int slot = atomicAdd(&s_cnt, 1);
-          if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = (g0 + i) * 4 + j; }
-        }
-    }
-    __syncthreads();
   }
-  const bool bounded = s_cnt <= kCandCap;
-  __syncthreads();
-  if (threadIdx.x == 0) { s_cnt = bounded ? s_cnt : 0; s_have = 0; s_tau = -INFINITY; }
-  __syncthreads();
-  for (int base = 0; !bounded && base < n4; base += blockDim.x) {
-    const int cnt = s_cnt;
-    __syncthreads();                       // every thread has read cnt before any append
-    if (cnt + 4 * (int)blockDim.x > kCandCap) {
-      cand_sort(cv, ci, cnt);
-      if (threadIdx.x == 0) {
-        s_cnt = min(cnt, K);
-        s_have = cnt >= K;
-        s_tau = cnt >= K ? cv[K - 1] : -INFINITY;
-      }
-      __syncthreads();
-    }
-    const bool have = s_have != 0;
-    const float tau = s_tau;
-    const int i = base + (int)threadIdx.x;
-    if (i < n4) {
-      const float4 l = l4[i];
-      const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int v = (g0 + i) * 4 + j;
-        if (!have || lv[j] > tau) {
-          const int slot = atomicAdd(&s_cnt, 1);
-          if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = v; }
-        }
-      }
-    }
-    __syncthreads();
-  }
-  {
-    const int cnt = min(s_cnt, kCandCap);
-    __syncthreads();
-    cand_sort(cv, ci, cnt);
-    if (threadIdx.x == 0) s_cnt = min(cnt, K);
-  }
+  const float floor_loc = cv[K - 1];
   bm = warp_argmax(bm);
   if (lane == 0) red_m[warp] = bm;
   __syncthreads();
   if (warp == 0) {
     ArgBest x = lane < nw ? red_m[lane] : ArgBest{-INFINITY, -1};
     x = warp_argmax(x);
-    if (lane == 0) part.m = x;
+    if (lane == 0) { part.m = x; part.fl = floor_loc; s_cnt = 0; }
   }
   cluster_sync_all();
   ArgBest M{-INFINITY, -1};
+  float F = -INFINITY;
   for (int r = 0; r < kSampCta; ++r) {
     const SampPart* pr = cluster_peer(&part, r);
     M = arg_better(M, ArgBest{pr->m.v, pr->m.i});
+    F = fmaxf(F, pr->fl);
   }
   const float m = M.v;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 l = l4[i];
+    const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (lv[j] >= F) {
+        const int slot = atomicAdd(&s_cnt, 1);
+        if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = (g0 + i) * 4 + j; }
+      }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) part.cnt = s_cnt;
+  cluster_sync_all();
+  int total = 0;
+  bool fits = true;
+  for (int r = 0; r < kSampCta; ++r) {
+    const int c = cluster_peer(&part, r)->cnt;
+    total += c;
+    fits = fits && c <= kCandCap;
+  }
+  const bool one_sort = fits && total <= kCandCap;   // the same outcome in every CTA of the cluster
+  if (!one_sort) {
+    const bool bounded = s_cnt <= kCandCap;
+    __syncthreads();
+    if (threadIdx.x == 0) { s_cnt = bounded ? s_cnt : 0; s_have = 0; s_tau = -INFINITY; }
+    __syncthreads();
+    for (int base = 0; !bounded && base < n4; base += blockDim.x) {
+      const int cnt = s_cnt;
+      __syncthreads();                       // every thread has read cnt before any append
+      if (cnt + 4 * (int)blockDim.x > kCandCap) {
+        cand_sort(cv, ci, cnt);
+        if (threadIdx.x == 0) {
+          s_cnt = min(cnt, K);
+          s_have = cnt >= K;
+          s_tau = cnt >= K ? cv[K - 1] : -INFINITY;
+        }
+        __syncthreads();
+      }
+      const bool have = s_have != 0;
+      const float tau = s_tau;
+      const int i = base + (int)threadIdx.x;
+      if (i < n4) {
+        const float4 l = l4[i];
+        const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int v = (g0 + i) * 4 + j;
+          if (!have || lv[j] > tau) {
+            const int slot = atomicAdd(&s_cnt, 1);
+            if (slot < kCandCap) { cv[slot] = lv[j]; ci[slot] = v; }
+          }
+        }
+      }
+      __syncthreads();
+    }
+    {
+      const int cnt = min(s_cnt, kCandCap);
+      __syncthreads();
+      cand_sort(cv, ci, cnt);
+      if (threadIdx.x == 0) s_cnt = min(cnt, K);
+    }
+    cluster_sync_all();                      // every list is final before rank 0 reads it
+  }
 
   if (rank == 0) {
-    // merge the clusters' lists: rank r's K best go to [r K, (r+1) K)
-    for (int r = 1; r < kSampCta; ++r) {
-      const float* pv = cluster_peer(cv, r);
-      const int* pi = cluster_peer(ci, r);
-      const int pc = *cluster_peer(&s_cnt, r);
-      for (int j = threadIdx.x; j < K; j += blockDim.x) {
-        cv[r * K + j] = j < pc ? pv[j] : -INFINITY;
-        ci[r * K + j] = j < pc ? pi[j] : 0x7fffffff;
+    if (one_sort) {
+      // every CTA's candidates after rank 0's own, then one sort
+      int off = s_cnt;
+      for (int r = 1; r < kSampCta; ++r) {
+        const float* pv = cluster_peer(cv, r);
+        const int* pi = cluster_peer(ci, r);
+        const int pc = cluster_peer(&part, r)->cnt;
+        for (int j = threadIdx.x; j < pc; j += blockDim.x) {
+          cv[off + j] = pv[j];
+          ci[off + j] = pi[j];
+        }
+        off += pc;
       }
+      for (int j = total + (int)threadIdx.x; j < K; j += blockDim.x) { cv[j] = -INFINITY; ci[j] = 0x7fffffff; }
+      __syncthreads();
+      cand_sort(cv, ci, max(total, K));
+    } else {
+      // merge the lists: rank r's K best go to [r K, (r+1) K)
+      for (int r = 1; r < kSampCta; ++r) {
+        const float* pv = cluster_peer(cv, r);
+        const int* pi = cluster_peer(ci, r);
+        const int pc = *cluster_peer(&s_cnt, r);
+        for (int j = threadIdx.x; j < K; j += blockDim.x) {
+          cv[r * K + j] = j < pc ? pv[j] : -INFINITY;
+          ci[r * K + j] = j < pc ? pi[j] : 0x7fffffff;
+        }
+      }
+      for (int j = s_cnt + (int)threadIdx.x; j < K; j += blockDim.x) { cv[j] = -INFINITY; ci[j] = 0x7fffffff; }
+      __syncthreads();
+      cand_sort(cv, ci, kSampCta * K);
     }
-    for (int j = s_cnt + (int)threadIdx.x; j < K; j += blockDim.x) { cv[j] = -INFINITY; ci[j] = 0x7fffffff; }
-    __syncthreads();
-    cand_sort(cv, ci, kSampCta * K);
     // Gumbel-max among the candidates; candidate weights
     ArgBest bg{-INFINITY, -1};
     for (int j = threadIdx.x; j < K; j += blockDim.x) {
