@@ -827,8 +827,12 @@ __device__ __forceinline__ ArgBest warp_argmax(ArgBest x) {
   return x;
 }
 
-// Vocab-wide sampler pass.  One cluster of kSampCta CTAs per row; CTA r of
-// the cluster owns the contiguous vocab slice [r V/kSampCta, (r+1) V/kSampCta).
+// Vocab-wide sampler pass.  One cluster of NC CTAs per row (sampler_cluster:
+// 2 up to a 65536-entry vocabulary, else 8); CTA r of the cluster owns the
+// contiguous vocab slice [r V/NC, (r+1) V/NC).  The results do not depend on
+// NC: the sums are exact integers, maxima break ties to the lower index, the
+// Philox counters are vocabulary indices, and the Gumbel filter only skips
+// values that cannot beat the running best of the thread that sees them.
 // Partial results are exchanged through distributed shared memory and every
 // CTA combines them in rank order (integer sums are exact, arg-maxima break
 // ties to the lower index), so all CTAs hold the same row values.
@@ -845,7 +849,10 @@ __device__ __forceinline__ ArgBest warp_argmax(ArgBest x) {
 // memory, so several clusters share an SM.  The arithmetic uses no
 // conversion-unit instructions per element.
 // ---------------------------------------------------------------------------
-constexpr int kSampCta = 8;        // CTAs per row (one thread-block cluster)
+constexpr int kSampCta = 8;        // most CTAs per row (one thread-block cluster)
+// CTAs per row: fewer, longer slices for small vocabularies, where each CTA's
+// fixed work (reductions, cluster barriers) would otherwise dominate.
+inline int sampler_cluster(int vocab) { return vocab <= 65536 ? 2 : kSampCta; }
 constexpr int kSampThreads = 256;
 
 struct SampPart {
@@ -855,8 +862,8 @@ struct SampPart {
   int cnt;    // top-k: this slice's buffered candidates
 };
 
-template <typename T>
-__global__ void __cluster_dims__(kSampCta, 1, 1) __launch_bounds__(kSampThreads)
+template <typename T, int NC>
+__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(kSampThreads)
 k_sampler(SamplerArgs a, T* __restrict__ probs) {
   pdl_enter();
   __shared__ SampPart part;
@@ -864,14 +871,14 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
   __shared__ long long red_s[32], red_u[32];
   uint32_t rank;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
-  const long long row = blockIdx.x / kSampCta;
+  const long long row = blockIdx.x / NC;
   const int canvas = (int)(row / a.positions), pos = (int)(row % a.positions);
   const int step = a.step_override >= 0 ? a.step_override : a.state->step;
   const float t = a.step_override >= 0 ? a.t_override : a.state->t;
   const float temp = __fadd_rn(a.temp_end, __fmul_rn(__fsub_rn(a.temp_start, a.temp_end), t));
   const float inv_t = __fdiv_rn(1.0f, temp);
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32) ^ (uint32_t)canvas;
-  const int n4 = a.vocab / (4 * kSampCta);        // float4 groups in this slice
+  const int n4 = a.vocab / (4 * NC);        // float4 groups in this slice
   const int g0 = (int)rank * n4;                  // first global float4 group
   const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab) + g0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -915,7 +922,7 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
   }
   cluster_sync_all();
   ArgBest M{-INFINITY, -1}, G{-INFINITY, -1};
-  for (int r = 0; r < kSampCta; ++r) {
+  for (int r = 0; r < NC; ++r) {
     const SampPart* pr = cluster_peer(&part, r);
     M = arg_better(M, ArgBest{pr->m.v, pr->m.i});
     G = arg_better(G, ArgBest{pr->g.v, pr->g.i});
@@ -957,7 +964,7 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
   }
   cluster_sync_all();
   long long S = 0, U = 0;
-  for (int r = 0; r < kSampCta; ++r) {
+  for (int r = 0; r < NC; ++r) {
     const SampPart* pr = cluster_peer(&part, r);
     S += pr->s;
     U += pr->u;
@@ -988,8 +995,9 @@ k_sampler(SamplerArgs a, T* __restrict__ probs) {
 template <typename T>
 cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cudaStream_t s, bool pdl) {
   const size_t smem = 0;
+  const int nc = sampler_cluster(sa.vocab);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(rows * kSampCta));
+  cfg.gridDim = dim3((unsigned)(rows * nc));
   cfg.blockDim = dim3(kSampThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -998,7 +1006,8 @@ cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cuda
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_sampler<T>, sa, probs);
+  return nc == 2 ? cudaLaunchKernelEx(&cfg, k_sampler<T, 2>, sa, probs)
+                 : cudaLaunchKernelEx(&cfg, k_sampler<T, kSampCta>, sa, probs);
 }
 
 // ---------------------------------------------------------------------------
@@ -1011,13 +1020,13 @@ cudaError_t launch_sampler(const SamplerArgs& sa, T* probs, long long rows, cuda
 // ... in candidate order, feed self-conditioning.  Entropy, row argmax and
 // the Q40 sums are those of the full row, as in k_sampler.
 //
-// Same cluster layout as k_sampler (kSampCta CTAs per row).  Pass 1 keeps
+// Same cluster layout as k_sampler (NC CTAs per row).  Pass 1 keeps
 // the slice's K best in a shared candidate buffer: every value above the
 // current threshold (the K-th best so far) is appended; when the next
 // iteration could overflow the buffer it is sorted and cut back to K.
 // Iterations visit increasing indices, so a later value equal to the
 // threshold can never displace a kept one and a strict comparison suffices.
-// Rank 0 merges the kSampCta lists through distributed shared memory and
+// Rank 0 merges the NC lists through distributed shared memory and
 // draws among the row's K candidates: Philox runs on K values per row, not V.
 // ---------------------------------------------------------------------------
 constexpr int kTopkMax = 256;      // largest supported truncation K
@@ -1046,8 +1055,8 @@ __device__ __forceinline__ void cand_sort(float* cv, int* ci, int n) {
     }
 }
 
-template <typename T>
-__global__ void __cluster_dims__(kSampCta, 1, 1) __launch_bounds__(kSampThreads)
+template <typename T, int NC>
+__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(kSampThreads)
 k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__ cand_w) {
   pdl_enter();
   __shared__ SampPart part;
@@ -1060,14 +1069,14 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
   __shared__ float s_tau, s_inv;
   uint32_t rank;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
-  const long long row = blockIdx.x / kSampCta;
+  const long long row = blockIdx.x / NC;
   const int canvas = (int)(row / a.positions), pos = (int)(row % a.positions);
   const int step = a.step_override >= 0 ? a.step_override : a.state->step;
   const float t = a.step_override >= 0 ? a.t_override : a.state->t;
   const float temp = __fadd_rn(a.temp_end, __fmul_rn(__fsub_rn(a.temp_start, a.temp_end), t));
   const float inv_t = __fdiv_rn(1.0f, temp);
   const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32) ^ (uint32_t)canvas;
-  const int n4 = a.vocab / (4 * kSampCta);
+  const int n4 = a.vocab / (4 * NC);
   const int g0 = (int)rank * n4;
   const float4* l4 = reinterpret_cast<const float4*>(a.logits + row * a.vocab) + g0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -1112,7 +1121,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
   cluster_sync_all();
   ArgBest M{-INFINITY, -1};
   float F = -INFINITY;
-  for (int r = 0; r < kSampCta; ++r) {
+  for (int r = 0; r < NC; ++r) {
     const SampPart* pr = cluster_peer(&part, r);
     M = arg_better(M, ArgBest{pr->m.v, pr->m.i});
     F = fmaxf(F, pr->fl);
@@ -1133,7 +1142,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
   cluster_sync_all();
   int total = 0;
   bool fits = true;
-  for (int r = 0; r < kSampCta; ++r) {
+  for (int r = 0; r < NC; ++r) {
     const int c = cluster_peer(&part, r)->cnt;
     total += c;
     fits = fits && c <= kCandCap;
@@ -1186,7 +1195,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
     if (one_sort) {
       // every CTA's candidates after rank 0's own, then one sort
       int off = s_cnt;
-      for (int r = 1; r < kSampCta; ++r) {
+      for (int r = 1; r < NC; ++r) {
         const float* pv = cluster_peer(cv, r);
         const int* pi = cluster_peer(ci, r);
         const int pc = cluster_peer(&part, r)->cnt;
@@ -1201,7 +1210,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
       cand_sort(cv, ci, max(total, K));
     } else {
       // merge the lists: rank r's K best go to [r K, (r+1) K)
-      for (int r = 1; r < kSampCta; ++r) {
+      for (int r = 1; r < NC; ++r) {
         const float* pv = cluster_peer(cv, r);
         const int* pi = cluster_peer(ci, r);
         const int pc = *cluster_peer(&s_cnt, r);
@@ -1212,7 +1221,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
       }
       for (int j = s_cnt + (int)threadIdx.x; j < K; j += blockDim.x) { cv[j] = -INFINITY; ci[j] = 0x7fffffff; }
       __syncthreads();
-      cand_sort(cv, ci, kSampCta * K);
+      cand_sort(cv, ci, NC * K);
     }
     // Gumbel-max among the candidates; candidate weights
     ArgBest bg{-INFINITY, -1};
@@ -1275,7 +1284,7 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
   }
   cluster_sync_all();
   long long S = 0, U = 0;
-  for (int r = 0; r < kSampCta; ++r) {
+  for (int r = 0; r < NC; ++r) {
     const SampPart* pr = cluster_peer(&part, r);
     S += pr->s;
     U += pr->u;
@@ -1293,8 +1302,9 @@ k_sampler_topk(SamplerArgs a, int K, int* __restrict__ cand_ids, T* __restrict__
 template <typename T>
 cudaError_t launch_sampler_topk(const SamplerArgs& sa, int K, int* cand_ids, T* cand_w, long long rows,
                                 cudaStream_t s, bool pdl) {
+  const int nc = sampler_cluster(sa.vocab);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(rows * kSampCta));
+  cfg.gridDim = dim3((unsigned)(rows * nc));
   cfg.blockDim = dim3(kSampThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -1303,7 +1313,8 @@ cudaError_t launch_sampler_topk(const SamplerArgs& sa, int K, int* cand_ids, T* 
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_sampler_topk<T>, sa, K, cand_ids, cand_w);
+  return nc == 2 ? cudaLaunchKernelEx(&cfg, k_sampler_topk<T, 2>, sa, K, cand_ids, cand_w)
+                 : cudaLaunchKernelEx(&cfg, k_sampler_topk<T, kSampCta>, sa, K, cand_ids, cand_w);
 }
 
 // Self-conditioning input of a truncated distribution: u[t] = sum_j w[t][j]
