@@ -132,10 +132,11 @@ struct LayerW {
 // down_m256 = 1 runs the down GEMM on 256-row tiles; gu_m128 = 1 runs the
 // gate|up GEMM on 128-row tiles; gu_cap / dn_cap > 0 cap the split-K factor
 // the device may pick for the gate|up / down GEMM; gather_sep = 1 keeps the
-// permute and the row gather as two kernels).
+// permute and the row gather as two kernels; samp_nc = 1, 2, 4 or 8 sets the
+// sampler's CTAs per row).
 struct Tune {
   int dense_bn = 0, dense_splits = 0, router_bn = 0, router_splits = 0, qkv_fused = 0, attn_merge = 0,
-      down_m256 = 0, gu_m128 = 0, gu_cap = 0, dn_cap = 0, gather_sep = 0;
+      down_m256 = 0, gu_m128 = 0, gu_cap = 0, dn_cap = 0, gather_sep = 0, samp_nc = 0;
 };
 inline Tune read_tune() {
   Tune t;
@@ -162,6 +163,7 @@ inline Tune read_tune() {
       else if (k == "gu_cap") t.gu_cap = v;
       else if (k == "dn_cap") t.dn_cap = v;
       else if (k == "gather_sep") t.gather_sep = v;
+      else if (k == "samp_nc") t.samp_nc = v;
     }
     pos = end + 1;
   }
@@ -1007,9 +1009,10 @@ dg_status run_round(dg_model* m, const KvGeom& g, const RoundIO& io, cudaStream_
     sa.step_override = io.step_override; sa.t_override = io.t_override;
     sa.H = io.entropy; sa.tok = io.tokens; sa.amax = io.argmax;
     if (m->c.sample_topk > 0)
-      CU_TRY(launch_sampler_topk<T>(sa, m->c.sample_topk, m->cand_ids, (T*)m->cand_w, Tn, s, g_use_pdl));
+      CU_TRY(launch_sampler_topk<T>(sa, m->c.sample_topk, m->cand_ids, (T*)m->cand_w, Tn, s, g_use_pdl,
+                                    m->tune.samp_nc));
     else
-      CU_TRY(launch_sampler<T>(sa, io.selfcond_next ? (T*)m->probs : nullptr, Tn, s, g_use_pdl));
+      CU_TRY(launch_sampler<T>(sa, io.selfcond_next ? (T*)m->probs : nullptr, Tn, s, g_use_pdl, m->tune.samp_nc));
   }
   // commit / re-noise / stop
   {
