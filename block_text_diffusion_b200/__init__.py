@@ -90,6 +90,7 @@ def lib():
             "dg_test_layer": ([P, P, I32, I32, I32, P, P, P, P], I32),
             "dg_test_moe": ([P, I32, I32, P, P, P, P], I32),
             "dg_test_attn_capacity": ([P], I32),
+            "dg_test_launch_shape": ([I32, I64, I32, I32, P], I32),
             "dg_touched_experts_sum": ([P, P, I32, P], I32),
             "dg_gemm_splitk_noalloc": ([P, P, P, I32, I32, I32, I32, P], I32),
         }

@@ -118,6 +118,17 @@ dg_status dg_test_grouped_gemm(const void* A, const void* B, const int32_t* coun
  * queries per canvas, G query heads per KV head, n_keys keys, rows = query
  * rows of the launch and part_rows_cap = rows the partial-output buffer
  * holds per split sum (binding only when the splits merge through it). */
+/* Launch choices of the step that depend only on the shape (host only, no
+ * device call).  out int32[2]: out[0] = CTAs per row of the vocab samplers
+ * for a vocabulary of `vocab` entries and `rows` logit rows (one
+ * thread-block cluster per row: 8 above 65536 entries; else 1 when the rows
+ * alone give every SM four CTAs, 2 otherwise); out[1] = 1 when the permute
+ * and the expert-row gather run as one kernel for `n_pairs` (token, slot)
+ * pairs over `n_experts` experts (the permutation fits 96 KB of shared
+ * memory), else 0.  DG_ERR_INVALID_ARG for a null out or non-positive
+ * sizes. */
+dg_status dg_test_launch_shape(int32_t vocab, int64_t rows, int32_t n_experts, int32_t n_pairs, int32_t* out);
+
 /* Thread-block clusters of the bf16 attention kernel that the device can
  * hold at once, per cluster size (the capacity the split-KV plan is given):
  * out int32[9], out[c] for c = 1..8, out[0] = 0; 0 where the device refuses

@@ -122,3 +122,43 @@ def test_noalloc_binding_rejects_non_contiguous_operands():
     out = torch.zeros((32, 256), dtype=torch.float32)
     with pytest.raises(ValueError):
         dg.gemm_splitk_noalloc(A, B, out)
+
+
+def launch_shape(lib, vocab, rows, n_experts, n_pairs):
+    out = (ctypes.c_int32 * 2)()
+    assert lib.dg_test_launch_shape(vocab, rows, n_experts, n_pairs, out) == 0
+    return list(out)
+
+
+@pytest.mark.parametrize("vocab,rows,want", [
+    (262144, 256, 8),            # 26B vocabulary: 8 CTAs per row at every batch
+    (262144, 8192, 8),
+    (32768, 256, 2),             # one canvas: too few rows to give every SM four CTAs alone
+    (32768, 1024, 1),            # four canvases and more: one CTA per row
+    (32768, 8192, 1),
+    (1024, 256, 2),
+    (65536, 4 * SMS, 1),         # the boundaries
+    (65536, 4 * SMS - 1, 2),
+    (65600, 4 * SMS, 8),
+])
+def test_sampler_cluster_size_rule(lib, vocab, rows, want):
+    assert launch_shape(lib, vocab, rows, 128, 2048)[0] == want
+
+
+def test_permute_and_gather_fuse_while_the_permutation_fits_shared_memory(lib):
+    # 1024 threads: 32 warp histograms of E ints, the offsets, then one int per pair
+    def fits(E, n_pairs):
+        return (32 * E + E + 1) * 4 + n_pairs * 4 <= 96 * 1024
+    for E, k in ((128, 8), (32, 4), (8, 2)):
+        for B in (1, 4, 8, 9, 10, 16, 22, 23, 32):
+            n = B * 256 * k
+            assert launch_shape(lib, 32768, 256, E, n)[1] == int(fits(E, n)), (E, k, B)
+    assert launch_shape(lib, 32768, 256, 128, 9 * 256 * 8)[1] == 1    # 26B shape: up to 9 canvases
+    assert launch_shape(lib, 32768, 256, 128, 10 * 256 * 8)[1] == 0
+
+
+def test_launch_shape_rejects_bad_sizes(lib):
+    out = (ctypes.c_int32 * 2)()
+    assert lib.dg_test_launch_shape(0, 256, 128, 2048, out) != 0
+    assert lib.dg_test_launch_shape(32768, 256, 128, 0, out) != 0
+    assert lib.dg_test_launch_shape(32768, 256, 128, 2048, None) != 0
