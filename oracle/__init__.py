@@ -15,8 +15,13 @@ Modules:
   model    -- weights, causal prompt encode, one denoising step, block loop
 
 Parity status: every building block is pinned by tests/test_oracle_*.py
-against closed forms, brute force or published test vectors.  The composed
-model (forward_canvas / denoise_step / generate_block) is "parity unpinned"
-beyond those invariants: the pages print no numeric worked example.
+against closed forms, brute force or published test vectors, and the
+composed model (prompt encode, canvas forward, denoising step, block loop)
+against an element-by-element brute-force evaluation on a micro
+configuration and against the method's invariants.  The pages print no
+numeric worked example; what stays unpinned is only the bf16
+double-rounding behaviour of the composed model at sizes beyond the micro
+brute force (the bf16 storage points themselves are pinned by unit tests of
+`store`).
 """
 from . import numerics, sampler, model  # noqa: F401
