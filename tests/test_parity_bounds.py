@@ -18,7 +18,12 @@ accumulation flips), and h after attention one step off in 30% of its
 elements (an rms deviation just under 2^-8).  The routing is held fixed
 (near-ties are checked separately by the GPU test).  Shape: the 26B-A4B
 stand-in (d 2816, 704-wide experts, top-8 of a 16-expert pool), where the
-MoE output is largest relative to the residual."""
+MoE output is largest relative to the residual.
+
+And the other direction, on one layer of the mid model: plausible mistakes
+planted in the oracle (an expert slot dropped from the gated sum, RoPE one
+position off, the attention residual missing) move the compared tensor past
+both its step bound and its rms bound, so the bounds still bite."""
 import numpy as np
 import pytest
 
@@ -109,3 +114,47 @@ def test_whole_layer_bound_covers_the_allowed_deviation_after_attention(moe26b):
     assert e.max() > 3 or rel_rms(got, ref) > REL_RMS
     # the MoE output is larger than the residual it is added to at this shape
     assert np.sqrt(np.mean(y ** 2)) > np.sqrt(np.mean(h ** 2))
+
+
+# --- the bounds bite: plausible mistakes, planted in the oracle, break them ---------
+@pytest.fixture(scope="module")
+def mid_layer():
+    w = I.MID_BF16
+    P = w.prompt_len
+    model = om.Model(w, layers=0, with_embed=False)
+    lw = om.layer_weights(w, 0, lazy_experts=True)
+    Kp, Vp = I.prompt_kv(61, w.n_layers, 1, w.n_kv_heads, P, w.head_dim, bf16=True)
+    kp = Kp[0, 0].transpose(1, 0, 2).astype(np.float64)
+    vp = Vp[0, 0].transpose(1, 0, 2).astype(np.float64)
+    h_in = I.normal(1061, 111, (256, w.d_model), std=0.1, bf16=True).astype(np.float64)
+    tr = []
+    om.block(model, lw, h_in, P + np.arange(256), kp, vp, causal=False, trace=tr)
+    return w, model, lw, h_in, kp, vp, P, tr[0]
+
+
+def over_bound(got, ref, addend, steps, rms):
+    e = bf16_steps(got, ref, addend=addend)
+    return e.max() > steps and rel_rms(got, ref) > rms
+
+
+def test_a_dropped_expert_slot_breaks_the_moe_bound(mid_layer):
+    w, model, lw, h_in, kp, vp, P, t = mid_layer
+    x2 = model.store(om.rmsnorm(t["h_attn"], w.rms_eps))
+    _, ids, gates = om.moe(model, lw, x2)
+    g = gates.copy()
+    g[:, -1] = 0.0                                  # the last slot's expert left out
+    got = model.store(t["h_attn"] + moe_fixed(w, model, lw, x2, ids, g))
+    assert over_bound(got, t["h_out"], t["h_attn"], 3, REL_RMS)
+
+
+def test_rope_one_position_off_breaks_the_attention_bound(mid_layer):
+    w, model, lw, h_in, kp, vp, P, t = mid_layer
+    tr = []
+    om.block(model, lw, h_in, P + 1 + np.arange(256), kp, vp, causal=False, trace=tr)
+    assert over_bound(tr[0]["h_attn"], t["h_attn"], h_in, 2, REL_RMS)
+
+
+def test_a_missing_attention_residual_breaks_the_attention_bound(mid_layer):
+    w, model, lw, h_in, kp, vp, P, t = mid_layer
+    got = model.store(t["h_attn"] - h_in)           # the output projection alone
+    assert over_bound(got, t["h_attn"], h_in, 2, REL_RMS)
